@@ -1,0 +1,257 @@
+"""ctypes marshalling for libflashmask.so (see include/flashmask.h)."""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence, Tuple
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_NAME = "libflashmask.so"
+_lib = None
+
+# Entry points of include/flashmask.h: name -> (restype, argtypes)
+_P = ctypes.c_void_p
+_DIMS = ctypes.c_void_p  # const flashmask_dims*
+_SIGS = {
+    "flashmask_fwd_workspace_size": (ctypes.c_size_t, [_DIMS]),
+    "flashmask_bwd_workspace_size": (ctypes.c_size_t, [_DIMS]),
+    "flashmask_fwd": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, ctypes.c_float, _DIMS, _P, _P, _P,
+                                     ctypes.c_size_t, _P]),
+    "flashmask_bwd": (ctypes.c_int, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_float, _DIMS, _P, _P, _P,
+                                     _P, ctypes.c_size_t, _P]),
+    "flashmask_classify": (ctypes.c_int, [_P, _P, _P, _P, _DIMS, _P, _P, ctypes.c_size_t, _P]),
+    "flashmask_localize": (ctypes.c_int, [_P, _P, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, _P]),
+    "flashmask_localize_multi": (ctypes.c_int, [_P, _P, ctypes.c_int64, _P, _P, ctypes.c_int32, _P]),
+    "flashmask_count_unmasked": (ctypes.c_int, [_P, _P, _P, _P, _DIMS, _P, _P]),
+    "flashmask_get_status": (ctypes.c_int, []),
+    "flashmask_set_wait_limit_ns": (None, [ctypes.c_int64]),
+    "flashmask_test_wait_timeout": (ctypes.c_int, [ctypes.c_int64, _P]),
+    "flashmask_strerror": (ctypes.c_char_p, [ctypes.c_int]),
+    "flashmask_version": (ctypes.c_int, []),
+}
+
+
+class _Dims(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in ("B", "Hq", "Hkv", "Hm", "Nq", "Nk", "d")]
+
+
+class FlashMaskError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        msg = load_library().flashmask_strerror(code).decode()
+        super().__init__(f"{where}: {msg} (code {code})")
+        self.code = code
+
+
+def lib_path() -> str:
+    return os.path.join(_HERE, _LIB_NAME)
+
+
+def load_library():
+    """Loads libflashmask.so from the package directory; raises if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = lib_path()
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with `python column_sparse_masked_b200/build.py`")
+    lib = ctypes.CDLL(path)
+    for name, (res, args) in _SIGS.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def version() -> int:
+    return int(load_library().flashmask_version())
+
+
+def _check(code: int, where: str):
+    if code != 0:
+        raise FlashMaskError(code, where)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _dims(B, Hq, Hkv, Hm, Nq, Nk, d) -> _Dims:
+    return _Dims(int(B), int(Hq), int(Hkv), int(Hm), int(Nq), int(Nk), int(d))
+
+
+def _need_cuda(name: str, t: torch.Tensor, dtype=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _masks(lts, lte, uts, ute):
+    vecs = [lts, lte, uts, ute]
+    for n, x in zip(("lts", "lte", "uts", "ute"), vecs):
+        if x is not None:
+            _need_cuda(n, x, torch.int32)
+    ref = next((x for x in vecs if x is not None), None)
+    Hm = ref.shape[1] if ref is not None else 1
+    return vecs, Hm
+
+
+def workspace_size(kind: str, B, Hq, Hkv, Hm, Nq, Nk, d) -> int:
+    lib = load_library()
+    dm = _dims(B, Hq, Hkv, Hm, Nq, Nk, d)
+    fn = lib.flashmask_fwd_workspace_size if kind == "fwd" else lib.flashmask_bwd_workspace_size
+    return int(fn(ctypes.byref(dm)))
+
+
+def _workspace(nbytes: int, device) -> torch.Tensor:
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, lts=None, lte=None, uts=None, ute=None,
+        scale: Optional[float] = None, out: Optional[Tuple[torch.Tensor, torch.Tensor]] = None,
+        workspace: Optional[torch.Tensor] = None):
+    """Masked attention forward -> (o [B,Nq,Hq,d] bf16, lse [B,Hq,Nq] fp32)."""
+    lib = load_library()
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _need_cuda(n, t, torch.bfloat16)
+    B, Nq, Hq, d = q.shape
+    Nk, Hkv = k.shape[1], k.shape[2]
+    vecs, Hm = _masks(lts, lte, uts, ute)
+    dm = _dims(B, Hq, Hkv, Hm, Nq, Nk, d)
+    if out is None:
+        o = torch.empty_like(q)
+        lse = torch.empty(B, Hq, Nq, dtype=torch.float32, device=q.device)
+    else:
+        o, lse = out
+    need = int(lib.flashmask_fwd_workspace_size(ctypes.byref(dm)))
+    ws = workspace if workspace is not None else _workspace(need, q.device)
+    rc = lib.flashmask_fwd(_ptr(q), _ptr(k), _ptr(v), *[_ptr(x) for x in vecs], ctypes.c_float(scale or 0.0),
+                           ctypes.byref(dm), _ptr(o), _ptr(lse), _ptr(ws), ctypes.c_size_t(ws.numel()),
+                           _stream(q.device))
+    _check(rc, "flashmask_fwd")
+    return o, lse
+
+
+def bwd(q, k, v, o, lse, dout, lts=None, lte=None, uts=None, ute=None, scale: Optional[float] = None,
+        out: Optional[Tuple[torch.Tensor, torch.Tensor, torch.Tensor]] = None,
+        workspace: Optional[torch.Tensor] = None):
+    """Masked attention backward of sum(O * dO) -> (dq, dk, dv), bf16."""
+    lib = load_library()
+    for n, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout)):
+        _need_cuda(n, t, torch.bfloat16)
+    _need_cuda("lse", lse, torch.float32)
+    B, Nq, Hq, d = q.shape
+    Nk, Hkv = k.shape[1], k.shape[2]
+    vecs, Hm = _masks(lts, lte, uts, ute)
+    dm = _dims(B, Hq, Hkv, Hm, Nq, Nk, d)
+    if out is None:
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    else:
+        dq, dk, dv = out
+    need = int(lib.flashmask_bwd_workspace_size(ctypes.byref(dm)))
+    ws = workspace if workspace is not None else _workspace(need, q.device)
+    rc = lib.flashmask_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), *[_ptr(x) for x in vecs],
+                           ctypes.c_float(scale or 0.0), ctypes.byref(dm), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws),
+                           ctypes.c_size_t(ws.numel()), _stream(q.device))
+    _check(rc, "flashmask_bwd")
+    return dq, dk, dv
+
+
+def classify(lts, lte, uts, ute, Nq: int, Nk: Optional[int] = None, Hq: int = 1) -> torch.Tensor:
+    """Tile classes uint8 [B, Hm, ceil(Nq/128), ceil(Nk/128)]: 0 skip, 1 partial, 2 full."""
+    lib = load_library()
+    vecs, Hm = _masks(lts, lte, uts, ute)
+    ref = next(x for x in vecs if x is not None)
+    B, Nk = ref.shape[0], (ref.shape[2] if Nk is None else Nk)
+    Hq = max(Hq, Hm)
+    dm = _dims(B, Hq, 1, Hm, Nq, Nk, 128)
+    nqt, nkt = -(-Nq // 128), -(-Nk // 128)
+    cls = torch.empty(B, Hm, nqt, nkt, dtype=torch.uint8, device=ref.device)
+    ws = _workspace(lib.flashmask_fwd_workspace_size(ctypes.byref(dm)), ref.device)
+    rc = lib.flashmask_classify(*[_ptr(x) for x in vecs], ctypes.byref(dm), _ptr(cls), _ptr(ws),
+                                ctypes.c_size_t(ws.numel()), _stream(ref.device))
+    _check(rc, "flashmask_classify")
+    return cls
+
+
+def localize(x: torch.Tensor, a: int, b: int, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Clip-shift-max of boundary values onto the query chunk [a, b)."""
+    lib = load_library()
+    _need_cuda("x", x, torch.int32)
+    out = torch.empty_like(x) if out is None else out
+    rc = lib.flashmask_localize(_ptr(x), _ptr(out), ctypes.c_int64(x.numel()), int(a), int(b), _stream(x.device))
+    _check(rc, "flashmask_localize")
+    return out
+
+
+def localize_multi(x: torch.Tensor, chunks: Sequence[Tuple[int, int]], out: Optional[torch.Tensor] = None):
+    """Localisation onto increasing disjoint chunks concatenated in order."""
+    lib = load_library()
+    _need_cuda("x", x, torch.int32)
+    out = torch.empty_like(x) if out is None else out
+    a = (ctypes.c_int32 * max(1, len(chunks)))(*[int(c[0]) for c in chunks])
+    b = (ctypes.c_int32 * max(1, len(chunks)))(*[int(c[1]) for c in chunks])
+    rc = lib.flashmask_localize_multi(_ptr(x), _ptr(out), ctypes.c_int64(x.numel()), a, b, len(chunks),
+                                      _stream(x.device))
+    _check(rc, "flashmask_localize_multi")
+    return out
+
+
+def count_unmasked(lts, lte, uts, ute, Nq: int, Hq: int) -> int:
+    """Unmasked (i, j) pairs over all batches and Hq query heads (closed form on the GPU)."""
+    lib = load_library()
+    vecs, Hm = _masks(lts, lte, uts, ute)
+    ref = next(x for x in vecs if x is not None)
+    B, Nk = ref.shape[0], ref.shape[2]
+    dm = _dims(B, Hq, 1, Hm, Nq, Nk, 128)
+    out = torch.zeros(1, dtype=torch.int64, device=ref.device)
+    rc = lib.flashmask_count_unmasked(*[_ptr(x) for x in vecs], ctypes.byref(dm), _ptr(out), _stream(ref.device))
+    _check(rc, "flashmask_count_unmasked")
+    return int(out.item())
+
+
+def get_status() -> int:
+    """Synchronises the device; returns and clears the kernels' status word."""
+    return int(load_library().flashmask_get_status())
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    load_library().flashmask_set_wait_limit_ns(ctypes.c_int64(int(ns)))
+
+
+def test_wait_timeout(limit_ns: int, device=None) -> None:
+    """Launches the bounded-wait self test (one CTA waits on a barrier nothing arrives on)."""
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    _check(load_library().flashmask_test_wait_timeout(ctypes.c_int64(int(limit_ns)), _stream(dev)),
+           "flashmask_test_wait_timeout")
+
+
+class _FlashMaskFn(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, q, k, v, lts, lte, uts, ute, scale):
+        o, lse = fwd(q, k, v, lts, lte, uts, ute, scale)
+        ctx.save_for_backward(q, k, v, o, lse, *(x if x is not None else torch.empty(0) for x in (lts, lte, uts, ute)))
+        ctx.none = tuple(x is None for x in (lts, lte, uts, ute))
+        ctx.scale = scale
+        return o
+
+    @staticmethod
+    def backward(ctx, do):
+        q, k, v, o, lse, *m = ctx.saved_tensors
+        m = [None if n else x for x, n in zip(m, ctx.none)]
+        dq, dk, dv = bwd(q, k, v, o, lse, do.contiguous(), *m, scale=ctx.scale)
+        return dq, dk, dv, None, None, None, None, None
+
+
+def flashmask_attention(q, k, v, lts=None, lte=None, uts=None, ute=None, scale: Optional[float] = None):
+    """Autograd-aware masked attention returning O (bf16)."""
+    return _FlashMaskFn.apply(q, k, v, lts, lte, uts, ute, scale)

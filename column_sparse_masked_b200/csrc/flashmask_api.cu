@@ -1,0 +1,439 @@
+// Host side of the C ABI declared in include/flashmask.h: argument checks,
+// workspace carving, TMA descriptor encoding and the launch sequence of each
+// entry point.  No device memory is allocated here.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <climits>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <unordered_map>
+
+#include "../../include/flashmask.h"
+#include "common.cuh"
+#include "launchers.h"
+
+namespace fm {
+
+// Per-device status word written by kernels (bounded-wait timeouts).
+__device__ int g_status_word;
+
+namespace {
+
+std::atomic<int64_t> g_wait_limit_ns{2000000000LL};
+std::mutex g_mu;
+
+struct DeviceInfo {
+  int sm_count = 0;
+  int cc = 0;
+  int* status = nullptr;
+};
+
+int current_device(DeviceInfo* out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FLASHMASK_ERR_NO_DEVICE;
+  static std::unordered_map<int, DeviceInfo> cache;
+  std::lock_guard<std::mutex> lock(g_mu);
+  auto it = cache.find(dev);
+  if (it == cache.end()) {
+    DeviceInfo di;
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&di.sm_count, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return FLASHMASK_ERR_NO_DEVICE;
+    di.cc = major * 10 + minor;
+    if (di.cc != 100) return FLASHMASK_ERR_NO_DEVICE;
+    if (cudaGetSymbolAddress(reinterpret_cast<void**>(&di.status), g_status_word) != cudaSuccess)
+      return FLASHMASK_ERR_CUDA;
+    it = cache.emplace(dev, di).first;
+  }
+  *out = it->second;
+  return FLASHMASK_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 4-D map over a [B, N, H, d] bf16 tensor: box = 64 columns x 1 head x 128 rows.
+int make_map(CUtensorMap* m, const void* ptr, int B, int N, int H, int d) {
+  auto enc = encode_fn();
+  if (!enc) return FLASHMASK_ERR_CUDA;
+  cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)N, (cuuint64_t)B};
+  cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2, (cuuint64_t)N * H * d * 2};
+  cuuint32_t box[4] = {64, 1, (cuuint32_t)kTile, 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FLASHMASK_OK : FLASHMASK_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_dims(const flashmask_dims* dm) {
+  if (!dm) return FLASHMASK_ERR_INVALID_ARG;
+  const flashmask_dims& d = *dm;
+  if (d.B < 0 || d.Hq <= 0 || d.Hkv <= 0 || d.Hm <= 0 || d.Nq < 0 || d.Nk < 0) return FLASHMASK_ERR_INVALID_ARG;
+  if (d.Hq % d.Hkv != 0) return FLASHMASK_ERR_INVALID_ARG;
+  if (d.Hm != 1 && d.Hm != d.Hq) return FLASHMASK_ERR_INVALID_ARG;
+  if (d.d != 64 && d.d != 128) return FLASHMASK_ERR_UNSUPPORTED;
+  if (d.Nq > (1 << 30) || d.Nk > (1 << 30)) return FLASHMASK_ERR_UNSUPPORTED;
+  const Shape s = make_shape(d.B, d.Hq, d.Hkv, d.Hm, d.Nq, d.Nk, d.d);
+  if ((int64_t)s.B * s.Hq * s.nQB >= INT_MAX || (int64_t)s.B * s.Hkv * s.nKt >= INT_MAX)
+    return FLASHMASK_ERR_UNSUPPORTED;
+  return FLASHMASK_OK;
+}
+
+int check_masks(const int32_t* lts, const int32_t* lte, const int32_t* uts, const int32_t* ute) {
+  if ((lts == nullptr) != (lte == nullptr)) return FLASHMASK_ERR_INVALID_ARG;
+  if ((uts == nullptr) != (ute == nullptr)) return FLASHMASK_ERR_INVALID_ARG;
+  for (const int32_t* p : {lts, lte, uts, ute})
+    if (p && !aligned16(p)) return FLASHMASK_ERR_ALIGN;
+  return FLASHMASK_OK;
+}
+
+int check_ws(const void* ws, size_t have, size_t need) {
+  if (need == 0) return FLASHMASK_OK;
+  if (!ws || have < need) return FLASHMASK_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(ws) & 255u) return FLASHMASK_ERR_ALIGN;
+  return FLASHMASK_OK;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? FLASHMASK_OK : FLASHMASK_ERR_CUDA; }
+
+#define FM_TRY(x)                       \
+  do {                                  \
+    int _rc = (x);                      \
+    if (_rc != FLASHMASK_OK) return _rc; \
+  } while (0)
+#define FM_CUDA(x) FM_TRY(cuda_status(x))
+
+float resolve_scale(float scale, int d) { return scale > 0.f ? scale : 1.0f / std::sqrt((float)d); }
+
+// Steps shared by forward, backward and classify: padded boundary records
+// and the per-k-tile block summary.
+MaskPrepParams prep_params(const Shape& s, const WsLayout& L, uint8_t* ws, const int32_t* lts, const int32_t* lte,
+                           const int32_t* uts, const int32_t* ute) {
+  MaskPrepParams mp{};
+  mp.lts = lts; mp.lte = lte; mp.uts = uts; mp.ute = ute;
+  mp.B = s.B; mp.Hm = s.Hm; mp.Nk = s.Nk; mp.nKt = s.nKt;
+  mp.rec = reinterpret_cast<int4*>(ws + L.rec);
+  mp.ksum = reinterpret_cast<int*>(ws + L.ksum);
+  return mp;
+}
+
+}  // namespace
+
+cudaError_t ensure_smem_limit(const void* func, int bytes) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  static std::unordered_map<const void*, uint64_t> done;  // bit per device
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    auto it = done.find(func);
+    if (it != done.end() && dev < 64 && (it->second >> dev) & 1u) return cudaSuccess;
+  }
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (dev < 64) done[func] |= (uint64_t)1 << dev;
+  return cudaSuccess;
+}
+
+}  // namespace fm
+
+using namespace fm;
+
+extern "C" {
+
+size_t flashmask_fwd_workspace_size(const flashmask_dims* d) {
+  if (check_dims(d) != FLASHMASK_OK) return 0;
+  return make_layout(make_shape(d->B, d->Hq, d->Hkv, d->Hm, d->Nq, d->Nk, d->d)).fwd_bytes;
+}
+
+size_t flashmask_bwd_workspace_size(const flashmask_dims* d) {
+  if (check_dims(d) != FLASHMASK_OK) return 0;
+  return make_layout(make_shape(d->B, d->Hq, d->Hkv, d->Hm, d->Nq, d->Nk, d->d)).bwd_bytes;
+}
+
+int flashmask_fwd(const void* q, const void* k, const void* v, const int32_t* lts, const int32_t* lte,
+                  const int32_t* uts, const int32_t* ute, float scale, const flashmask_dims* dims, void* o,
+                  float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+  FM_TRY(check_dims(dims));
+  FM_TRY(check_masks(lts, lte, uts, ute));
+  const flashmask_dims& d = *dims;
+  const Shape s = make_shape(d.B, d.Hq, d.Hkv, d.Hm, d.Nq, d.Nk, d.d);
+  if ((int64_t)s.B * s.Nq == 0) return FLASHMASK_OK;
+  if (!q || !o || !lse || (s.Nk > 0 && (!k || !v))) return FLASHMASK_ERR_INVALID_ARG;
+  for (const void* p : {q, k, v, (const void*)o, (const void*)lse})
+    if (p && !aligned16(p)) return FLASHMASK_ERR_ALIGN;
+  const WsLayout L = make_layout(s);
+  FM_TRY(check_ws(workspace, workspace_bytes, L.fwd_bytes));
+  DeviceInfo di;
+  FM_TRY(current_device(&di));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+
+  CUtensorMap tq, tk, tv;
+  FM_TRY(make_map(&tq, q, s.B, s.Nq, s.Hq, s.d));
+  if (s.Nk > 0) {
+    FM_TRY(make_map(&tk, k, s.B, s.Nk, s.Hkv, s.d));
+    FM_TRY(make_map(&tv, v, s.B, s.Nk, s.Hkv, s.d));
+  } else {  // never read: every work list is empty
+    FM_TRY(make_map(&tk, workspace, 1, 1, 1, s.d));
+    tv = tk;
+  }
+  const MaskPrepParams mp = prep_params(s, L, ws, lts, lte, uts, ute);
+  FM_CUDA(launch_mask_prep(mp, st));
+
+  PlanParams pp{};
+  pp.s = s;
+  pp.ksum = mp.ksum;
+  pp.fcount = reinterpret_cast<int*>(ws + L.fcount);
+  pp.flist = reinterpret_cast<int*>(ws + L.flist);
+  FM_CUDA(launch_plan_fwd(pp, st));
+
+  SortParams sp{};
+  sp.s = s;
+  sp.mode = 0;
+  sp.count = pp.fcount;
+  sp.order = reinterpret_cast<int*>(ws + L.forder);
+  sp.counter = reinterpret_cast<int*>(ws + L.counters);
+  sp.n_units = (int)s.n_units_fwd;
+  FM_CUDA(launch_sort_units(sp, st));
+
+  FwdParams fp{};
+  fp.s = s;
+  fp.scale_log2 = resolve_scale(scale, s.d) * 1.4426950408889634f;
+  fp.rec = mp.rec;
+  fp.flist = pp.flist;
+  fp.fcount = pp.fcount;
+  fp.order = sp.order;
+  fp.counter = sp.counter;
+  fp.n_items = (int)(s.n_units_fwd * s.Ef);
+  fp.o = static_cast<__nv_bfloat16*>(o);
+  fp.lse = lse;
+  fp.status = di.status;
+  fp.wait_limit_ns = (uint64_t)g_wait_limit_ns.load();
+  const int grid = fp.n_items < di.sm_count ? fp.n_items : di.sm_count;
+  if (grid > 0) FM_CUDA(launch_fwd(fp, tq, tk, tv, grid, st));
+  return FLASHMASK_OK;
+}
+
+int flashmask_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+                  const int32_t* lts, const int32_t* lte, const int32_t* uts, const int32_t* ute, float scale,
+                  const flashmask_dims* dims, void* dq, void* dk, void* dv, void* workspace,
+                  size_t workspace_bytes, void* stream) {
+  FM_TRY(check_dims(dims));
+  FM_TRY(check_masks(lts, lte, uts, ute));
+  const flashmask_dims& d = *dims;
+  const Shape s = make_shape(d.B, d.Hq, d.Hkv, d.Hm, d.Nq, d.Nk, d.d);
+  if (s.B == 0) return FLASHMASK_OK;
+  const bool has_q = s.Nq > 0, has_k = s.Nk > 0;
+  if (has_q && (!q || !o || !lse || !dout || !dq)) return FLASHMASK_ERR_INVALID_ARG;
+  if (has_k && (!k || !v || !dk || !dv)) return FLASHMASK_ERR_INVALID_ARG;
+  for (const void* p : {q, k, v, o, (const void*)lse, dout, (const void*)dq, (const void*)dk, (const void*)dv})
+    if (p && !aligned16(p)) return FLASHMASK_ERR_ALIGN;
+  const WsLayout L = make_layout(s);
+  FM_TRY(check_ws(workspace, workspace_bytes, L.bwd_bytes));
+  DeviceInfo di;
+  FM_TRY(current_device(&di));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const float sc = resolve_scale(scale, s.d);
+
+  CUtensorMap tq, tk, tv, tdo;
+  if (has_q) {
+    FM_TRY(make_map(&tq, q, s.B, s.Nq, s.Hq, s.d));
+    FM_TRY(make_map(&tdo, dout, s.B, s.Nq, s.Hq, s.d));
+  } else {
+    FM_TRY(make_map(&tq, workspace, 1, 1, 1, s.d));
+    tdo = tq;
+  }
+  if (has_k) {
+    FM_TRY(make_map(&tk, k, s.B, s.Nk, s.Hkv, s.d));
+    FM_TRY(make_map(&tv, v, s.B, s.Nk, s.Hkv, s.d));
+  } else {
+    FM_TRY(make_map(&tk, workspace, 1, 1, 1, s.d));
+    tv = tk;
+  }
+  const MaskPrepParams mp = prep_params(s, L, ws, lts, lte, uts, ute);
+  FM_CUDA(launch_mask_prep(mp, st));
+
+  PlanParams pp{};
+  pp.s = s;
+  pp.ksum = mp.ksum;
+  pp.bcount = reinterpret_cast<int*>(ws + L.bcount);
+  pp.blist = reinterpret_cast<int*>(ws + L.blist);
+  FM_CUDA(launch_plan_bwd(pp, st));
+
+  SortParams sp{};
+  sp.s = s;
+  sp.mode = 1;
+  sp.count = pp.bcount;
+  sp.order = reinterpret_cast<int*>(ws + L.border);
+  sp.counter = reinterpret_cast<int*>(ws + L.counters) + 1;
+  sp.n_units = (int)s.n_units_bwd;
+  if (sp.n_units > 0) FM_CUDA(launch_sort_units(sp, st));
+
+  BwdPreParams bp{};
+  bp.s = s;
+  bp.o = static_cast<const __nv_bfloat16*>(o);
+  bp.dout = static_cast<const __nv_bfloat16*>(dout);
+  bp.lse = lse;
+  bp.lse2 = reinterpret_cast<float*>(ws + L.lse2);
+  bp.dsum = reinterpret_cast<float*>(ws + L.dsum);
+  bp.dqacc = reinterpret_cast<float*>(ws + L.dqacc);
+  if (has_q) FM_CUDA(launch_bwd_pre(bp, st));
+
+  BwdParams kp{};
+  kp.s = s;
+  kp.scale = sc;
+  kp.scale_log2 = sc * 1.4426950408889634f;
+  kp.rec = mp.rec;
+  kp.blist = pp.blist;
+  kp.bcount = pp.bcount;
+  kp.order = sp.order;
+  kp.counter = sp.counter;
+  kp.n_items = (int)(s.n_units_bwd * s.Eb);
+  kp.lse2 = bp.lse2;
+  kp.dsum = bp.dsum;
+  kp.dqacc = bp.dqacc;
+  kp.dk = static_cast<__nv_bfloat16*>(dk);
+  kp.dv = static_cast<__nv_bfloat16*>(dv);
+  kp.status = di.status;
+  kp.wait_limit_ns = (uint64_t)g_wait_limit_ns.load();
+  const int grid = kp.n_items < di.sm_count ? kp.n_items : di.sm_count;
+  if (grid > 0) FM_CUDA(launch_bwd(kp, tq, tk, tv, tdo, grid, st));
+
+  if (has_q) {
+    DqFinParams fp{};
+    fp.dqacc = bp.dqacc;
+    fp.dq = static_cast<__nv_bfloat16*>(dq);
+    fp.scale = sc;
+    fp.n = (int64_t)s.B * s.Nq * s.Hq * s.d;
+    FM_CUDA(launch_dq_finalize(fp, st));
+  }
+  return FLASHMASK_OK;
+}
+
+int flashmask_classify(const int32_t* lts, const int32_t* lte, const int32_t* uts, const int32_t* ute,
+                       const flashmask_dims* dims, uint8_t* cls, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+  FM_TRY(check_dims(dims));
+  FM_TRY(check_masks(lts, lte, uts, ute));
+  const flashmask_dims& d = *dims;
+  const Shape s = make_shape(d.B, d.Hq, d.Hkv, d.Hm, d.Nq, d.Nk, d.d);
+  if ((int64_t)s.B * s.nQt * s.nKt == 0) return FLASHMASK_OK;
+  if (!cls) return FLASHMASK_ERR_INVALID_ARG;
+  const WsLayout L = make_layout(s);
+  FM_TRY(check_ws(workspace, workspace_bytes, L.fwd_bytes));
+  DeviceInfo di;
+  FM_TRY(current_device(&di));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const MaskPrepParams mp = prep_params(s, L, ws, lts, lte, uts, ute);
+  FM_CUDA(launch_mask_prep(mp, st));
+  PlanParams pp{};
+  pp.s = s;
+  pp.ksum = mp.ksum;
+  pp.cls = cls;
+  FM_CUDA(launch_classify_export(pp, st));
+  return FLASHMASK_OK;
+}
+
+int flashmask_localize(const int32_t* in, int32_t* out, int64_t n, int32_t a, int32_t b, void* stream) {
+  if (n < 0 || a < 0 || b < a) return FLASHMASK_ERR_INVALID_ARG;
+  if (n == 0) return FLASHMASK_OK;
+  if (!in || !out) return FLASHMASK_ERR_INVALID_ARG;
+  DeviceInfo di;
+  FM_TRY(current_device(&di));
+  FM_CUDA(launch_localize(in, out, n, a, b, static_cast<cudaStream_t>(stream)));
+  return FLASHMASK_OK;
+}
+
+int flashmask_localize_multi(const int32_t* in, int32_t* out, int64_t n, const int32_t* starts,
+                             const int32_t* ends, int32_t nchunks, void* stream) {
+  if (n < 0 || nchunks < 0 || nchunks > 64) return FLASHMASK_ERR_INVALID_ARG;
+  if (nchunks > 0 && (!starts || !ends)) return FLASHMASK_ERR_INVALID_ARG;
+  for (int c = 0; c < nchunks; ++c) {
+    if (starts[c] < 0 || ends[c] < starts[c]) return FLASHMASK_ERR_INVALID_ARG;
+    if (c > 0 && starts[c] < ends[c - 1]) return FLASHMASK_ERR_INVALID_ARG;
+  }
+  if (n == 0) return FLASHMASK_OK;
+  if (!in || !out) return FLASHMASK_ERR_INVALID_ARG;
+  DeviceInfo di;
+  FM_TRY(current_device(&di));
+  FM_CUDA(launch_localize_multi(in, out, n, starts, ends, nchunks, static_cast<cudaStream_t>(stream)));
+  return FLASHMASK_OK;
+}
+
+int flashmask_count_unmasked(const int32_t* lts, const int32_t* lte, const int32_t* uts, const int32_t* ute,
+                             const flashmask_dims* dims, int64_t* pairs, void* stream) {
+  FM_TRY(check_dims(dims));
+  FM_TRY(check_masks(lts, lte, uts, ute));
+  if (!pairs) return FLASHMASK_ERR_INVALID_ARG;
+  DeviceInfo di;
+  FM_TRY(current_device(&di));
+  const flashmask_dims& d = *dims;
+  MaskPrepParams mp{};
+  mp.lts = lts; mp.lte = lte; mp.uts = uts; mp.ute = ute;
+  mp.B = d.B; mp.Hm = d.Hm; mp.Nk = d.Nk;
+  FM_CUDA(launch_count_unmasked(mp, d.Hq, d.Nq, pairs, static_cast<cudaStream_t>(stream)));
+  return FLASHMASK_OK;
+}
+
+int flashmask_get_status(void) {
+  DeviceInfo di;
+  FM_TRY(current_device(&di));
+  if (cudaDeviceSynchronize() != cudaSuccess) return FLASHMASK_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, di.status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return FLASHMASK_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpy(di.status, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return FLASHMASK_ERR_CUDA;
+  return v;
+}
+
+void flashmask_set_wait_limit_ns(int64_t ns) { g_wait_limit_ns.store(ns > 0 ? ns : 2000000000LL); }
+
+int flashmask_test_wait_timeout(int64_t limit_ns, void* stream) {
+  if (limit_ns <= 0) return FLASHMASK_ERR_INVALID_ARG;
+  DeviceInfo di;
+  FM_TRY(current_device(&di));
+  FM_CUDA(launch_wait_timeout(di.status, (uint64_t)limit_ns, static_cast<cudaStream_t>(stream)));
+  return FLASHMASK_OK;
+}
+
+const char* flashmask_strerror(int code) {
+  switch (code) {
+    case FLASHMASK_OK: return "ok";
+    case FLASHMASK_ERR_INVALID_ARG: return "invalid argument (null pointer, negative size or head counts)";
+    case FLASHMASK_ERR_UNSUPPORTED: return "unsupported configuration (head_dim must be 64 or 128; sizes too large)";
+    case FLASHMASK_ERR_ALIGN: return "pointer not 16-byte aligned (workspace: 256-byte)";
+    case FLASHMASK_ERR_WORKSPACE: return "workspace missing or too small";
+    case FLASHMASK_ERR_CUDA: return "CUDA runtime or launch failure";
+    case FLASHMASK_ERR_TIMEOUT: return "a device-side bounded wait timed out";
+    case FLASHMASK_ERR_NO_DEVICE: return "no sm_100 (B200-class) device is current";
+    default: return "unknown error code";
+  }
+}
+
+int flashmask_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,32 @@
+// Host-side launchers of the kernels; each returns the launch status.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+
+namespace fm {
+
+cudaError_t launch_mask_prep(const MaskPrepParams& p, cudaStream_t st);
+cudaError_t launch_plan_fwd(const PlanParams& p, cudaStream_t st);
+cudaError_t launch_plan_bwd(const PlanParams& p, cudaStream_t st);
+cudaError_t launch_classify_export(const PlanParams& p, cudaStream_t st);
+cudaError_t launch_sort_units(const SortParams& p, cudaStream_t st);
+cudaError_t launch_localize(const int32_t* in, int32_t* out, int64_t n, int32_t a, int32_t b, cudaStream_t st);
+cudaError_t launch_localize_multi(const int32_t* in, int32_t* out, int64_t n, const int32_t* starts,
+                                  const int32_t* ends, int nchunks, cudaStream_t st);
+cudaError_t launch_count_unmasked(const MaskPrepParams& p, int Hq, int Nq, int64_t* out, cudaStream_t st);
+cudaError_t launch_wait_timeout(int* status, uint64_t limit_ns, cudaStream_t st);
+
+// Forward / backward attention kernels.  `grid` is the persistent CTA count.
+cudaError_t launch_fwd(const FwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       int grid, cudaStream_t st);
+cudaError_t launch_bwd_pre(const BwdPreParams& p, cudaStream_t st);
+cudaError_t launch_bwd(const BwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                       const CUtensorMap& tdo, int grid, cudaStream_t st);
+cudaError_t launch_dq_finalize(const DqFinParams& p, cudaStream_t st);
+
+// Raises a kernel's dynamic shared-memory limit once per (kernel, device).
+cudaError_t ensure_smem_limit(const void* func, int bytes);
+
+}  // namespace fm

@@ -1,0 +1,364 @@
+// Mask-side kernels: boundary-record preparation and the per-k-tile block
+// summary, tile classification into per-block work lists, the longest-first
+// order of scheduling units, clip-shift-max localisation and the closed-form
+// count of unmasked pairs.
+//
+// Method: "FlashMask-3 targets masked distributed attention on Hopper GPUs",
+// In-depth insight -- the column-wise mask (four query-axis boundary vectors
+// per key column), tiles decided from O(n) data, and the zero-communication
+// clip-shift-max localisation of a query chunk.
+#include <cuda_runtime.h>
+#include <climits>
+#include <cstdint>
+
+#include "common.cuh"
+#include "launchers.h"
+#include "sm100_primitives.cuh"
+
+namespace fm {
+
+// ----------------------------------------------------------------------------
+// 1. padded boundary records + block summary, one CTA per (k-tile, hm, b)
+// ----------------------------------------------------------------------------
+__global__ void __launch_bounds__(128) mask_prep_kernel(MaskPrepParams p) {
+  const int kt = blockIdx.x, hm = blockIdx.y, b = blockIdx.z;
+  const int t = threadIdx.x;
+  const int j = kt * kTile + t;
+  const size_t row = (size_t)b * p.Hm + hm;
+  const bool real = j < p.Nk;
+  int4 r = make_int4(0, INT_MAX, 0, 0);  // padded column: hidden from every row
+  if (real) {
+    const size_t idx = row * p.Nk + j;
+    r.x = p.lts ? p.lts[idx] : 0;
+    r.y = p.lte ? p.lte[idx] : 0;
+    r.z = p.uts ? p.uts[idx] : 0;
+    r.w = p.ute ? p.ute[idx] : 0;
+  }
+  p.rec[(row * p.nKt + kt) * kTile + t] = r;
+  // min/max over the real columns of the tile
+  int v[8];
+  v[kMnLts] = real ? r.x : INT_MAX; v[kMxLts] = real ? r.x : INT_MIN;
+  v[kMnLte] = real ? r.y : INT_MAX; v[kMxLte] = real ? r.y : INT_MIN;
+  v[kMnUts] = real ? r.z : INT_MAX; v[kMxUts] = real ? r.z : INT_MIN;
+  v[kMnUte] = real ? r.w : INT_MAX; v[kMxUte] = real ? r.w : INT_MIN;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+#pragma unroll
+    for (int e = 0; e < 8; e += 2) {
+      v[e] = min(v[e], __shfl_xor_sync(0xffffffffu, v[e], off));
+      v[e + 1] = max(v[e + 1], __shfl_xor_sync(0xffffffffu, v[e + 1], off));
+    }
+  }
+  __shared__ int part[4][8];
+  if ((t & 31) == 0)
+#pragma unroll
+    for (int e = 0; e < 8; ++e) part[t >> 5][e] = v[e];
+  __syncthreads();
+  if (t < 8) {
+    int a = part[0][t];
+    for (int w = 1; w < 4; ++w) a = (t & 1) ? max(a, part[w][t]) : min(a, part[w][t]);
+    p.ksum[(row * p.nKt + kt) * 8 + t] = a;
+  }
+}
+
+// Block-wide exclusive prefix of a 0/1 flag over 128 threads; returns the
+// position of this thread among the set flags and writes the total.
+__device__ __forceinline__ int block_compact128(bool flag, int* warp_tot, int* total) {
+  const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+  const unsigned bal = __ballot_sync(0xffffffffu, flag);
+  const int pos = __popc(bal & ((1u << lane) - 1u));
+  if (lane == 0) warp_tot[w] = __popc(bal);
+  __syncthreads();
+  int base = 0;
+  for (int i = 0; i < w; ++i) base += warp_tot[i];
+  if (t == 0) *total = warp_tot[0] + warp_tot[1] + warp_tot[2] + warp_tot[3];
+  __syncthreads();
+  return base + pos;
+}
+
+// ----------------------------------------------------------------------------
+// 2a. forward work lists: per (b, hm, block of two q-tiles) the k-tiles that
+//     are not skipped for at least one of the two q-tiles, in increasing order
+// ----------------------------------------------------------------------------
+__global__ void __launch_bounds__(128) plan_fwd_kernel(PlanParams p) {
+  const Shape& s = p.s;
+  const int qb = blockIdx.x, hm = blockIdx.y, b = blockIdx.z;
+  const size_t row = (size_t)b * s.Hm + hm;
+  const int qt0 = 2 * qb, qt1 = 2 * qb + 1;
+  const int r00 = qt0 * kTile, r01 = min(r00 + kTile, s.Nq);
+  const int r10 = qt1 * kTile, r11 = min(r10 + kTile, s.Nq);
+  const bool ragged_k = (s.Nk % kTile) != 0;
+  int* list = p.flist + (row * s.nQB + qb) * s.nKt;
+  __shared__ int warp_tot[4];
+  __shared__ int total;
+  int count = 0;
+  for (int base = 0; base < s.nKt; base += kTile) {
+    const int kt = base + threadIdx.x;
+    int c0 = kClsSkip, c1 = kClsSkip;
+    if (kt < s.nKt) {
+      int sm[8];
+      const int* src = p.ksum + (row * s.nKt + kt) * 8;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) sm[e] = src[e];
+      c0 = classify_tile(sm, r00, r01);
+      if (qt1 < s.nQt) c1 = classify_tile(sm, r10, r11);
+    }
+    const bool keep = (c0 != kClsSkip) || (c1 != kClsSkip);
+    const int pos = block_compact128(keep, warp_tot, &total);
+    if (keep) list[count + pos] = fwd_entry(kt, c0, c1, (ragged_k && kt == s.nKt - 1) ? 1 : 0);
+    count += total;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) p.fcount[row * s.nQB + qb] = count;
+}
+
+// ----------------------------------------------------------------------------
+// 2b. backward work lists: per (b, hm, k-tile) the q-tiles that are not skipped
+// ----------------------------------------------------------------------------
+__global__ void __launch_bounds__(128) plan_bwd_kernel(PlanParams p) {
+  const Shape& s = p.s;
+  const int kt = blockIdx.x, hm = blockIdx.y, b = blockIdx.z;
+  const size_t row = (size_t)b * s.Hm + hm;
+  int sm[8];
+  const int* src = p.ksum + (row * s.nKt + kt) * 8;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) sm[e] = src[e];
+  int* list = p.blist + (row * s.nKt + kt) * s.nQt;
+  __shared__ int warp_tot[4];
+  __shared__ int total;
+  int count = 0;
+  for (int base = 0; base < s.nQt; base += kTile) {
+    const int qt = base + threadIdx.x;
+    int c = kClsSkip;
+    if (qt < s.nQt) c = classify_tile(sm, qt * kTile, min(qt * kTile + kTile, s.Nq));
+    const bool keep = c != kClsSkip;
+    const int pos = block_compact128(keep, warp_tot, &total);
+    if (keep) list[count + pos] = bwd_entry(qt, c);
+    count += total;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) p.bcount[row * s.nKt + kt] = count;
+}
+
+// ----------------------------------------------------------------------------
+// 2c. class export [B, Hm, nQt, nKt]
+// ----------------------------------------------------------------------------
+__global__ void __launch_bounds__(128) classify_export_kernel(PlanParams p) {
+  const Shape& s = p.s;
+  const int qt = blockIdx.x, hm = blockIdx.y, b = blockIdx.z;
+  const size_t row = (size_t)b * s.Hm + hm;
+  const int r0 = qt * kTile, r1 = min(r0 + kTile, s.Nq);
+  for (int kt = threadIdx.x; kt < s.nKt; kt += blockDim.x) {
+    int sm[8];
+    const int* src = p.ksum + (row * s.nKt + kt) * 8;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) sm[e] = src[e];
+    p.cls[(row * s.nQt + qt) * s.nKt + kt] = (uint8_t)classify_tile(sm, r0, r1);
+  }
+}
+
+// ----------------------------------------------------------------------------
+// 3. longest-first order of scheduling units (one CTA, bitonic sort in smem).
+//    Key = (~cost << 32) | unit: descending cost, ascending unit id on ties.
+//    Also zeroes the work counter of the persistent kernel that follows.
+// ----------------------------------------------------------------------------
+constexpr int kSortMax = 8192;
+
+__global__ void __launch_bounds__(1024) sort_units_kernel(SortParams p) {
+  extern __shared__ unsigned long long keys[];
+  const Shape& s = p.s;
+  const int n = p.n_units;
+  const int t = threadIdx.x;
+  if (t == 0) p.counter[0] = 0;
+  if (n > kSortMax) {  // too many units for the in-smem sort: identity order
+    for (int u = t; u < n; u += blockDim.x) p.order[u] = u;
+    return;
+  }
+  int np2 = 1;
+  while (np2 < n) np2 <<= 1;
+  for (int u = t; u < np2; u += blockDim.x) {
+    unsigned long long key = ~0ull;
+    if (u < n) {
+      unsigned cost;
+      if (p.mode == 0) {
+        cost = (unsigned)p.count[u];
+      } else {
+        // unit u = (b, mu, kt); its q-heads' lists live at mask heads
+        // [mu*Gm, mu*Gm + Gm) with Gm = 1 for a shared mask.
+        const int kt = u % s.nKt, mu = (u / s.nKt) % s.Mu, b = u / (s.nKt * s.Mu);
+        if (s.Hm == 1) {
+          cost = (unsigned)p.count[(size_t)b * s.nKt + kt] * (unsigned)s.G;
+        } else {
+          cost = 0;
+          for (int g = 0; g < s.G; ++g) cost += (unsigned)p.count[((size_t)b * s.Hm + mu * s.G + g) * s.nKt + kt];
+        }
+      }
+      key = ((unsigned long long)(~cost) << 32) | (unsigned)u;
+    }
+    keys[u] = key;
+  }
+  __syncthreads();
+  for (int k = 2; k <= np2; k <<= 1) {
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      for (int i = t; i < np2; i += blockDim.x) {
+        const int ixj = i ^ j;
+        if (ixj > i) {
+          const bool up = (i & k) == 0;
+          const unsigned long long a = keys[i], c = keys[ixj];
+          if ((a > c) == up) {
+            keys[i] = c;
+            keys[ixj] = a;
+          }
+        }
+      }
+      __syncthreads();
+    }
+  }
+  for (int u = t; u < n; u += blockDim.x) p.order[u] = (int)(keys[u] & 0xffffffffu);
+}
+
+// ----------------------------------------------------------------------------
+// 4. clip-shift-max localisation
+// ----------------------------------------------------------------------------
+__global__ void localize_kernel(const int32_t* in, int32_t* out, int64_t n, int32_t a, int32_t b) {
+  for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < n; t += (int64_t)gridDim.x * blockDim.x) {
+    const int32_t x = min(in[t], b) - a;  // clip to the chunk end, shift to local rows
+    out[t] = max(x, 0);                   // max with zero
+  }
+}
+
+struct Chunks {
+  int32_t a[64], b[64];
+  int n;
+};
+
+__global__ void localize_multi_kernel(const int32_t* in, int32_t* out, int64_t n, Chunks c) {
+  for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < n; t += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t x = in[t];
+    int64_t acc = 0;
+    for (int k = 0; k < c.n; ++k) acc += min(max(x, (int64_t)c.a[k]), (int64_t)c.b[k]) - c.a[k];
+    out[t] = (int32_t)acc;
+  }
+}
+
+// ----------------------------------------------------------------------------
+// 5. unmasked pairs, closed form per key column (one CTA, deterministic)
+//    masked_j = |L n [0,Nq)| + |U n [0,Nq)| - |L n U n [0,Nq)|
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ int64_t overlap_len(int64_t a, int64_t b, int64_t lo, int64_t hi) {
+  const int64_t x = max(a, lo), y = min(b, hi);
+  return y > x ? y - x : 0;
+}
+
+__global__ void __launch_bounds__(1024) count_unmasked_kernel(MaskPrepParams p, int Hq, int Nq, int64_t* out) {
+  const int64_t total = (int64_t)p.B * p.Hm * p.Nk;
+  const int64_t weight = (p.Hm == 1) ? Hq : 1;
+  unsigned long long acc = 0;
+  for (int64_t t = threadIdx.x; t < total; t += blockDim.x) {
+    const int64_t lts = p.lts ? p.lts[t] : 0, lte = p.lte ? p.lte[t] : 0;
+    const int64_t uts = p.uts ? p.uts[t] : 0, ute = p.ute ? p.ute[t] : 0;
+    const int64_t mL = overlap_len(lts, lte, 0, Nq);
+    const int64_t mU = overlap_len(uts, ute, 0, Nq);
+    const int64_t mLU = overlap_len(max(lts, uts), min(lte, ute), 0, Nq);
+    acc += (unsigned long long)((Nq - (mL + mU - mLU)) * weight);
+  }
+  __shared__ unsigned long long red[32];
+  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    unsigned long long s = 0;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) s += red[w];
+    *out = (int64_t)s;
+  }
+}
+
+// ----------------------------------------------------------------------------
+// 6. bounded-wait self test: waits on a barrier that nothing arrives on
+// ----------------------------------------------------------------------------
+__global__ void wait_timeout_kernel(int* status, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    WaitCtx w{&abort_flag, status, limit_ns};
+    (void)mbar_wait(&bar, 0, w);  // gives up after limit_ns, records the timeout
+  }
+  __syncthreads();
+}
+
+// ----------------------------------------------------------------------------
+// host launchers
+// ----------------------------------------------------------------------------
+cudaError_t launch_mask_prep(const MaskPrepParams& p, cudaStream_t st) {
+  if (p.B == 0 || p.Hm == 0 || p.nKt == 0) return cudaSuccess;
+  mask_prep_kernel<<<dim3(p.nKt, p.Hm, p.B), 128, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_plan_fwd(const PlanParams& p, cudaStream_t st) {
+  if (p.s.B == 0 || p.s.nQB == 0) return cudaSuccess;
+  plan_fwd_kernel<<<dim3(p.s.nQB, p.s.Hm, p.s.B), 128, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_plan_bwd(const PlanParams& p, cudaStream_t st) {
+  if (p.s.B == 0 || p.s.nKt == 0) return cudaSuccess;
+  plan_bwd_kernel<<<dim3(p.s.nKt, p.s.Hm, p.s.B), 128, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_classify_export(const PlanParams& p, cudaStream_t st) {
+  if (p.s.B == 0 || p.s.nQt == 0 || p.s.nKt == 0) return cudaSuccess;
+  classify_export_kernel<<<dim3(p.s.nQt, p.s.Hm, p.s.B), 128, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_sort_units(const SortParams& p, cudaStream_t st) {
+  const int n = p.n_units;
+  int np2 = 1;
+  while (np2 < n) np2 <<= 1;
+  const size_t smem = (n <= kSortMax) ? (size_t)np2 * sizeof(unsigned long long) : 0;
+  cudaError_t e = ensure_smem_limit((const void*)sort_units_kernel, (int)(kSortMax * sizeof(unsigned long long)));
+  if (e != cudaSuccess) return e;
+  sort_units_kernel<<<1, 1024, smem, st>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_localize(const int32_t* in, int32_t* out, int64_t n, int32_t a, int32_t b, cudaStream_t st) {
+  if (n == 0) return cudaSuccess;
+  const int64_t blocks = (n + 255) / 256;
+  localize_kernel<<<(unsigned)(blocks < 65535 ? blocks : 65535), 256, 0, st>>>(in, out, n, a, b);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_localize_multi(const int32_t* in, int32_t* out, int64_t n, const int32_t* starts,
+                                  const int32_t* ends, int nchunks, cudaStream_t st) {
+  if (n == 0) return cudaSuccess;
+  Chunks c{};
+  c.n = nchunks;
+  for (int k = 0; k < nchunks; ++k) {
+    c.a[k] = starts[k];
+    c.b[k] = ends[k];
+  }
+  const int64_t blocks = (n + 255) / 256;
+  localize_multi_kernel<<<(unsigned)(blocks < 65535 ? blocks : 65535), 256, 0, st>>>(in, out, n, c);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_count_unmasked(const MaskPrepParams& p, int Hq, int Nq, int64_t* out, cudaStream_t st) {
+  count_unmasked_kernel<<<1, 1024, 0, st>>>(p, Hq, Nq, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_wait_timeout(int* status, uint64_t limit_ns, cudaStream_t st) {
+  wait_timeout_kernel<<<1, 32, 0, st>>>(status, limit_ns);
+  return cudaGetLastError();
+}
+
+}  // namespace fm

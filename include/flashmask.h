@@ -1,0 +1,165 @@
+/*
+ * flashmask.h -- C ABI of the B200 (sm_100a) column-sparse masked attention
+ * library.
+ *
+ * The method: "FlashMask-3 targets masked distributed attention on Hopper
+ * GPUs", section "In-depth insight".  A structured attention mask is stored
+ * column-wise: for every key column j four int32 query-axis boundaries
+ * LTS[j], LTE[j], UTS[j], UTE[j] (O(n) storage instead of O(n^2)).  Query row
+ * i is masked for key j iff
+ *
+ *     LTS[j] <= i < LTE[j]   or   UTS[j] <= i < UTE[j]      (half-open)
+ *
+ * An interval with start >= end is empty.  That encoding covers causal,
+ * document, prefix-LM, share-question, sliding-window and block-sparse masks.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All tensor pointers are DEVICE pointers owned by the caller.  The
+ *    library never allocates or frees device memory; scratch space is passed
+ *    in as `workspace` (size from the *_workspace_size queries).
+ *  - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
+ *    NULL = legacy default stream) and returns 0 or a negative FLASHMASK_ERR_*
+ *    code.  Argument errors are detected on the host before any launch.
+ *  - Layouts (contiguous, row-major, bf16 = IEEE bfloat16 bit patterns):
+ *      q, o, dout, dq      [B, Nq, Hq, d]
+ *      k, v, dk, dv        [B, Nk, Hkv, d]
+ *      lse                 [B, Hq, Nq]   float32, natural log of the
+ *                                        row's softmax normaliser
+ *      lts, lte, uts, ute  [B, Hm, Nk]   int32
+ *    q-head h reads KV head h / (Hq / Hkv) and mask head (Hm == 1 ? 0 : h).
+ *  - A NULL (lts, lte) pair or a NULL (uts, ute) pair means that interval is
+ *    empty for every column.
+ *  - scale <= 0 selects 1/sqrt(d).
+ *  - Supported: d in {64, 128}; Hq % Hkv == 0; Hm in {1, Hq}; any
+ *    Nq, Nk >= 0 (ragged tails are handled); all pointers 16-byte aligned.
+ *  - Tiles are 128 query rows x 128 key columns.
+ *  - Device-side failures (a bounded wait that timed out) are recorded in a
+ *    per-device status word that flashmask_get_status() reads and clears.
+ */
+#ifndef FLASHMASK_H_
+#define FLASHMASK_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define FLASHMASK_OK 0
+#define FLASHMASK_ERR_INVALID_ARG (-1) /* null pointer, negative size, bad head counts   */
+#define FLASHMASK_ERR_UNSUPPORTED (-2) /* d not in {64,128}, sizes above int32 ranges     */
+#define FLASHMASK_ERR_ALIGN (-3)       /* a pointer is not 16-byte aligned                */
+#define FLASHMASK_ERR_WORKSPACE (-4)   /* workspace missing or smaller than required      */
+#define FLASHMASK_ERR_CUDA (-5)        /* a CUDA runtime call or launch failed            */
+#define FLASHMASK_ERR_TIMEOUT (-6)     /* a kernel's bounded wait expired (status word)   */
+#define FLASHMASK_ERR_NO_DEVICE (-7)   /* no sm_100 device current                        */
+
+/* Problem shape.  B batch, Hq query heads, Hkv key/value heads, Hm mask heads
+ * (1 or Hq), Nq query rows, Nk key columns, d head dimension. */
+typedef struct flashmask_dims {
+  int32_t B, Hq, Hkv, Hm, Nq, Nk, d;
+} flashmask_dims;
+
+/* Bytes of workspace flashmask_fwd needs for `dims` (mask summary, padded
+ * boundary records, per-tile work lists, scheduler order). */
+size_t flashmask_fwd_workspace_size(const flashmask_dims* dims);
+
+/*
+ * Forward: O = softmax(scale * Q K^T + mask) V per (batch, q-head) and
+ * LSE = m + ln(sum exp(s - m)) per row ("FlashMask-3 targets masked
+ * distributed attention on Hopper GPUs", In-depth insight: mask-aware
+ * attention forward).  Tiles that the per-tile min/max summary proves fully
+ * masked are skipped; the element mask is applied only on partially masked
+ * tiles.  Rows with no visible key produce O = 0 and LSE = -inf.
+ * Outputs: o (bf16, written in full), lse (fp32, written in full).
+ */
+int flashmask_fwd(const void* q, const void* k, const void* v, const int32_t* lts, const int32_t* lte,
+                  const int32_t* uts, const int32_t* ute, float scale, const flashmask_dims* dims, void* o,
+                  float* lse, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of workspace flashmask_bwd needs (forward's plus the backward lists,
+ * per-row D = rowsum(dO*O), and an fp32 dQ accumulator [B, Nq, Hq, d]). */
+size_t flashmask_bwd_workspace_size(const flashmask_dims* dims);
+
+/*
+ * Backward of the forward above for the loss sum(O * dO) (same page:
+ * "forward+backward"): dQ, dK, dV.  dK and dV sum the contributions of the
+ * Hq/Hkv q-heads that share a KV head.  `o` and `lse` must be the forward's
+ * outputs for the same inputs.  Key columns that no row sees get dK = dV = 0;
+ * fully masked rows get dQ = 0.  Outputs are written in full.
+ */
+int flashmask_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+                  const int32_t* lts, const int32_t* lte, const int32_t* uts, const int32_t* ute, float scale,
+                  const flashmask_dims* dims, void* dq, void* dk, void* dv, void* workspace,
+                  size_t workspace_bytes, void* stream);
+
+/*
+ * Tile classification (the block summary of the method: per key tile the
+ * min/max of each boundary vector).  cls is uint8 [B, Hm, ceil(Nq/128),
+ * ceil(Nk/128)].  With mn_X/mx_X the min/max of X over the tile's columns
+ * and the q-tile's rows [r0, r1), r1 = min(r0 + 128, Nq):
+ *   0 skip     (mx_LTS <= r0 && mn_LTE >= r1) || (mx_UTS <= r0 && mn_UTE >= r1)
+ *   2 full     (mn_LTS >= r1 || mx_LTE <= r0 || mn_LTS >= mx_LTE) &&
+ *              (mn_UTS >= r1 || mx_UTE <= r0 || mn_UTS >= mx_UTE)
+ *   1 partial  otherwise.
+ * Uses the forward workspace.
+ */
+int flashmask_classify(const int32_t* lts, const int32_t* lte, const int32_t* uts, const int32_t* ute,
+                       const flashmask_dims* dims, uint8_t* cls, void* workspace, size_t workspace_bytes,
+                       void* stream);
+
+/*
+ * Clip-shift-max localisation (same page: the "provably zero-communication"
+ * per-chunk mask localisation): for the contiguous query chunk [a, b),
+ * out[t] = max(min(in[t], b) - a, 0) for t < n.  Applied to each of the four
+ * vectors, the result encodes exactly rows [a, b) of the full mask.  in and
+ * out are device int32 arrays of n elements (may alias).  0 <= a <= b.
+ */
+int flashmask_localize(const int32_t* in, int32_t* out, int64_t n, int32_t a, int32_t b, void* stream);
+
+/*
+ * Localisation onto several increasing, disjoint chunks [starts[c], ends[c])
+ * concatenated in order into one local query sequence ("any multi-chunk
+ * context-parallel assignment"): out[t] = sum_c (clamp(in[t], starts[c],
+ * ends[c]) - starts[c]).  starts/ends are HOST arrays of nchunks (<= 64)
+ * values.
+ */
+int flashmask_localize_multi(const int32_t* in, int32_t* out, int64_t n, const int32_t* starts,
+                             const int32_t* ends, int32_t nchunks, void* stream);
+
+/*
+ * Number of unmasked (i, j) pairs over all batches and all Hq query heads,
+ * written as one int64 to the device pointer `pairs` (closed form per key
+ * column; used for the effective-FLOP count 4*d*pairs forward, 10*d*pairs
+ * backward).
+ */
+int flashmask_count_unmasked(const int32_t* lts, const int32_t* lte, const int32_t* uts, const int32_t* ute,
+                             const flashmask_dims* dims, int64_t* pairs, void* stream);
+
+/* Synchronises the current device, returns its status word (0 or a negative
+ * FLASHMASK_ERR_* code written by a kernel) and resets it to 0. */
+int flashmask_get_status(void);
+
+/* Sets the limit of every bounded device-side wait, in nanoseconds (default
+ * 2e9).  Values <= 0 restore the default.  Host-side setting, process-wide. */
+void flashmask_set_wait_limit_ns(int64_t ns);
+
+/* Launches one CTA whose only job is a bounded wait on a barrier that nothing
+ * arrives on; the wait gives up after `limit_ns` and records
+ * FLASHMASK_ERR_TIMEOUT in the status word.  Used to test the failure path
+ * without hanging or faulting the GPU. */
+int flashmask_test_wait_timeout(int64_t limit_ns, void* stream);
+
+/* Human-readable text of an error code (static storage). */
+const char* flashmask_strerror(int code);
+
+/* Library version, 10000 * major + 100 * minor + patch. */
+int flashmask_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FLASHMASK_H_ */

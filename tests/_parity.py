@@ -1,0 +1,70 @@
+"""Shared helpers of the GPU parity tests: input construction and comparisons.
+
+Tolerances: max |err| <= 2e-2 for O, dQ, dK, dV and <= 1e-3 for LSE (natural
+log units); -inf LSE (row with no visible key) must match -inf exactly.
+"""
+import numpy as np
+import torch
+
+from column_sparse_masked_b200 import workloads as wl
+
+TOL_OUT = 2e-2
+TOL_LSE = 1e-3
+
+
+def make_case(B, Nq, Nk, Hq, Hkv, Hm, d, kind, seed):
+    """CPU bf16 tensors and int32 mask vectors [B, Hm, Nk] for a test case."""
+    rng = np.random.default_rng(seed)
+    q = wl.randn_bf16((B, Nq, Hq, d), seed)
+    k = wl.randn_bf16((B, Nk, Hkv, d), seed + 1)
+    v = wl.randn_bf16((B, Nk, Hkv, d), seed + 2)
+    do = wl.randn_bf16((B, Nq, Hq, d), seed + 3)
+    vecs = [np.zeros((B, Hm, Nk), np.int32) for _ in range(4)]
+    for b in range(B):
+        for hm in range(Hm):
+            if kind == "none":
+                vv = wl.empty_vectors(Nk)
+            elif kind == "causal":
+                vv = wl.causal_vectors(Nk)
+            elif kind == "doc":
+                vv = wl.causal_document_vectors(wl.doc_lengths_uniform(rng, Nk, 50, 400))
+            elif kind == "random":
+                vv = wl.random_interval_vectors(rng, Nq, Nk)
+            elif kind == "fullrows":  # rows [5, 140) see nothing
+                vv = [np.full(Nk, 5, np.int32), np.full(Nk, 140, np.int32), np.zeros(Nk, np.int32),
+                      np.zeros(Nk, np.int32)]
+            elif kind == "blocksparse":
+                vv = wl.drop_key_tiles(wl.causal_document_vectors(wl.doc_lengths_uniform(rng, Nk, 100, 700)),
+                                       rng, 0.3)
+            else:
+                raise ValueError(kind)
+            for t in range(4):
+                vecs[t][b, hm] = vv[t]
+    masks = [torch.from_numpy(x) for x in vecs]
+    return q, k, v, do, masks
+
+
+def cuda(*ts):
+    return [None if t is None else t.cuda() for t in ts]
+
+
+def max_err(gpu: torch.Tensor, ref: np.ndarray) -> float:
+    g = gpu.detach().float().cpu().numpy().astype(np.float64)
+    return float(np.abs(g - ref).max()) if g.size else 0.0
+
+
+def check_lse(gpu: torch.Tensor, ref: np.ndarray, tol=TOL_LSE):
+    g = gpu.detach().cpu().numpy().astype(np.float64)
+    ninf_g, ninf_r = np.isneginf(g), np.isneginf(ref)
+    assert np.array_equal(ninf_g, ninf_r), f"-inf pattern differs at {np.argwhere(ninf_g != ninf_r)[:5]}"
+    fin = ~ninf_r
+    err = float(np.abs(g[fin] - ref[fin]).max()) if fin.any() else 0.0
+    assert err <= tol, f"LSE max err {err}"
+    return err
+
+
+def check_out(name, gpu, ref, tol=TOL_OUT):
+    err = max_err(gpu, ref)
+    assert np.isfinite(gpu.detach().float().cpu().numpy()).all(), f"{name} has non-finite values"
+    assert err <= tol, f"{name} max err {err}"
+    return err

@@ -1,0 +1,168 @@
+"""GPU parity: CUDA path (through the C ABI) vs the CPU oracle, element by
+element, on seeded inputs that span several 128-tiles with ragged tails,
+GQA, per-head masks, unmasked/causal/document/random/block-sparse masks and
+fully masked rows.  Classification, localisation and pair counts bit-exact."""
+import numpy as np
+import pytest
+import torch
+
+import column_sparse_masked_b200 as fm
+from column_sparse_masked_b200 import workloads as wl
+
+from _parity import TOL_LSE, TOL_OUT, check_lse, check_out, cuda, make_case
+
+pytestmark = pytest.mark.gpu
+
+# (B, Nq, Nk, Hq, Hkv, Hm, d, mask kind, seed)
+CASES = [
+    (1, 256, 256, 2, 2, 1, 128, "causal", 11),
+    (1, 384, 384, 2, 1, 1, 64, "none", 12),
+    (1, 300, 300, 2, 1, 1, 64, "random", 13),
+    (2, 517, 389, 4, 2, 1, 128, "random", 14),
+    (1, 640, 640, 4, 4, 4, 128, "random", 15),
+    (1, 1000, 1000, 4, 2, 1, 128, "doc", 16),
+    (1, 200, 200, 2, 2, 1, 64, "fullrows", 17),
+    (1, 1100, 1100, 2, 1, 1, 128, "blocksparse", 18),
+    (1, 129, 1, 2, 2, 1, 128, "random", 19),
+    (1, 1, 300, 2, 2, 1, 128, "random", 20),
+]
+
+
+def _ids(c):
+    return f"B{c[0]}_q{c[1]}_k{c[2]}_h{c[3]}-{c[4]}-m{c[5]}_d{c[6]}_{c[7]}"
+
+
+@pytest.fixture(scope="module")
+def oracle_mod():
+    import oracle
+
+    oracle.build_oracle()
+    return oracle
+
+
+@pytest.mark.parametrize("case", CASES, ids=_ids)
+def test_forward_backward_parity(oracle_mod, case):
+    B, Nq, Nk, Hq, Hkv, Hm, d, kind, seed = case
+    q, k, v, do, masks = make_case(*case)
+    qg, kg, vg, dog = cuda(q, k, v, do)
+    mg = cuda(*masks)
+    o, lse = fm.fwd(qg, kg, vg, *mg)
+    dq, dk, dv = fm.bwd(qg, kg, vg, o, lse, dog, *mg)
+    torch.cuda.synchronize()
+    assert fm.get_status() == 0
+    ro, rl = oracle_mod.attention_forward(q, k, v, *masks)
+    check_out("O", o, ro)
+    check_lse(lse, rl)
+    rdq, rdk, rdv = oracle_mod.attention_backward(q, k, v, do, *masks)
+    check_out("dQ", dq, rdq)
+    check_out("dK", dk, rdk)
+    check_out("dV", dv, rdv)
+
+
+def test_forward_is_deterministic():
+    q, k, v, do, masks = make_case(1, 700, 700, 4, 2, 1, 128, "random", 31)
+    qg, kg, vg = cuda(q, k, v)
+    mg = cuda(*masks)
+    o1, l1 = fm.fwd(qg, kg, vg, *mg)
+    o2, l2 = fm.fwd(qg, kg, vg, *mg)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_none_pairs_mean_empty(oracle_mod):
+    q, k, v, do, masks = make_case(1, 333, 333, 2, 2, 1, 128, "causal", 41)
+    qg, kg, vg = cuda(q, k, v)
+    mg = cuda(*masks)
+    o_a, l_a = fm.fwd(qg, kg, vg, None, None, mg[2], mg[3])
+    z = torch.zeros_like(mg[0])
+    o_b, l_b = fm.fwd(qg, kg, vg, z, z, mg[2], mg[3])
+    assert torch.equal(o_a, o_b) and torch.equal(l_a, l_b)
+
+
+def test_empty_inputs():
+    q, k, v, do, masks = make_case(1, 256, 256, 2, 2, 1, 128, "causal", 51)
+    # Nk = 0: every row sees nothing -> O = 0, LSE = -inf, dQ = 0
+    qg = q.cuda()
+    k0 = torch.empty(1, 0, 2, 128, dtype=torch.bfloat16, device="cuda")
+    m0 = [torch.empty(1, 1, 0, dtype=torch.int32, device="cuda") for _ in range(4)]
+    o, lse = fm.fwd(qg, k0, k0, *m0)
+    assert torch.all(o == 0) and torch.all(torch.isneginf(lse))
+    dq, dk, dv = fm.bwd(qg, k0, k0, o, lse, do.cuda(), *m0)
+    assert torch.all(dq == 0) and dk.numel() == 0
+    # Nq = 0: dK = dV = 0
+    q0 = torch.empty(1, 0, 2, 128, dtype=torch.bfloat16, device="cuda")
+    o0, l0 = fm.fwd(q0, k.cuda(), v.cuda(), *cuda(*masks))
+    dq, dk, dv = fm.bwd(q0, k.cuda(), v.cuda(), o0, l0, q0, *cuda(*masks))
+    assert torch.all(dk == 0) and torch.all(dv == 0)
+    torch.cuda.synchronize()
+    assert fm.get_status() == 0
+
+
+@pytest.mark.parametrize("seed", range(4))
+def test_classify_bit_exact(oracle_mod, seed):
+    rng = np.random.default_rng(600 + seed)
+    nq, nk = int(rng.integers(1, 1500)), int(rng.integers(1, 1500))
+    vecs = [np.stack([x for x in wl.random_interval_vectors(rng, nq, nk, p_empty=0.4)])]
+    vecs = [torch.from_numpy(np.ascontiguousarray(vecs[0][t][None, None])) for t in range(4)]
+    got = fm.classify(*cuda(*vecs), Nq=nq).cpu().numpy()
+    ref = oracle_mod.classify(*vecs, nq, nk)
+    assert np.array_equal(got, ref)
+
+
+@pytest.mark.parametrize("name", wl.CONFIG_ORDER)
+def test_classify_configs_bit_exact(oracle_mod, name):
+    w = wl.CONFIGS[name]
+    vecs = [torch.from_numpy(x) for x in wl.mask_vectors(w)]
+    got = fm.classify(*cuda(*vecs), Nq=w.N).cpu().numpy()
+    ref = oracle_mod.classify(*vecs, w.N, w.N)
+    assert np.array_equal(got, ref)
+
+
+@pytest.mark.parametrize("seed", range(3))
+def test_localize_bit_exact(oracle_mod, seed):
+    rng = np.random.default_rng(700 + seed)
+    x = torch.from_numpy(rng.integers(-5, 5000, size=(3, 1, 1000)).astype(np.int32))
+    for a, b in ((0, 1000), (128, 1024), (300, 301), (4000, 4000), (17, 3999)):
+        got = fm.localize(x.cuda(), a, b).cpu().numpy()
+        assert np.array_equal(got, oracle_mod.localize(x, a, b))
+    chunks = [(0, 100), (250, 900), (1000, 1200), (3000, 4096)]
+    got = fm.localize_multi(x.cuda(), chunks).cpu().numpy()
+    assert np.array_equal(got, oracle_mod.localize_multi(x, chunks))
+
+
+@pytest.mark.parametrize("name", ["tiny_doc", "doc8k", "sharequestion32k"])
+def test_count_unmasked_matches_oracle(oracle_mod, name):
+    w = wl.CONFIGS[name]
+    vecs = [torch.from_numpy(x) for x in wl.mask_vectors(w)]
+    got = fm.count_unmasked(*cuda(*vecs), Nq=w.N, Hq=w.Hq)
+    assert got == oracle_mod.count_unmasked(*vecs, w.N, w.N, w.Hq)
+
+
+def test_count_unmasked_random(oracle_mod):
+    rng = np.random.default_rng(9)
+    vv = wl.random_interval_vectors(rng, 500, 700)
+    vecs = [torch.from_numpy(np.ascontiguousarray(np.stack([x, x[::-1]])[:, None])) for x in vv]
+    got = fm.count_unmasked(*cuda(*vecs), Nq=500, Hq=3)
+    assert got == oracle_mod.count_unmasked(*vecs, 500, 700, 3)
+
+
+def test_bounded_wait_timeout_reports_status():
+    """A wait on a barrier that nothing arrives on gives up and records the timeout."""
+    assert fm.get_status() == 0
+    fm.test_wait_timeout(2_000_000)  # 2 ms
+    assert fm.get_status() == -6
+    assert fm.get_status() == 0  # cleared
+    q, k, v, do, masks = make_case(1, 256, 256, 2, 2, 1, 128, "causal", 61)
+    o, lse = fm.fwd(*cuda(q, k, v), *cuda(*masks))
+    torch.cuda.synchronize()
+    assert fm.get_status() == 0 and torch.isfinite(lse).all()
+
+
+def test_autograd_wrapper(oracle_mod):
+    q, k, v, do, masks = make_case(1, 300, 300, 2, 2, 1, 128, "doc", 71)
+    qg, kg, vg = [t.cuda().requires_grad_(True) for t in (q, k, v)]
+    o = fm.flashmask_attention(qg, kg, vg, *cuda(*masks))
+    o.backward(do.cuda())
+    rdq, rdk, rdv = oracle_mod.attention_backward(q, k, v, do, *masks)
+    check_out("dQ", qg.grad, rdq)
+    check_out("dK", kg.grad, rdk)
+    check_out("dV", vg.grad, rdv)
