@@ -1,0 +1,373 @@
+#!/usr/bin/env python
+"""FlashMask forward+backward benchmark on B200: effective TFLOP/s over unmasked pairs.
+
+One step = one forward (``flashmask_fwd``) and one backward (``flashmask_bwd``)
+over one batch of the workload, through the library's C ABI.  Effective FLOPs
+count only unmasked (i, j) pairs: 4*d*pairs forward, 10*d*pairs backward
+(pairs from the library's closed-form count).  The default workload is the
+8K causal-document mask with 32 query / 8 KV heads, head_dim 128.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config NAME]
+
+N > 1 runs under torchrun as independent replicas (one per GPU, no data-path
+collective; the path has no exchange step): value = all ranks' FLOPs / max
+over ranks of the device time.  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from column_sparse_masked_b200 import workloads as wl  # noqa: E402
+
+METRIC = "FlashMask fwd+bwd effective TFLOP/s (unmasked FLOPs only), % of B200 bf16 peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+CPU_SAMPLE_ROWS = 8192  # bounded oracle sample: first rows/keys of (batch 0, q-head 0)
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="doc8k", choices=wl.CONFIG_ORDER)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return json.load(f), "MEASURED_PEAKS.json"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples every 200 ms while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-i", str(self.gpu), "-lms", "200"], stdout=self.f,
+                                         stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        out = {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        if self.proc is None:
+            return out
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(n)
+        os.unlink(self.path)
+        if sm:
+            out.update(sm_mhz=statistics.median(sm), sm_max_mhz=max(mx), reasons=sorted(reasons), samples=len(sm))
+        return out
+
+
+def effective_flops(pairs: int, d: int):
+    return 4.0 * d * pairs, 10.0 * d * pairs
+
+
+def kernel_source_hash(name: str) -> str:
+    with open(os.path.join(ROOT, "column_sparse_masked_b200", "csrc", name), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def recorded_traffic(kernel_file: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it matches the current kernel source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f)
+    e = rec.get(kernel_file, {}).get(workload)
+    if not e or e.get("source_sha256_16") != kernel_source_hash(kernel_file):
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ----------------------------------------------------------------------------
+# CPU oracle leg (bounded sample) -- the only place bench.py executes oracle/
+# ----------------------------------------------------------------------------
+def oracle_sample(w: wl.Workload, rows: int, inp=None):
+    """(b=0, q-head 0) restricted to its first `rows` queries and keys (mask localised onto [0, rows))."""
+    import oracle
+
+    full = wl.make_inputs(w, with_grad=True) if inp is None else inp
+    n = min(rows, w.N)
+    q = full["q"][:1, :n, :1].contiguous()
+    k = full["k"][:1, :n, :1].contiguous()
+    v = full["v"][:1, :n, :1].contiguous()
+    do = full["do"][:1, :n, :1].contiguous()
+    vecs = [oracle.localize(full[m][:1, :1, :n].numpy(), 0, n) for m in ("lts", "lte", "uts", "ute")]
+    pairs = oracle.count_unmasked(*vecs, n, n, 1)
+    return q, k, v, do, vecs, pairs, n
+
+
+def run_oracle_step(sample):
+    import oracle
+
+    q, k, v, do, vecs, pairs, n = sample
+    t0 = time.perf_counter()
+    oracle.attention_forward(q, k, v, *vecs)
+    oracle.attention_backward(q, k, v, do, *vecs)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(w: wl.Workload, rows: int = CPU_SAMPLE_ROWS, inp=None):
+    import oracle
+
+    sample = oracle_sample(w, rows, inp)
+    dt = run_oracle_step(sample)
+    pairs, n = sample[5], sample[6]
+    ff, fb = effective_flops(pairs, w.d)
+    return {"value": (ff + fb) / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "seconds": dt,
+            "sample": f"{w.name}: batch 0, q-head 0 with its KV head, first {n} queries x {n} keys "
+                      f"(mask localised onto [0,{n})), fp64 fwd+bwd, {pairs} unmasked pairs"}
+
+
+# ----------------------------------------------------------------------------
+# our arm
+# ----------------------------------------------------------------------------
+def run_ours(args, rank, world, local_rank):
+    import column_sparse_masked_b200 as fm
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = wl.CONFIGS[args.config]
+    inp = wl.make_inputs(w, with_grad=True)
+    names = ("q", "k", "v", "do", "lts", "lte", "uts", "ute")
+    host = {n: inp[n].pin_memory() for n in names}
+    d_in = {n: host[n].to(dev) for n in names}
+    masks = [d_in[n] for n in ("lts", "lte", "uts", "ute")]
+    pairs = fm.count_unmasked(*masks, Nq=w.N, Hq=w.Hq)
+    f_fwd, f_bwd = effective_flops(pairs, w.d)
+    o = torch.empty_like(d_in["q"])
+    lse = torch.empty(w.B, w.Hq, w.N, dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(d_in["q"]), torch.empty_like(d_in["k"]), torch.empty_like(d_in["v"])
+    ws = torch.empty(fm.workspace_size("bwd", w.B, w.Hq, w.Hkv, 1, w.N, w.N, w.d), dtype=torch.uint8, device=dev)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+
+    def step(src):
+        fm.fwd(src["q"], src["k"], src["v"], *[src[n] for n in ("lts", "lte", "uts", "ute")], out=(o, lse),
+               workspace=ws)
+        fm.bwd(src["q"], src["k"], src["v"], o, lse, src["do"], *[src[n] for n in ("lts", "lte", "uts", "ute")],
+               out=(dq, dk, dv), workspace=ws)
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        step(d_in)
+    torch.cuda.synchronize()
+    assert fm.get_status() == 0, "device status word set during warm-up"
+
+    # ---- device-resident timing ----
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    vis = [x for x in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if x.strip()]
+    clocks = ClockSampler(vis[local_rank] if local_rank < len(vis) else str(local_rank))
+    barrier(world)
+    torch.cuda.synchronize()
+    launches0 = fm.launch_count()
+    fm.profiler_read()
+    fm.profiler_enable(True)
+    clocks.start()
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        evs[i][0].record()
+        step(d_in)
+        evs[i][1].record()
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    fm.profiler_enable(False)
+    prof = fm.profiler_read()
+    launches = fm.launch_count() - launches0
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    local_ms = sum(step_ms)
+    total_ms = max_over_ranks(local_ms, world, dev)
+    assert fm.get_status() == 0, "device status word set during the timed steps"
+    value = world * (f_fwd + f_bwd) * args.steps / (total_ms / 1e3) / 1e12
+
+    # ---- end to end: host buffers, copies inside the timed region ----
+    h_out = {"o": torch.empty_like(o, device="cpu").pin_memory(),
+             "lse": torch.empty_like(lse, device="cpu").pin_memory(),
+             "dq": torch.empty_like(dq, device="cpu").pin_memory(),
+             "dk": torch.empty_like(dk, device="cpu").pin_memory(),
+             "dv": torch.empty_like(dv, device="cpu").pin_memory()}
+    d_e2e = {n: torch.empty_like(d_in[n]) for n in names}
+
+    def e2e_step():
+        for n in names:
+            d_e2e[n].copy_(host[n], non_blocking=True)
+        step(d_e2e)
+        for n, t in (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv)):
+            h_out[n].copy_(t, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    e_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.fill_(i & 0xFF)
+        e_evs[i][0].record()
+        e2e_step()
+        e_evs[i][1].record()
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e_evs), world, dev)
+    h2d = sum(host[n].numel() * host[n].element_size() for n in names)
+    d2h = sum(t.numel() * t.element_size() for t in h_out.values())
+
+    # ---- roofline of the dominant kernel ----
+    peaks, peak_src = load_peaks()
+    kinds = {"fwd": (prof["fwd_ms"], prof["fwd_launches"], f_fwd, "fwd_sm100.cu", f"fm_fwd_kernel<{w.d}>"),
+             "bwd": (prof["bwd_ms"], prof["bwd_launches"], f_bwd, "bwd_sm100.cu", f"fm_bwd_kernel<{w.d}>")}
+    dom = max(kinds, key=lambda k: kinds[k][0])
+    ms, nl, fl, src, kname = kinds[dom]
+    achieved = fl / (ms / nl / 1e3) / 1e12 if nl else None
+    peak = float(peaks["bf16_tflops"])
+    roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+            "frac": (achieved / peak) if achieved else None,
+            "traffic": recorded_traffic(src, w.name), "kernel": kname,
+            "kernel_ms_per_launch": ms / nl if nl else None,
+            "peak_source": f"{peak_src} bf16_tflops (burst, cuBLAS bf16)",
+            "fwd_kernel_tflops": (f_fwd / (prof["fwd_ms"] / prof["fwd_launches"] / 1e3) / 1e12)
+            if prof["fwd_launches"] else None,
+            "bwd_kernel_tflops": (f_bwd / (prof["bwd_ms"] / prof["bwd_launches"] / 1e3) / 1e12)
+            if prof["bwd_launches"] else None,
+            "kernel_share_of_step": (prof["fwd_ms"] + prof["bwd_ms"]) / local_ms if local_ms else None}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "pct_of_bf16_peak": 100.0 * value / world / peak,
+        "config": {"workload": w.name, "description": w.description, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv,
+                   "seqlen": w.N, "head_dim": w.d, "unmasked_pairs": pairs,
+                   "flops_per_step": {"fwd": f_fwd, "bwd": f_bwd},
+                   "l2": "flushed before every step (2x L2 bytes written, outside the step's events)",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "e2e": {"value": world * (f_fwd + f_bwd) * args.steps / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.steps},
+        "roofline": roof,
+        "gpu_launches": launches,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, inp=inp)
+    return line
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    import oracle
+
+    w = wl.CONFIGS[args.config]
+    rows = 4096
+    sample = oracle_sample(w, rows)
+    pairs, n = sample[5], sample[6]
+    ff, fb = effective_flops(pairs, w.d)
+    for _ in range(args.warmup):
+        run_oracle_step(sample)
+    times = [run_oracle_step(sample) for _ in range(args.steps)]
+    total = sum(times)
+    v = (ff + fb) * args.steps / total / 1e12
+    desc = (f"{w.name}: batch 0, q-head 0 with its KV head, first {n} queries x {n} keys "
+            f"(mask localised onto [0,{n})), fp64 fwd+bwd per step, {pairs} unmasked pairs")
+    return {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "sample_rows": n, "unmasked_pairs_per_step": pairs},
+        "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse_args()
+    rank, world, local_rank = dist_env()
+    if world > 1 and args.impl == "ours":
+        from datetime import timedelta
+
+        torch.distributed.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_ours(args, rank, world, local_rank) if args.impl == "ours" else run_reference(args, rank, world)
+        if rank == 0 and line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1 and torch.distributed.is_initialized():
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -25,10 +25,13 @@ from ._binding import (  # noqa: F401
     fwd,
     bwd,
     get_status,
+    launch_count,
     lib_path,
     load_library,
     localize,
     localize_multi,
+    profiler_enable,
+    profiler_read,
     set_wait_limit_ns,
     test_wait_timeout,
     version,
@@ -37,6 +40,6 @@ from ._binding import (  # noqa: F401
 
 __all__ = [
     "FlashMaskError", "classify", "count_unmasked", "flashmask_attention", "fwd", "bwd", "get_status",
-    "lib_path", "load_library", "localize", "localize_multi", "set_wait_limit_ns", "test_wait_timeout",
+    "launch_count", "lib_path", "load_library", "localize", "localize_multi", "profiler_enable", "profiler_read", "set_wait_limit_ns", "test_wait_timeout",
     "version", "workspace_size",
 ]

@@ -28,6 +28,9 @@ _SIGS = {
     "flashmask_get_status": (ctypes.c_int, []),
     "flashmask_set_wait_limit_ns": (None, [ctypes.c_int64]),
     "flashmask_test_wait_timeout": (ctypes.c_int, [ctypes.c_int64, _P]),
+    "flashmask_profiler_enable": (ctypes.c_int, [ctypes.c_int]),
+    "flashmask_profiler_read": (ctypes.c_int, [_P, _P, _P, _P]),
+    "flashmask_launch_count": (ctypes.c_int64, []),
     "flashmask_strerror": (ctypes.c_char_p, [ctypes.c_int]),
     "flashmask_version": (ctypes.c_int, []),
 }
@@ -233,6 +236,25 @@ def test_wait_timeout(limit_ns: int, device=None) -> None:
     dev = torch.device("cuda") if device is None else torch.device(device)
     _check(load_library().flashmask_test_wait_timeout(ctypes.c_int64(int(limit_ns)), _stream(dev)),
            "flashmask_test_wait_timeout")
+
+
+def profiler_enable(on: bool = True) -> None:
+    """Brackets every attention-kernel launch with CUDA events (for benchmarks)."""
+    _check(load_library().flashmask_profiler_enable(1 if on else 0), "flashmask_profiler_enable")
+
+
+def profiler_read():
+    """Returns {'fwd_ms', 'fwd_launches', 'bwd_ms', 'bwd_launches'} since the last read."""
+    fm, bm = ctypes.c_double(0), ctypes.c_double(0)
+    fl, bl = ctypes.c_int64(0), ctypes.c_int64(0)
+    _check(load_library().flashmask_profiler_read(ctypes.byref(fm), ctypes.byref(fl), ctypes.byref(bm),
+                                                  ctypes.byref(bl)), "flashmask_profiler_read")
+    return {"fwd_ms": fm.value, "fwd_launches": fl.value, "bwd_ms": bm.value, "bwd_launches": bl.value}
+
+
+def launch_count() -> int:
+    """Kernels launched by the library since process start."""
+    return int(load_library().flashmask_launch_count())
 
 
 class _FlashMaskFn(torch.autograd.Function):

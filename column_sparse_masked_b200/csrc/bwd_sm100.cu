@@ -491,7 +491,10 @@ static cudaError_t launch_bwd_d(const BwdParams& p, const CUtensorMap& tq, const
   const int smem = (int)sizeof(BwdSmem<D>);
   cudaError_t e = ensure_smem_limit((const void*)fm_bwd_kernel<D>, smem);
   if (e != cudaSuccess) return e;
+  profile_begin(1, st);
+  note_launch();
   fm_bwd_kernel<D><<<grid, BwdCfg<D>::kThreads, smem, st>>>(tq, tk, tv, tdo, p);
+  profile_end(1, st);
   return cudaGetLastError();
 }
 
@@ -507,9 +510,11 @@ cudaError_t launch_bwd_pre(const BwdPreParams& p, cudaStream_t st) {
   int64_t blocks = (rows * 32 + 255) / 256;
   if (blocks > 148 * 64) blocks = 148 * 64;
   if (p.s.d == 128)
-    fm_bwd_pre_kernel<128><<<(unsigned)blocks, 256, 0, st>>>(p);
+    { note_launch(); fm_bwd_pre_kernel<128><<<(unsigned)blocks, 256, 0, st>>>(p);
+    }
   else
-    fm_bwd_pre_kernel<64><<<(unsigned)blocks, 256, 0, st>>>(p);
+    { note_launch(); fm_bwd_pre_kernel<64><<<(unsigned)blocks, 256, 0, st>>>(p);
+    }
   return cudaGetLastError();
 }
 
@@ -517,7 +522,8 @@ cudaError_t launch_dq_finalize(const DqFinParams& p, cudaStream_t st) {
   if (p.n == 0) return cudaSuccess;
   int64_t blocks = (p.n / 4 + 255) / 256;
   if (blocks > 148 * 32) blocks = 148 * 32;
-  fm_dq_finalize_kernel<<<(unsigned)blocks, 256, 0, st>>>(p);
+  { note_launch(); fm_dq_finalize_kernel<<<(unsigned)blocks, 256, 0, st>>>(p);
+  }
   return cudaGetLastError();
 }
 

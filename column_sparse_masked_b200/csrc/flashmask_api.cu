@@ -9,9 +9,11 @@
 #include <climits>
 #include <cmath>
 #include <cstdint>
+#include <cstdio>
 #include <cstring>
 #include <mutex>
 #include <unordered_map>
+#include <vector>
 
 #include "../../include/flashmask.h"
 #include "common.cuh"
@@ -25,6 +27,7 @@ __device__ int g_status_word;
 namespace {
 
 std::atomic<int64_t> g_wait_limit_ns{2000000000LL};
+thread_local char g_last_cuda_error[256] = "";
 std::mutex g_mu;
 
 struct DeviceInfo {
@@ -36,6 +39,10 @@ struct DeviceInfo {
 int current_device(DeviceInfo* out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return FLASHMASK_ERR_NO_DEVICE;
+  // Binds the device's primary context to the calling thread: a thread that
+  // has made no CUDA call yet (an autograd worker, a user thread) has none,
+  // and tensor-map encoding needs one.
+  if (cudaSetDevice(dev) != cudaSuccess) return FLASHMASK_ERR_NO_DEVICE;
   static std::unordered_map<int, DeviceInfo> cache;
   std::lock_guard<std::mutex> lock(g_mu);
   auto it = cache.find(dev);
@@ -80,7 +87,9 @@ int make_map(CUtensorMap* m, const void* ptr, int B, int N, int H, int d) {
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, es,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? FLASHMASK_OK : FLASHMASK_ERR_CUDA;
+  if (r == CUDA_SUCCESS) return FLASHMASK_OK;
+  snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "cuTensorMapEncodeTiled failed (CUresult %d)", (int)r);
+  return FLASHMASK_ERR_CUDA;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -114,14 +123,19 @@ int check_ws(const void* ws, size_t have, size_t need) {
   return FLASHMASK_OK;
 }
 
-int cuda_status(cudaError_t e) { return e == cudaSuccess ? FLASHMASK_OK : FLASHMASK_ERR_CUDA; }
+int cuda_status(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return FLASHMASK_OK;
+  snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "CUDA runtime or launch failure in %s: %s", what,
+           cudaGetErrorString(e));
+  return FLASHMASK_ERR_CUDA;
+}
 
 #define FM_TRY(x)                       \
   do {                                  \
     int _rc = (x);                      \
     if (_rc != FLASHMASK_OK) return _rc; \
   } while (0)
-#define FM_CUDA(x) FM_TRY(cuda_status(x))
+#define FM_CUDA(x) FM_TRY(cuda_status((x), #x))
 
 float resolve_scale(float scale, int d) { return scale > 0.f ? scale : 1.0f / std::sqrt((float)d); }
 
@@ -137,7 +151,51 @@ MaskPrepParams prep_params(const Shape& s, const WsLayout& L, uint8_t* ws, const
   return mp;
 }
 
+// ---- launch counter and kernel profiler ----
+std::atomic<int64_t> g_launches{0};
+std::atomic<int> g_profiling{0};
+struct ProfRec {
+  cudaEvent_t start = nullptr, stop = nullptr;
+  int kind = 0;
+};
+std::vector<ProfRec> g_prof_pool;  // guarded by g_mu
+size_t g_prof_used = 0;
+constexpr size_t kProfMax = 4096;
+
 }  // namespace
+
+void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+// A begin/end pair is recorded only while profiling is on; `end` closes the
+// record opened by the matching `begin` of the same thread (launches of the
+// library are issued from one thread per call).
+thread_local ProfRec* t_open_rec = nullptr;
+
+void profile_begin(int kind, cudaStream_t st) {
+  t_open_rec = nullptr;
+  if (!g_profiling.load(std::memory_order_relaxed)) return;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (g_prof_used >= kProfMax) return;
+  if (g_prof_used == g_prof_pool.size()) {
+    ProfRec r;
+    if (cudaEventCreate(&r.start) != cudaSuccess || cudaEventCreate(&r.stop) != cudaSuccess) return;
+    g_prof_pool.push_back(r);
+  }
+  ProfRec* r = &g_prof_pool[g_prof_used++];
+  r->kind = kind;
+  if (cudaEventRecord(r->start, st) != cudaSuccess) {
+    --g_prof_used;
+    return;
+  }
+  t_open_rec = r;
+}
+
+void profile_end(int kind, cudaStream_t st) {
+  if (!t_open_rec) return;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (t_open_rec->kind == kind) cudaEventRecord(t_open_rec->stop, st);
+  t_open_rec = nullptr;
+}
 
 cudaError_t ensure_smem_limit(const void* func, int bytes) {
   int dev = 0;
@@ -420,6 +478,36 @@ int flashmask_test_wait_timeout(int64_t limit_ns, void* stream) {
   return FLASHMASK_OK;
 }
 
+int flashmask_profiler_enable(int on) {
+  g_profiling.store(on ? 1 : 0);
+  return FLASHMASK_OK;
+}
+
+int flashmask_profiler_read(double* fwd_ms, int64_t* fwd_launches, double* bwd_ms, int64_t* bwd_launches) {
+  std::lock_guard<std::mutex> lock(g_mu);
+  double ms[2] = {0.0, 0.0};
+  int64_t cnt[2] = {0, 0};
+  int rc = FLASHMASK_OK;
+  for (size_t i = 0; i < g_prof_used; ++i) {
+    ProfRec& r = g_prof_pool[i];
+    float t = 0.f;
+    if (cudaEventSynchronize(r.stop) != cudaSuccess || cudaEventElapsedTime(&t, r.start, r.stop) != cudaSuccess) {
+      rc = FLASHMASK_ERR_CUDA;
+      continue;
+    }
+    ms[r.kind & 1] += t;
+    cnt[r.kind & 1] += 1;
+  }
+  g_prof_used = 0;
+  if (fwd_ms) *fwd_ms = ms[0];
+  if (fwd_launches) *fwd_launches = cnt[0];
+  if (bwd_ms) *bwd_ms = ms[1];
+  if (bwd_launches) *bwd_launches = cnt[1];
+  return rc;
+}
+
+int64_t flashmask_launch_count(void) { return g_launches.load(); }
+
 const char* flashmask_strerror(int code) {
   switch (code) {
     case FLASHMASK_OK: return "ok";
@@ -427,7 +515,8 @@ const char* flashmask_strerror(int code) {
     case FLASHMASK_ERR_UNSUPPORTED: return "unsupported configuration (head_dim must be 64 or 128; sizes too large)";
     case FLASHMASK_ERR_ALIGN: return "pointer not 16-byte aligned (workspace: 256-byte)";
     case FLASHMASK_ERR_WORKSPACE: return "workspace missing or too small";
-    case FLASHMASK_ERR_CUDA: return "CUDA runtime or launch failure";
+    case FLASHMASK_ERR_CUDA:
+      return g_last_cuda_error[0] ? g_last_cuda_error : "CUDA runtime or launch failure";
     case FLASHMASK_ERR_TIMEOUT: return "a device-side bounded wait timed out";
     case FLASHMASK_ERR_NO_DEVICE: return "no sm_100 (B200-class) device is current";
     default: return "unknown error code";

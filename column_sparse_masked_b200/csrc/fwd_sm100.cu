@@ -418,7 +418,10 @@ static cudaError_t launch_fwd_d(const FwdParams& p, const CUtensorMap& tq, const
   const int smem = (int)sizeof(FwdSmem<D>);
   cudaError_t e = ensure_smem_limit((const void*)fm_fwd_kernel<D>, smem);
   if (e != cudaSuccess) return e;
+  profile_begin(0, st);
+  note_launch();
   fm_fwd_kernel<D><<<grid, FwdCfg<D>::kThreads, smem, st>>>(tq, tk, tv, p);
+  profile_end(0, st);
   return cudaGetLastError();
 }
 

@@ -26,6 +26,12 @@ cudaError_t launch_bwd(const BwdParams& p, const CUtensorMap& tq, const CUtensor
                        const CUtensorMap& tdo, int grid, cudaStream_t st);
 cudaError_t launch_dq_finalize(const DqFinParams& p, cudaStream_t st);
 
+// Launch bookkeeping: counts every launch; brackets the attention kernels
+// with profiler events when profiling is enabled (kind 0 forward, 1 backward).
+void note_launch();
+void profile_begin(int kind, cudaStream_t st);
+void profile_end(int kind, cudaStream_t st);
+
 // Raises a kernel's dynamic shared-memory limit once per (kernel, device).
 cudaError_t ensure_smem_limit(const void* func, int bytes);
 

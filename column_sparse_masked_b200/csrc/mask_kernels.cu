@@ -297,25 +297,29 @@ __global__ void wait_timeout_kernel(int* status, uint64_t limit_ns) {
 // ----------------------------------------------------------------------------
 cudaError_t launch_mask_prep(const MaskPrepParams& p, cudaStream_t st) {
   if (p.B == 0 || p.Hm == 0 || p.nKt == 0) return cudaSuccess;
-  mask_prep_kernel<<<dim3(p.nKt, p.Hm, p.B), 128, 0, st>>>(p);
+  { note_launch(); mask_prep_kernel<<<dim3(p.nKt, p.Hm, p.B), 128, 0, st>>>(p);
+  }
   return cudaGetLastError();
 }
 
 cudaError_t launch_plan_fwd(const PlanParams& p, cudaStream_t st) {
   if (p.s.B == 0 || p.s.nQB == 0) return cudaSuccess;
-  plan_fwd_kernel<<<dim3(p.s.nQB, p.s.Hm, p.s.B), 128, 0, st>>>(p);
+  { note_launch(); plan_fwd_kernel<<<dim3(p.s.nQB, p.s.Hm, p.s.B), 128, 0, st>>>(p);
+  }
   return cudaGetLastError();
 }
 
 cudaError_t launch_plan_bwd(const PlanParams& p, cudaStream_t st) {
   if (p.s.B == 0 || p.s.nKt == 0) return cudaSuccess;
-  plan_bwd_kernel<<<dim3(p.s.nKt, p.s.Hm, p.s.B), 128, 0, st>>>(p);
+  { note_launch(); plan_bwd_kernel<<<dim3(p.s.nKt, p.s.Hm, p.s.B), 128, 0, st>>>(p);
+  }
   return cudaGetLastError();
 }
 
 cudaError_t launch_classify_export(const PlanParams& p, cudaStream_t st) {
   if (p.s.B == 0 || p.s.nQt == 0 || p.s.nKt == 0) return cudaSuccess;
-  classify_export_kernel<<<dim3(p.s.nQt, p.s.Hm, p.s.B), 128, 0, st>>>(p);
+  { note_launch(); classify_export_kernel<<<dim3(p.s.nQt, p.s.Hm, p.s.B), 128, 0, st>>>(p);
+  }
   return cudaGetLastError();
 }
 
@@ -326,14 +330,16 @@ cudaError_t launch_sort_units(const SortParams& p, cudaStream_t st) {
   const size_t smem = (n <= kSortMax) ? (size_t)np2 * sizeof(unsigned long long) : 0;
   cudaError_t e = ensure_smem_limit((const void*)sort_units_kernel, (int)(kSortMax * sizeof(unsigned long long)));
   if (e != cudaSuccess) return e;
-  sort_units_kernel<<<1, 1024, smem, st>>>(p);
+  { note_launch(); sort_units_kernel<<<1, 1024, smem, st>>>(p);
+  }
   return cudaGetLastError();
 }
 
 cudaError_t launch_localize(const int32_t* in, int32_t* out, int64_t n, int32_t a, int32_t b, cudaStream_t st) {
   if (n == 0) return cudaSuccess;
   const int64_t blocks = (n + 255) / 256;
-  localize_kernel<<<(unsigned)(blocks < 65535 ? blocks : 65535), 256, 0, st>>>(in, out, n, a, b);
+  { note_launch(); localize_kernel<<<(unsigned)(blocks < 65535 ? blocks : 65535), 256, 0, st>>>(in, out, n, a, b);
+  }
   return cudaGetLastError();
 }
 
@@ -347,17 +353,20 @@ cudaError_t launch_localize_multi(const int32_t* in, int32_t* out, int64_t n, co
     c.b[k] = ends[k];
   }
   const int64_t blocks = (n + 255) / 256;
-  localize_multi_kernel<<<(unsigned)(blocks < 65535 ? blocks : 65535), 256, 0, st>>>(in, out, n, c);
+  { note_launch(); localize_multi_kernel<<<(unsigned)(blocks < 65535 ? blocks : 65535), 256, 0, st>>>(in, out, n, c);
+  }
   return cudaGetLastError();
 }
 
 cudaError_t launch_count_unmasked(const MaskPrepParams& p, int Hq, int Nq, int64_t* out, cudaStream_t st) {
-  count_unmasked_kernel<<<1, 1024, 0, st>>>(p, Hq, Nq, out);
+  { note_launch(); count_unmasked_kernel<<<1, 1024, 0, st>>>(p, Hq, Nq, out);
+  }
   return cudaGetLastError();
 }
 
 cudaError_t launch_wait_timeout(int* status, uint64_t limit_ns, cudaStream_t st) {
-  wait_timeout_kernel<<<1, 32, 0, st>>>(status, limit_ns);
+  { note_launch(); wait_timeout_kernel<<<1, 32, 0, st>>>(status, limit_ns);
+  }
   return cudaGetLastError();
 }
 

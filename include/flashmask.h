@@ -152,6 +152,21 @@ void flashmask_set_wait_limit_ns(int64_t ns);
  * without hanging or faulting the GPU. */
 int flashmask_test_wait_timeout(int64_t limit_ns, void* stream);
 
+/*
+ * Kernel timing for benchmarks.  While enabled (on != 0), every launch of the
+ * forward or backward attention kernel is bracketed by a CUDA event pair
+ * recorded on the call's stream.  flashmask_profiler_read() waits for the
+ * recorded events, returns the summed kernel milliseconds and launch counts
+ * of each kind (either output pointer may be NULL) and clears them.  Event
+ * pairs are pooled (at most 4096 outstanding).  Host-side, process-wide.
+ */
+int flashmask_profiler_enable(int on);
+int flashmask_profiler_read(double* fwd_ms, int64_t* fwd_launches, double* bwd_ms, int64_t* bwd_launches);
+
+/* Number of kernels this library has launched since the process started
+ * (every kind: summary, lists, ordering, attention, preprocess, finalise). */
+int64_t flashmask_launch_count(void);
+
 /* Human-readable text of an error code (static storage). */
 const char* flashmask_strerror(int code);
 
