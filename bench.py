@@ -68,6 +68,15 @@ def max_over_ranks(x: float, world: int, device) -> float:
     return float(t.item())
 
 
+def aggregate(local_ms: float, flops_per_step: float, steps: int, world: int, device) -> tuple:
+    """Whole-job throughput of `world` replicas: all ranks' FLOPs / max-over-ranks device time.
+
+    Returns (TFLOP/s, max ms).  Every rank calls it (it holds a collective).
+    """
+    total_ms = max_over_ranks(local_ms, world, device)
+    return world * flops_per_step * steps / (total_ms / 1e3) / 1e12, total_ms
+
+
 def barrier(world: int):
     if world > 1:
         torch.distributed.barrier()
@@ -249,9 +258,8 @@ def run_ours(args, rank, world, local_rank):
     launches = fm.launch_count() - launches0
     step_ms = [a.elapsed_time(b) for a, b in evs]
     local_ms = sum(step_ms)
-    total_ms = max_over_ranks(local_ms, world, dev)
+    value, total_ms = aggregate(local_ms, f_fwd + f_bwd, args.steps, world, dev)
     assert fm.get_status() == 0, "device status word set during the timed steps"
-    value = world * (f_fwd + f_bwd) * args.steps / (total_ms / 1e3) / 1e12
 
     # ---- end to end: host buffers, copies inside the timed region ----
     h_out = {"o": torch.empty_like(o, device="cpu").pin_memory(),
@@ -280,7 +288,7 @@ def run_ours(args, rank, world, local_rank):
         e_evs[i][1].record()
     torch.cuda.synchronize()
     barrier(world)
-    e2e_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in e_evs), world, dev)
+    e2e_value, e2e_ms = aggregate(sum(a.elapsed_time(b) for a, b in e_evs), f_fwd + f_bwd, args.steps, world, dev)
     h2d = sum(host[n].numel() * host[n].element_size() for n in names)
     d2h = sum(t.numel() * t.element_size() for t in h_out.values())
 
@@ -313,7 +321,7 @@ def run_ours(args, rank, world, local_rank):
                    "flops_per_step": {"fwd": f_fwd, "bwd": f_bwd},
                    "l2": "flushed before every step (2x L2 bytes written, outside the step's events)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
-        "e2e": {"value": world * (f_fwd + f_bwd) * args.steps / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.steps},
         "roofline": roof,
         "gpu_launches": launches,
