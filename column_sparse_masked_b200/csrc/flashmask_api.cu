@@ -519,6 +519,9 @@ const char* flashmask_strerror(int code) {
       return g_last_cuda_error[0] ? g_last_cuda_error : "CUDA runtime or launch failure";
     case FLASHMASK_ERR_TIMEOUT: return "a device-side bounded wait timed out";
     case FLASHMASK_ERR_NO_DEVICE: return "no sm_100 (B200-class) device is current";
+    case FLASHMASK_ERR_TOO_LARGE:
+      return "problem too large for flashmask_fwd_noalloc: its forward workspace exceeds "
+             "FLASHMASK_NOALLOC_SCRATCH_BYTES (16 MiB); use flashmask_fwd with a workspace";
     default: return "unknown error code";
   }
 }
@@ -526,3 +529,50 @@ const char* flashmask_strerror(int code) {
 int flashmask_version(void) { return 100; }
 
 }  // extern "C"
+
+// ----------------------------------------------------------------------------
+// Forward without a caller-provided workspace (see flashmask_fwd_noalloc in
+// include/flashmask.h).  For callers that may not allocate device memory once
+// running; the forward's scratch lives in this file-scope device array.
+// ----------------------------------------------------------------------------
+namespace fm {
+namespace {
+
+static __device__ __align__(256) uint8_t g_noalloc_scratch[FLASHMASK_NOALLOC_SCRATCH_BYTES];
+
+// Device address of the array, looked up once per device with that device
+// current.  In host code the array's name is only a host-side stand-in, so
+// the address must come from cudaGetSymbolAddress.
+int noalloc_scratch_address(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FLASHMASK_ERR_NO_DEVICE;
+  static std::unordered_map<int, void*> addr;
+  std::lock_guard<std::mutex> lock(g_mu);
+  auto it = addr.find(dev);
+  if (it == addr.end()) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr) return cuda_status(e == cudaSuccess ? cudaErrorInvalidSymbol : e,
+                                                             "cudaGetSymbolAddress(g_noalloc_scratch)");
+    it = addr.emplace(dev, p).first;
+  }
+  *out = it->second;
+  return FLASHMASK_OK;
+}
+
+}  // namespace
+}  // namespace fm
+
+extern "C" int flashmask_fwd_noalloc(const void* q, const void* k, const void* v, const int32_t* lts,
+                                     const int32_t* lte, const int32_t* uts, const int32_t* ute, float scale,
+                                     const flashmask_dims* dims, void* o, float* lse, void* stream) {
+  FM_TRY(check_dims(dims));
+  const size_t need = flashmask_fwd_workspace_size(dims);
+  if (need > (size_t)FLASHMASK_NOALLOC_SCRATCH_BYTES) return FLASHMASK_ERR_TOO_LARGE;
+  DeviceInfo di;
+  FM_TRY(current_device(&di));  // binds the device's context to this thread first
+  void* scratch = nullptr;
+  FM_TRY(noalloc_scratch_address(&scratch));
+  return flashmask_fwd(q, k, v, lts, lte, uts, ute, scale, dims, o, lse, scratch,
+                       (size_t)FLASHMASK_NOALLOC_SCRATCH_BYTES, stream);
+}

@@ -55,6 +55,7 @@ extern "C" {
 #define FLASHMASK_ERR_CUDA (-5)        /* a CUDA runtime call or launch failed            */
 #define FLASHMASK_ERR_TIMEOUT (-6)     /* a kernel's bounded wait expired (status word)   */
 #define FLASHMASK_ERR_NO_DEVICE (-7)   /* no sm_100 device current                        */
+#define FLASHMASK_ERR_TOO_LARGE (-8)   /* problem needs more than the static no-alloc scratch */
 
 /* Problem shape.  B batch, Hq query heads, Hkv key/value heads, Hm mask heads
  * (1 or Hq), Nq query rows, Nk key columns, d head dimension. */
@@ -78,6 +79,42 @@ size_t flashmask_fwd_workspace_size(const flashmask_dims* dims);
 int flashmask_fwd(const void* q, const void* k, const void* v, const int32_t* lts, const int32_t* lte,
                   const int32_t* uts, const int32_t* ute, float scale, const flashmask_dims* dims, void* o,
                   float* lse, void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of the library's static device scratch used by flashmask_fwd_noalloc. */
+#define FLASHMASK_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+/*
+ * Forward that allocates nothing: the same computation and outputs as
+ * flashmask_fwd, but its scratch (mask records, block summary, work lists,
+ * scheduler order) lives in one file-scope device array of
+ * FLASHMASK_NOALLOC_SCRATCH_BYTES inside the library instead of a
+ * caller-provided workspace.  (No counterpart in the paper: this is an
+ * interface convenience, not part of the method.)
+ *
+ * For callers that cannot allocate device memory while they run: a serving
+ * process that reserves its whole memory budget at start-up and treats any
+ * later allocation as a fault, or a plugin whose host framework owns the
+ * device allocator and offers its plugins no way to request workspace.
+ * The caller still owns and passes q, k, v, the mask vectors, o and lse.
+ *
+ *  - Every GPU that loads the library holds the 16 MiB array until the
+ *    process exits, whether or not this entry point is used.
+ *  - The first call on a device looks up the array's device address with
+ *    that device current (once per device); make that first call before
+ *    any stream capture.
+ *  - Problems whose forward workspace (flashmask_fwd_workspace_size) exceeds
+ *    the array are rejected with FLASHMASK_ERR_TOO_LARGE before any launch;
+ *    the 16 MiB covers, e.g., one 131072-token sequence with one mask head.
+ *  - All calls share the one array and it keeps the previous call's
+ *    contents; each call writes everything it later reads (and resets its
+ *    work counter) itself.  Calls whose kernels overlap on the GPU -- on
+ *    different streams, or from different host threads -- race on the
+ *    array: serialise them.
+ * No cudaMalloc, cudaFree or other allocating routine is called.
+ */
+int flashmask_fwd_noalloc(const void* q, const void* k, const void* v, const int32_t* lts, const int32_t* lte,
+                          const int32_t* uts, const int32_t* ute, float scale, const flashmask_dims* dims,
+                          void* o, float* lse, void* stream);
 
 /* Bytes of workspace flashmask_bwd needs (forward's plus the backward lists,
  * per-row D = rowsum(dO*O), and an fp32 dQ accumulator [B, Nq, Hq, d]). */
