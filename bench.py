@@ -293,23 +293,29 @@ def run_ours(args, rank, world, local_rank):
     d2h = sum(t.numel() * t.element_size() for t in h_out.values())
 
     # ---- roofline of the dominant kernel ----
+    # Per-kernel work = the matmuls that kernel executes over unmasked pairs:
+    # forward 2 (QK^T, PV) = 4*d*pairs; backward key side 4 (S, dP, dV, dK) =
+    # 8*d*pairs; backward query side 3 (S and dP recomputed, dQ) = 6*d*pairs.
     peaks, peak_src = load_peaks()
-    kinds = {"fwd": (prof["fwd_ms"], prof["fwd_launches"], f_fwd, "fwd_sm100.cu", f"fm_fwd_kernel<{w.d}>"),
-             "bwd": (prof["bwd_ms"], prof["bwd_launches"], f_bwd, "bwd_sm100.cu", f"fm_bwd_kernel<{w.d}>")}
-    dom = max(kinds, key=lambda k: kinds[k][0])
-    ms, nl, fl, src, kname = kinds[dom]
-    achieved = fl / (ms / nl / 1e3) / 1e12 if nl else None
+    d = w.d
+    kinds = {"fwd": ("fwd_sm100.cu", f"fm_fwd_kernel<{d}>", 4.0 * d * pairs),
+             "bwd_kv": ("bwd_dkdv_sm100.cu", f"fm_bwd_dkdv_kernel<{d}>", 8.0 * d * pairs),
+             "bwd_q": ("bwd_dq_sm100.cu", f"fm_bwd_dq_kernel<{d}>", 6.0 * d * pairs)}
+    per_kernel = {}
+    for k, (src, kname, fl) in kinds.items():
+        ms, nl = prof[f"{k}_ms"], prof[f"{k}_launches"]
+        per_kernel[k] = {"kernel": kname, "ms_per_launch": ms / nl if nl else None, "launches": nl,
+                         "tflops": fl / (ms / nl / 1e3) / 1e12 if nl else None, "src": src, "flops": fl}
+    dom = max(per_kernel, key=lambda k: prof[f"{k}_ms"])
+    pk = per_kernel[dom]
     peak = float(peaks["bf16_tflops"])
-    roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-            "frac": (achieved / peak) if achieved else None,
-            "traffic": recorded_traffic(src, w.name), "kernel": kname,
-            "kernel_ms_per_launch": ms / nl if nl else None,
+    roof = {"bound": "tensor", "achieved": pk["tflops"], "peak": peak, "unit": "TFLOP/s",
+            "frac": (pk["tflops"] / peak) if pk["tflops"] else None,
+            "traffic": recorded_traffic(pk["src"], w.name), "kernel": pk["kernel"],
+            "kernel_ms_per_launch": pk["ms_per_launch"], "algorithmic_flops_per_launch": pk["flops"],
             "peak_source": f"{peak_src} bf16_tflops (burst, cuBLAS bf16)",
-            "fwd_kernel_tflops": (f_fwd / (prof["fwd_ms"] / prof["fwd_launches"] / 1e3) / 1e12)
-            if prof["fwd_launches"] else None,
-            "bwd_kernel_tflops": (f_bwd / (prof["bwd_ms"] / prof["bwd_launches"] / 1e3) / 1e12)
-            if prof["bwd_launches"] else None,
-            "kernel_share_of_step": (prof["fwd_ms"] + prof["bwd_ms"]) / local_ms if local_ms else None}
+            "kernels": {k: {kk: v for kk, v in pkk.items() if kk not in ("src",)} for k, pkk in per_kernel.items()},
+            "kernel_share_of_step": sum(prof[f"{k}_ms"] for k in kinds) / local_ms if local_ms else None}
 
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,

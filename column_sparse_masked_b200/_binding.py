@@ -29,7 +29,7 @@ _SIGS = {
     "flashmask_set_wait_limit_ns": (None, [ctypes.c_int64]),
     "flashmask_test_wait_timeout": (ctypes.c_int, [ctypes.c_int64, _P]),
     "flashmask_profiler_enable": (ctypes.c_int, [ctypes.c_int]),
-    "flashmask_profiler_read": (ctypes.c_int, [_P, _P, _P, _P]),
+    "flashmask_profiler_read": (ctypes.c_int, [_P, _P]),
     "flashmask_launch_count": (ctypes.c_int64, []),
     "flashmask_strerror": (ctypes.c_char_p, [ctypes.c_int]),
     "flashmask_version": (ctypes.c_int, []),
@@ -244,12 +244,15 @@ def profiler_enable(on: bool = True) -> None:
 
 
 def profiler_read():
-    """Returns {'fwd_ms', 'fwd_launches', 'bwd_ms', 'bwd_launches'} since the last read."""
-    fm, bm = ctypes.c_double(0), ctypes.c_double(0)
-    fl, bl = ctypes.c_int64(0), ctypes.c_int64(0)
-    _check(load_library().flashmask_profiler_read(ctypes.byref(fm), ctypes.byref(fl), ctypes.byref(bm),
-                                                  ctypes.byref(bl)), "flashmask_profiler_read")
-    return {"fwd_ms": fm.value, "fwd_launches": fl.value, "bwd_ms": bm.value, "bwd_launches": bl.value}
+    """{'fwd_ms', 'fwd_launches', 'bwd_kv_ms', 'bwd_kv_launches', 'bwd_q_ms', 'bwd_q_launches'} since the last read."""
+    ms = (ctypes.c_double * 3)()
+    cnt = (ctypes.c_int64 * 3)()
+    _check(load_library().flashmask_profiler_read(ms, cnt), "flashmask_profiler_read")
+    out = {}
+    for i, k in enumerate(("fwd", "bwd_kv", "bwd_q")):
+        out[f"{k}_ms"] = ms[i]
+        out[f"{k}_launches"] = cnt[i]
+    return out
 
 
 def launch_count() -> int:

@@ -1,0 +1,463 @@
+// Mask-aware attention backward, key side (dK, dV), for sm_100a.
+//
+// "FlashMask-3 targets masked distributed attention on Hopper GPUs", In-depth
+// insight: forward+backward of mask-aware attention.  For the loss sum(O*dO):
+//   dV_j = sum_i P_ij dO_i,   dK_j = scale * sum_i dS_ij q_i,
+//   dS = P o (dP - D),  dP = dO V^T,  D_i = rowsum(dO_i o O_i).
+// dQ is produced by a separate query-stationary kernel (bwd_dq_sm100.cu), so
+// this kernel does no cross-CTA reduction at all.
+//
+// KV-stationary persistent CTAs, one per SM.  A work item is (batch, KV head,
+// 128-key tile): K and V stay in shared memory, dV and dK accumulate in TMEM
+// over every q-head of the GQA group and every non-skipped 128-row q-tile.
+// TMEM (512 columns at d = 128):
+//   S^T [0,128) (P^T bf16 written over it)   dP^T [128,256) (dS^T bf16 over it)
+//   dV [256, 256+d)                          dK [256+d, 256+2d)
+// The MMA warp issues, per q-tile t:
+//   ... dV(t) = P^T(t) dO(t) ; S^T(t+1) = K Q(t+1)^T ; dK(t) = dS^T(t) Q(t) ;
+//   dP^T(t+1) = V dO(t+1)^T ...
+// Tensor-core instructions of one thread execute in issue order, so S^T(t+1)
+// may overwrite the S^T region right after dV(t) (which reads P^T(t) from it)
+// and dP^T(t+1) right after dK(t).  While the tensor core runs dV(t)+S^T(t+1)
+// the compute warps turn dP^T(t) into dS^T(t); while it runs dK(t)+dP^T(t+1)
+// they turn S^T(t+1) into P^T(t+1).
+//
+// Roles (320 threads): warps 0-7 compute (two warpgroups; thread = key lane,
+// warpgroup 0 takes query columns 0-63 of the tile, warpgroup 1 columns
+// 64-127), warp 8 TMA producer, warp 9 MMA issuer.  Work items reach every
+// role through a ring of mbarriers (no CTA-wide barrier between items).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <climits>
+#include <cmath>
+
+#include "common.cuh"
+#include "launchers.h"
+#include "sm100_primitives.cuh"
+
+namespace fm {
+
+namespace kvb {
+constexpr int kThreads = 320;
+constexpr int kProducerWarp = 8, kMmaWarp = 9;
+constexpr int kRing = 4;
+constexpr int kStages = 2;
+constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256;
+}  // namespace kvb
+
+template <int D>
+struct __align__(1024) DkdvSmem {
+  uint8_t k[kTile * D * 2];
+  uint8_t v[kTile * D * 2];
+  uint8_t q[kvb::kStages][kTile * D * 2];
+  uint8_t dout[kvb::kStages][kTile * D * 2];
+  float lse2[kvb::kStages][kTile];
+  float dsum[kvb::kStages][kTile];
+  int ring_item[kvb::kRing];
+  uint64_t ring_full[kvb::kRing], ring_empty[kvb::kRing];
+  uint64_t kv_full, kv_empty;
+  uint64_t qd_full[kvb::kStages], qd_empty[kvb::kStages];
+  uint64_t s_full, dp_full, p_full, ds_full;
+  uint64_t s_read, dp_read;  // both compute warpgroups have loaded S^T / dP^T (bf16 results overlap them)
+  uint64_t dkdv_full, dkdv_free;
+  uint64_t teardown;
+  uint32_t tmem_base;
+  int abort_flag;
+  int no_abort;
+};
+
+struct KvItem {
+  int b, hkv, kt, total;  // total = q-tiles over all q-heads of the group
+};
+
+__device__ __forceinline__ KvItem decode_kv_item(const BwdParams& p, int item) {
+  const Shape& sh = p.s;
+  KvItem it;
+  const ItemCoord c = decode_kv_item_coord(sh, p.order[item]);
+  it.b = c.b;
+  it.hkv = c.hkv;
+  it.kt = c.t;
+  it.total = 0;
+  for (int gi = 0; gi < sh.G; ++gi) {
+    const int h = it.hkv * sh.G + gi;
+    const int hm = (sh.Hm == 1) ? 0 : h;
+    it.total += p.bcount[((size_t)it.b * sh.Hm + hm) * sh.nKt + it.kt];
+  }
+  return it;
+}
+
+// Calls f(j, h, hm, qt, cls) for the item's q-tiles in the order every role walks them.
+template <typename F>
+__device__ __forceinline__ bool for_each_qtile(const BwdParams& p, const KvItem& it, F&& f) {
+  const Shape& sh = p.s;
+  int j = 0;
+  for (int gi = 0; gi < sh.G; ++gi) {
+    const int h = it.hkv * sh.G + gi;
+    const int hm = (sh.Hm == 1) ? 0 : h;
+    const size_t lrow = ((size_t)it.b * sh.Hm + hm) * sh.nKt + it.kt;
+    const int* list = p.blist + lrow * sh.nQt;
+    const int cnt = p.bcount[lrow];
+    for (int t = 0; t < cnt; ++t, ++j) {
+      const int e = list[t];
+      if (!f(j, h, hm, e >> 2, e & 3)) return false;
+    }
+  }
+  return true;
+}
+
+// D[tmem] = A B^T, both K-major SW128 over the head dimension (128 x 128 tile).
+template <int D>
+__device__ __forceinline__ void kv_issue_ss(uint32_t d_tmem, const uint8_t* as, const uint8_t* bs) {
+  constexpr uint32_t idesc = idesc_bf16(128, 128, false, false);
+  const uint32_t aa = smem_addr(as), ba = smem_addr(bs);
+#pragma unroll
+  for (int kk = 0; kk < D / 16; ++kk) {
+    const uint32_t off = (kk / 4) * 16384 + (kk % 4) * 32;
+    mma_ss(d_tmem, sdesc_sw128(aa + off, 16, 1024), sdesc_sw128(ba + off, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+  }
+}
+
+// D[tmem] (+)= A[tmem] B, B = [128 rows (K) x D] tile read MN-major.
+template <int D>
+__device__ __forceinline__ void kv_issue_ts(uint32_t d_tmem, uint32_t a_tmem, const uint8_t* bs, bool accumulate) {
+  constexpr uint32_t idesc = idesc_bf16(128, D, false, true);
+  const uint32_t ba = smem_addr(bs);
+#pragma unroll
+  for (int kk = 0; kk < kTile / 16; ++kk)
+    mma_ts(d_tmem, a_tmem + kk * 8, sdesc_sw128(ba + kk * 2048, 16384, 1024), idesc,
+           (accumulate || kk > 0) ? 1u : 0u);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kvb::kThreads, 1)
+    fm_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                       const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tdo,
+                       const BwdParams p) {
+  using namespace kvb;
+  constexpr int kTileBytes = kTile * D * 2;
+  constexpr int kBoxes = D / 64;
+  constexpr uint32_t kColDK = kColDV + D;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  DkdvSmem<D>& s = *reinterpret_cast<DkdvSmem<D>*>(smem_raw);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const Shape& sh = p.s;
+
+  if (smem_addr(smem_raw) & 1023u) {
+    if (tid == 0) atomicCAS(p.status, 0, -5);
+    return;
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(&s.tmem_base, 512);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    for (int i = 0; i < kRing; ++i) {
+      mbar_init(&s.ring_full[i], 1);
+      mbar_init(&s.ring_empty[i], 9);  // MMA lane 0 + lane 0 of the 8 compute warps
+    }
+    mbar_init(&s.kv_full, 1);
+    mbar_init(&s.kv_empty, 1);
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&s.qd_full[i], 1);
+      mbar_init(&s.qd_empty[i], 1);
+    }
+    mbar_init(&s.s_full, 1);
+    mbar_init(&s.dp_full, 1);
+    mbar_init(&s.p_full, 256);
+    mbar_init(&s.ds_full, 256);
+    mbar_init(&s.s_read, 256);
+    mbar_init(&s.dp_read, 256);
+    mbar_init(&s.dkdv_full, 1);
+    mbar_init(&s.dkdv_free, 256);
+    mbar_init(&s.teardown, 1);
+    s.abort_flag = 0;
+    s.no_abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == kProducerWarp && lane == 0) {
+    tma_prefetch_map(&tq);
+    tma_prefetch_map(&tk);
+    tma_prefetch_map(&tv);
+    tma_prefetch_map(&tdo);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s.tmem_base;
+  const WaitCtx w{&s.abort_flag, p.status, p.wait_limit_ns};
+  uint32_t kv_par = 0, kv_armed = 0, qd_par[kStages] = {}, qd_armed = 0;
+
+  if (warp == kProducerWarp) {
+    if (lane == 0) {
+      uint32_t sq = 0, act = 0;
+      bool ok = true;
+      for (uint32_t k = 0; ok; ++k) {
+        const int slot = k % kRing;
+        if (!(ok = mbar_wait(&s.ring_empty[slot], ((k / kRing) & 1) ^ 1, w))) break;
+        const int item = s.abort_flag ? INT_MAX : atomicAdd(p.counter, 1);
+        s.ring_item[slot] = item;
+        mbar_arrive(&s.ring_full[slot]);
+        if (item >= p.n_items) break;
+        const KvItem it = decode_kv_item(p, item);
+        if (it.total == 0) continue;
+        if (!(ok = mbar_wait(&s.kv_empty, (act & 1) ^ 1, w))) break;
+        mbar_arrive_expect_tx(&s.kv_full, 2 * kTileBytes);
+        kv_par = act & 1;
+        kv_armed = 1;
+#pragma unroll
+        for (int bx = 0; bx < kBoxes; ++bx) {
+          tma_load_4d(s.k + bx * 16384, &tk, &s.kv_full, bx * 64, it.hkv, it.kt * kTile, it.b);
+          tma_load_4d(s.v + bx * 16384, &tv, &s.kv_full, bx * 64, it.hkv, it.kt * kTile, it.b);
+        }
+        ++act;
+        ok = for_each_qtile(p, it, [&](int, int h, int, int qt, int) {
+          const int st = sq % kStages;
+          const uint32_t ph = (sq / kStages) & 1;
+          if (!mbar_wait(&s.qd_empty[st], ph ^ 1, w)) return false;
+          mbar_arrive_expect_tx(&s.qd_full[st], 2 * kTileBytes + 2 * kTile * 4);
+#pragma unroll
+          for (int bx = 0; bx < kBoxes; ++bx) {
+            tma_load_4d(s.q[st] + bx * 16384, &tq, &s.qd_full[st], bx * 64, h, qt * kTile, it.b);
+            tma_load_4d(s.dout[st] + bx * 16384, &tdo, &s.qd_full[st], bx * 64, h, qt * kTile, it.b);
+          }
+          const size_t roff = ((size_t)it.b * sh.Hq + h) * sh.nQt * kTile + (size_t)qt * kTile;
+          bulk_load(s.lse2[st], p.lse2 + roff, kTile * 4, &s.qd_full[st]);
+          bulk_load(s.dsum[st], p.dsum + roff, kTile * 4, &s.qd_full[st]);
+          qd_par[st] = ph;
+          qd_armed |= 1u << st;
+          ++sq;
+          return true;
+        });
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    if (lane == 0) {
+      uint32_t sq = 0, tc = 0, act = 0;
+      bool ok = true;
+      for (uint32_t k = 0; ok; ++k) {
+        const int slot = k % kRing;
+        if (!(ok = mbar_wait(&s.ring_full[slot], (k / kRing) & 1, w))) break;
+        const int item = s.ring_item[slot];
+        mbar_arrive(&s.ring_empty[slot]);
+        if (item >= p.n_items) break;
+        const KvItem it = decode_kv_item(p, item);
+        const int n = it.total;
+        if (n == 0) continue;
+        if (!(ok = mbar_wait(&s.kv_full, act & 1, w))) break;
+        // first q-tile: S^T and dP^T
+        {
+          const int st = sq % kStages;
+          if (!(ok = mbar_wait(&s.qd_full[st], (sq / kStages) & 1, w))) break;
+          tc_fence_after();
+          kv_issue_ss<D>(tmem + kColS, s.k, s.q[st]);
+          mma_commit(&s.s_full);
+          kv_issue_ss<D>(tmem + kColDP, s.v, s.dout[st]);
+          mma_commit(&s.dp_full);
+        }
+        for (int j = 0; j < n; ++j) {
+          const uint32_t sj = sq + j, tj = tc + j;
+          const int st = sj % kStages, st2 = (sj + 1) % kStages;
+          const uint32_t par = tj & 1;
+          if (j == 0 && !(ok = mbar_wait(&s.dkdv_free, (act & 1) ^ 1, w))) break;  // previous item read out
+          if (!(ok = mbar_wait(&s.p_full, par, w))) break;
+          tc_fence_after();
+          kv_issue_ts<D>(tmem + kColDV, tmem + kColS, s.dout[st], j > 0);  // dV += P^T dO
+          if (j + 1 < n) {
+            if (!(ok = mbar_wait(&s.qd_full[st2], ((sj + 1) / kStages) & 1, w))) break;
+            tc_fence_after();
+            kv_issue_ss<D>(tmem + kColS, s.k, s.q[st2]);  // S^T(j+1), after dV(j) read P^T(j)
+            mma_commit(&s.s_full);
+          }
+          if (!(ok = mbar_wait(&s.ds_full, par, w))) break;
+          tc_fence_after();
+          kv_issue_ts<D>(tmem + kColDK, tmem + kColDP, s.q[st], j > 0);  // dK += dS^T Q
+          mma_commit(&s.qd_empty[st]);
+          if (j + 1 < n) {
+            kv_issue_ss<D>(tmem + kColDP, s.v, s.dout[st2]);  // dP^T(j+1), after dK(j) read dS^T(j)
+            mma_commit(&s.dp_full);
+          }
+        }
+        if (!ok) break;
+        sq += n;
+        tc += n;
+        ++act;
+        mma_commit(&s.dkdv_full);
+        mma_commit(&s.kv_empty);
+      }
+    }
+  } else {
+    // ---------------- compute warpgroups: thread = key, 64 query columns each ----------------
+    const int wg = warp >> 2, wq = warp & 3;
+    const int jl = wq * 32 + lane;  // key lane
+    const uint32_t tb = tmem + ((uint32_t)(wq * 32) << 16);
+    const uint32_t c0 = wg * 64;  // first query column of this warpgroup
+    uint32_t sq = 0, tc = 0, act = 0;
+    bool ok = true;
+    for (uint32_t k = 0; ok; ++k) {
+      const int slot = k % kRing;
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(&s.ring_full[slot], (k / kRing) & 1, w)))) break;
+      const int item = s.ring_item[slot];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.ring_empty[slot]);
+      if (item >= p.n_items) break;
+      const KvItem it = decode_kv_item(p, item);
+      const int key = it.kt * kTile + jl;
+      if (it.total > 0) {
+        int cur_hm = -1;
+        int4 rec = make_int4(0, 0, 0, 0);
+        ok = for_each_qtile(p, it, [&](int, int, int hm, int qt, int cls) {
+          if (hm != cur_hm) {
+            rec = p.rec[(((size_t)it.b * sh.Hm + hm) * sh.nKt + it.kt) * kTile + jl];
+            cur_hm = hm;
+          }
+          const int st = sq % kStages;
+          const uint32_t par = tc & 1;
+          if (!__all_sync(0xffffffffu, mbar_wait(&s.s_full, par, w))) return false;
+          if (!__all_sync(0xffffffffu, mbar_wait(&s.qd_full[st], (sq / kStages) & 1, w))) return false;
+          tc_fence_after();
+          const float* l2 = s.lse2[st] + c0;
+          const float* dsm = s.dsum[st] + c0;
+          const bool need = cls == kClsPartial;
+          const int row0 = qt * kTile + c0;
+          // P^T for 64 query columns, in place over the loaded S^T values
+          uint32_t pr[64];
+          tmem_ld32x(tb + kColS + c0, pr);
+          tmem_ld32x(tb + kColS + c0 + 32, pr + 32);
+          tmem_ld_wait();
+          // P^T of query columns 64-127 is written into TMEM columns 32-63, which
+          // hold S^T of columns 32-63: write only after both warpgroups loaded S^T.
+          tc_fence_before();
+          mbar_arrive(&s.s_read);
+#pragma unroll
+          for (int i = 0; i < 64; ++i) {
+            float pv = fast_exp2(__uint_as_float(pr[i]) * p.scale_log2 - l2[i]);
+            if (need) {
+              const int row = row0 + i;
+              const bool masked = (rec.x <= row && row < rec.y) || (rec.z <= row && row < rec.w);
+              pv = masked ? 0.f : pv;
+            }
+            pr[i] = __float_as_uint(pv);
+          }
+          if (!__all_sync(0xffffffffu, mbar_wait(&s.s_read, par, w))) return false;
+          tc_fence_after();
+          {
+            uint32_t pk[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              pk[i] = pack_bf16x2(__uint_as_float(pr[2 * i]), __uint_as_float(pr[2 * i + 1]));
+            tmem_st32x(tb + kColS + c0 / 2, pk);  // bf16 pairs: columns [c0/2, c0/2 + 32)
+          }
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(&s.p_full);
+          // dS^T = P^T o (dP^T - D)
+          if (!__all_sync(0xffffffffu, mbar_wait(&s.dp_full, par, w))) return false;
+          tc_fence_after();
+          {
+            uint32_t r[64];
+            tmem_ld32x(tb + kColDP + c0, r);
+            tmem_ld32x(tb + kColDP + c0 + 32, r + 32);
+            tmem_ld_wait();
+            // dS^T of columns 64-127 lands in TMEM columns 160-191 = dP^T of columns
+            // 32-63: write only after both warpgroups loaded dP^T.
+            tc_fence_before();
+            mbar_arrive(&s.dp_read);
+#pragma unroll
+            for (int i = 0; i < 64; ++i)
+              pr[i] = __float_as_uint(__uint_as_float(pr[i]) * (__uint_as_float(r[i]) - dsm[i]));
+          }
+          if (!__all_sync(0xffffffffu, mbar_wait(&s.dp_read, par, w))) return false;
+          tc_fence_after();
+          {
+            uint32_t pk[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              pk[i] = pack_bf16x2(__uint_as_float(pr[2 * i]), __uint_as_float(pr[2 * i + 1]));
+            tmem_st32x(tb + kColDP + c0 / 2, pk);
+          }
+          tmem_st_wait();
+          tc_fence_before();
+          mbar_arrive(&s.ds_full);
+          ++sq;
+          ++tc;
+          return true;
+        });
+        if (!ok) break;
+        // epilogue: warpgroup 0 writes dV, warpgroup 1 writes dK
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(&s.dkdv_full, act & 1, w)))) break;
+        tc_fence_after();
+        const bool valid = key < sh.Nk;
+        const size_t off = (((size_t)it.b * sh.Nk + (valid ? key : 0)) * sh.Hkv + it.hkv) * D;
+        __nv_bfloat16* dst = (wg == 0 ? p.dv : p.dk) + off;
+        const float mul = (wg == 0) ? 1.f : p.scale;
+        const uint32_t col = (wg == 0) ? kColDV : kColDK;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t rr[32];
+          tmem_ld32x(tb + col + c * 32, rr);
+          tmem_ld_wait();
+          uint32_t pk2[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            pk2[i] = pack_bf16x2(__uint_as_float(rr[2 * i]) * mul, __uint_as_float(rr[2 * i + 1]) * mul);
+          if (valid) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) d4[i] = make_uint4(pk2[4 * i], pk2[4 * i + 1], pk2[4 * i + 2], pk2[4 * i + 3]);
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&s.dkdv_free);
+        ++act;
+      } else if (key < sh.Nk) {
+        // no q-tile reaches this key tile: dK = dV = 0 (each warpgroup one of them)
+        const size_t off = (((size_t)it.b * sh.Nk + key) * sh.Hkv + it.hkv) * D;
+        uint4* d4 = reinterpret_cast<uint4*>((wg == 0 ? p.dv : p.dk) + off);
+#pragma unroll
+        for (int i = 0; i < D / 8; ++i) d4[i] = make_uint4(0, 0, 0, 0);
+      }
+    }
+  }
+
+  // ---------------- teardown ----------------
+  __syncthreads();
+  if (s.abort_flag) {
+    const WaitCtx w2{&s.no_abort, p.status, p.wait_limit_ns};
+    if (warp == kMmaWarp && lane == 0) {
+      mma_commit(&s.teardown);
+      (void)mbar_wait(&s.teardown, 0, w2);
+    }
+    if (warp == kProducerWarp && lane == 0) {
+      if (kv_armed) (void)mbar_wait(&s.kv_full, kv_par, w2);
+      for (int st = 0; st < kStages; ++st)
+        if (qd_armed & (1u << st)) (void)mbar_wait(&s.qd_full[st], qd_par[st], w2);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+template <int D>
+static cudaError_t launch_dkdv_d(const BwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
+                                 const CUtensorMap& tv, const CUtensorMap& tdo, int grid, cudaStream_t st) {
+  const int smem = (int)sizeof(DkdvSmem<D>);
+  cudaError_t e = ensure_smem_limit((const void*)fm_bwd_dkdv_kernel<D>, smem);
+  if (e != cudaSuccess) return e;
+  profile_begin(1, st);
+  note_launch();
+  fm_bwd_dkdv_kernel<D><<<grid, kvb::kThreads, smem, st>>>(tq, tk, tv, tdo, p);
+  profile_end(1, st);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_dkdv(const BwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const CUtensorMap& tdo, int grid, cudaStream_t st) {
+  if (p.s.d == 128) return launch_dkdv_d<128>(p, tq, tk, tv, tdo, grid, st);
+  return launch_dkdv_d<64>(p, tq, tk, tv, tdo, grid, st);
+}
+
+}  // namespace fm

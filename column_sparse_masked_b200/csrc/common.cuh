@@ -41,10 +41,12 @@ struct Shape {
   int nQt;    // q-tiles
   int nKt;    // k-tiles
   int nQB;    // forward blocks of two q-tiles
-  int Ef;     // forward: q-heads per scheduling unit (Hq / Hm)
-  int Mu;     // backward: scheduling units per (batch, k-tile): 1 if Hm == 1 else Hkv
-  int Eb;     // backward: KV heads per unit (Hkv / Mu)
-  int64_t n_units_fwd, n_units_bwd;
+  // Work items of the three attention kernels, indexed group-major: a group
+  // is one (batch, KV head), i.e. the data one L2-resident working set shares.
+  //   forward   (b, hkv, q-block, q-head in group): B*Hq*nQB items
+  //   key side  (b, hkv, k-tile):                   B*Hkv*nKt items
+  //   query side(b, hkv, q-tile, q-head in group):  B*Hq*nQt items
+  int64_t n_fwd_items, n_kv_items, n_q_items;
 };
 
 inline Shape make_shape(int B, int Hq, int Hkv, int Hm, int Nq, int Nk, int d) {
@@ -54,18 +56,16 @@ inline Shape make_shape(int B, int Hq, int Hkv, int Hm, int Nq, int Nk, int d) {
   s.nQt = (Nq + kTile - 1) / kTile;
   s.nKt = (Nk + kTile - 1) / kTile;
   s.nQB = (s.nQt + 1) / 2;
-  s.Ef = Hq / Hm;
-  s.Mu = (Hm == 1) ? 1 : Hkv;
-  s.Eb = Hkv / s.Mu;
-  s.n_units_fwd = (int64_t)B * Hm * s.nQB;
-  s.n_units_bwd = (int64_t)B * s.Mu * s.nKt;
+  s.n_fwd_items = (int64_t)B * Hq * s.nQB;
+  s.n_kv_items = (int64_t)B * Hkv * s.nKt;
+  s.n_q_items = (int64_t)B * Hq * s.nQt;
   return s;
 }
 
 // Workspace layout (byte offsets, each region 256-byte aligned).
 struct WsLayout {
-  size_t rec, ksum, fcount, flist, forder, counters;       // forward part
-  size_t bcount, blist, border, lse2, dsum, dqacc;         // backward part
+  size_t rec, ksum, fcount, flist, qcount, forder, counters;  // forward part
+  size_t bcount, blist, border, qorder, lse2, dsum;        // backward part
   size_t fwd_bytes, bwd_bytes;
 };
 
@@ -80,17 +80,43 @@ inline WsLayout make_layout(const Shape& s) {
   L.ksum = take(bhm * s.nKt * 8 * 4);
   L.fcount = take(bhm * s.nQB * 4);
   L.flist = take(bhm * s.nQB * s.nKt * 4);
-  L.forder = take((size_t)s.n_units_fwd * 4);
+  L.qcount = take(bhm * s.nQB * 2 * 4);
+  L.forder = take((size_t)s.n_fwd_items * 4);
   L.counters = take(64);
   L.fwd_bytes = off;
   L.bcount = take(bhm * s.nKt * 4);
   L.blist = take(bhm * s.nKt * s.nQt * 4);
-  L.border = take((size_t)s.n_units_bwd * 4);
+  L.border = take((size_t)s.n_kv_items * 4);
+  L.qorder = take((size_t)s.n_q_items * 4);
   L.lse2 = take((size_t)s.B * s.Hq * s.nQt * kTile * 4);
   L.dsum = take((size_t)s.B * s.Hq * s.nQt * kTile * 4);
-  L.dqacc = take((size_t)s.B * s.Nq * s.Hq * s.d * 4);
   L.bwd_bytes = off;
   return L;
+}
+
+struct ItemCoord {
+  int b, hkv, t, hg;  // t = q-block, k-tile or q-tile; hg = q-head within the GQA group
+};
+__host__ __device__ __forceinline__ ItemCoord decode_fwd_item(const Shape& s, int i) {
+  ItemCoord c;
+  c.hg = i % s.G; i /= s.G;
+  c.t = i % s.nQB; i /= s.nQB;
+  c.hkv = i % s.Hkv; c.b = i / s.Hkv;
+  return c;
+}
+__host__ __device__ __forceinline__ ItemCoord decode_kv_item_coord(const Shape& s, int i) {
+  ItemCoord c;
+  c.hg = 0;
+  c.t = i % s.nKt; i /= s.nKt;
+  c.hkv = i % s.Hkv; c.b = i / s.Hkv;
+  return c;
+}
+__host__ __device__ __forceinline__ ItemCoord decode_q_item_coord(const Shape& s, int i) {
+  ItemCoord c;
+  c.hg = i % s.G; i /= s.G;
+  c.t = i % s.nQt; i /= s.nQt;
+  c.hkv = i % s.Hkv; c.b = i / s.Hkv;
+  return c;
 }
 
 // ----------------------------------------------------------------------------
@@ -107,17 +133,22 @@ struct PlanParams {
   Shape s;
   const int* ksum;
   int* fcount; int* flist;   // forward lists  [B, Hm, nQB] / [B, Hm, nQB, nKt]
+  int* qcount;               // per q-tile non-skipped k-tiles [B, Hm, nQB*2]
   int* bcount; int* blist;   // backward lists [B, Hm, nKt] / [B, Hm, nKt, nQt]
   uint8_t* cls;              // optional export [B, Hm, nQt, nKt]
 };
 
+// Longest-first order of the work items, in waves of `wave` consecutive
+// (batch, KV head) groups (0 = natural group-major order, no sorting).
 struct SortParams {
   Shape s;
-  int mode;               // 0: forward units, 1: backward units
-  const int* count;       // fcount or bcount
-  int* order;             // out: unit order, descending cost
+  int mode;               // 0: forward items, 1: key-side items, 2: query-side items
+  const int* count;       // fcount, bcount or qcount
+  int* order;             // out: item order
   int* counter;           // zeroed for the persistent kernel that follows
-  int n_units;
+  int n_items;
+  int items_per_group;
+  int wave;
 };
 
 struct FwdParams {
@@ -142,7 +173,6 @@ struct BwdPreParams {
   const float* lse;
   float* lse2;     // [B, Hq, nQt*128]: LSE * log2(e); +inf for empty and padded rows
   float* dsum;     // [B, Hq, nQt*128]: rowsum(dO * O); 0 for padded rows
-  float* dqacc;    // [B, Nq, Hq, d] zeroed
 };
 
 struct BwdParams {
@@ -150,25 +180,25 @@ struct BwdParams {
   float scale;
   float scale_log2;
   const int4* rec;
+  // key side (dK, dV): per (b, hm, k-tile) q-tile lists, units (b, mu, k-tile)
   const int* blist;
   const int* bcount;
   const int* order;
   int* counter;
   int n_items;
+  // query side (dQ): per (b, hm, q-block) k-tile lists, units (b, hm, q-block)
+  const int* flist;
+  const int* fcount;
+  const int* forder;
+  int* counter2;
+  int n_items2;
   const float* lse2;
   const float* dsum;
-  float* dqacc;
+  __nv_bfloat16* dq;
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
   int* status;
   uint64_t wait_limit_ns;
-};
-
-struct DqFinParams {
-  const float* dqacc;
-  __nv_bfloat16* dq;
-  float scale;
-  int64_t n;  // elements
 };
 
 }  // namespace fm

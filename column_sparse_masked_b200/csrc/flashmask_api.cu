@@ -76,13 +76,13 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 4-D map over a [B, N, H, d] bf16 tensor: box = 64 columns x 1 head x 128 rows.
-int make_map(CUtensorMap* m, const void* ptr, int B, int N, int H, int d) {
+// 4-D map over a [B, N, H, d] bf16 tensor: box = 64 columns x 1 head x box_rows rows.
+int make_map(CUtensorMap* m, const void* ptr, int B, int N, int H, int d, int box_rows = kTile) {
   auto enc = encode_fn();
   if (!enc) return FLASHMASK_ERR_CUDA;
   cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)N, (cuuint64_t)B};
   cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2, (cuuint64_t)N * H * d * 2};
-  cuuint32_t box[4] = {64, 1, (cuuint32_t)kTile, 1};
+  cuuint32_t box[4] = {64, 1, (cuuint32_t)box_rows, 1};
   cuuint32_t es[4] = {1, 1, 1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(ptr), dims, strides, box, es,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -103,7 +103,7 @@ int check_dims(const flashmask_dims* dm) {
   if (d.d != 64 && d.d != 128) return FLASHMASK_ERR_UNSUPPORTED;
   if (d.Nq > (1 << 30) || d.Nk > (1 << 30)) return FLASHMASK_ERR_UNSUPPORTED;
   const Shape s = make_shape(d.B, d.Hq, d.Hkv, d.Hm, d.Nq, d.Nk, d.d);
-  if ((int64_t)s.B * s.Hq * s.nQB >= INT_MAX || (int64_t)s.B * s.Hkv * s.nKt >= INT_MAX)
+  if (s.n_q_items >= INT_MAX || s.n_kv_items >= INT_MAX)
     return FLASHMASK_ERR_UNSUPPORTED;
   return FLASHMASK_OK;
 }
@@ -161,6 +161,20 @@ struct ProfRec {
 std::vector<ProfRec> g_prof_pool;  // guarded by g_mu
 size_t g_prof_used = 0;
 constexpr size_t kProfMax = 4096;
+
+// Groups per longest-first wave: as many (batch, KV head) groups as keep the
+// data a group's items share (Q/dO for the key side, K/V otherwise) within
+// about half of the 126 MB L2; 0 (natural, position order) when a single group
+// is larger than that.
+int wave_groups(size_t group_bytes, int n_groups, int64_t n_items, int sm_count) {
+  const size_t budget = (size_t)64 << 20;
+  // With few items per CTA the tail of the longest-first order decides the
+  // makespan: order all groups together.
+  if (group_bytes == 0 || n_items < (int64_t)16 * sm_count) return n_groups;
+  const size_t w = budget / group_bytes;
+  if (w == 0) return 0;
+  return (int)(w < (size_t)n_groups ? w : (size_t)n_groups);
+}
 
 }  // namespace
 
@@ -265,6 +279,7 @@ int flashmask_fwd(const void* q, const void* k, const void* v, const int32_t* lt
   pp.ksum = mp.ksum;
   pp.fcount = reinterpret_cast<int*>(ws + L.fcount);
   pp.flist = reinterpret_cast<int*>(ws + L.flist);
+  pp.qcount = reinterpret_cast<int*>(ws + L.qcount);
   FM_CUDA(launch_plan_fwd(pp, st));
 
   SortParams sp{};
@@ -273,7 +288,9 @@ int flashmask_fwd(const void* q, const void* k, const void* v, const int32_t* lt
   sp.count = pp.fcount;
   sp.order = reinterpret_cast<int*>(ws + L.forder);
   sp.counter = reinterpret_cast<int*>(ws + L.counters);
-  sp.n_units = (int)s.n_units_fwd;
+  sp.n_items = (int)s.n_fwd_items;
+  sp.items_per_group = s.nQB * s.G;
+  sp.wave = wave_groups((size_t)s.Nk * s.d * 2 * 2, s.B * s.Hkv, s.n_fwd_items, di.sm_count);
   FM_CUDA(launch_sort_units(sp, st));
 
   FwdParams fp{};
@@ -284,7 +301,7 @@ int flashmask_fwd(const void* q, const void* k, const void* v, const int32_t* lt
   fp.fcount = pp.fcount;
   fp.order = sp.order;
   fp.counter = sp.counter;
-  fp.n_items = (int)(s.n_units_fwd * s.Ef);
+  fp.n_items = (int)s.n_fwd_items;
   fp.o = static_cast<__nv_bfloat16*>(o);
   fp.lse = lse;
   fp.status = di.status;
@@ -320,7 +337,7 @@ int flashmask_bwd(const void* q, const void* k, const void* v, const void* o, co
   if (has_q) {
     FM_TRY(make_map(&tq, q, s.B, s.Nq, s.Hq, s.d));
     FM_TRY(make_map(&tdo, dout, s.B, s.Nq, s.Hq, s.d));
-  } else {
+  } else {  // never read: every work list is empty
     FM_TRY(make_map(&tq, workspace, 1, 1, 1, s.d));
     tdo = tq;
   }
@@ -334,21 +351,39 @@ int flashmask_bwd(const void* q, const void* k, const void* v, const void* o, co
   const MaskPrepParams mp = prep_params(s, L, ws, lts, lte, uts, ute);
   FM_CUDA(launch_mask_prep(mp, st));
 
+  // key side: per k-tile q-tile lists, longest-first units
   PlanParams pp{};
   pp.s = s;
   pp.ksum = mp.ksum;
   pp.bcount = reinterpret_cast<int*>(ws + L.bcount);
   pp.blist = reinterpret_cast<int*>(ws + L.blist);
+  pp.fcount = reinterpret_cast<int*>(ws + L.fcount);
+  pp.flist = reinterpret_cast<int*>(ws + L.flist);
   FM_CUDA(launch_plan_bwd(pp, st));
-
-  SortParams sp{};
-  sp.s = s;
-  sp.mode = 1;
-  sp.count = pp.bcount;
-  sp.order = reinterpret_cast<int*>(ws + L.border);
-  sp.counter = reinterpret_cast<int*>(ws + L.counters) + 1;
-  sp.n_units = (int)s.n_units_bwd;
-  if (sp.n_units > 0) FM_CUDA(launch_sort_units(sp, st));
+  int* counters = reinterpret_cast<int*>(ws + L.counters);
+  SortParams sb{};
+  sb.s = s;
+  sb.mode = 1;
+  sb.count = pp.bcount;
+  sb.order = reinterpret_cast<int*>(ws + L.border);
+  sb.counter = counters + 1;
+  sb.n_items = (int)s.n_kv_items;
+  sb.items_per_group = s.nKt;
+  sb.wave = wave_groups((size_t)s.G * s.Nq * s.d * 2 * 2, s.B * s.Hkv, s.n_kv_items, di.sm_count);
+  if (sb.n_items > 0) FM_CUDA(launch_sort_units(sb, st));
+  // query side: per q-block k-tile lists (the forward's), per q-tile counts
+  pp.qcount = reinterpret_cast<int*>(ws + L.qcount);
+  FM_CUDA(launch_plan_fwd(pp, st));
+  SortParams sf{};
+  sf.s = s;
+  sf.mode = 2;
+  sf.count = pp.qcount;
+  sf.order = reinterpret_cast<int*>(ws + L.qorder);
+  sf.counter = counters + 2;
+  sf.n_items = (int)s.n_q_items;
+  sf.items_per_group = s.nQt * s.G;
+  sf.wave = wave_groups((size_t)s.Nk * s.d * 2 * 2, s.B * s.Hkv, s.n_q_items, di.sm_count);
+  if (sf.n_items > 0) FM_CUDA(launch_sort_units(sf, st));
 
   BwdPreParams bp{};
   bp.s = s;
@@ -357,7 +392,6 @@ int flashmask_bwd(const void* q, const void* k, const void* v, const void* o, co
   bp.lse = lse;
   bp.lse2 = reinterpret_cast<float*>(ws + L.lse2);
   bp.dsum = reinterpret_cast<float*>(ws + L.dsum);
-  bp.dqacc = reinterpret_cast<float*>(ws + L.dqacc);
   if (has_q) FM_CUDA(launch_bwd_pre(bp, st));
 
   BwdParams kp{};
@@ -367,27 +401,25 @@ int flashmask_bwd(const void* q, const void* k, const void* v, const void* o, co
   kp.rec = mp.rec;
   kp.blist = pp.blist;
   kp.bcount = pp.bcount;
-  kp.order = sp.order;
-  kp.counter = sp.counter;
-  kp.n_items = (int)(s.n_units_bwd * s.Eb);
+  kp.order = sb.order;
+  kp.counter = sb.counter;
+  kp.n_items = (int)s.n_kv_items;
+  kp.flist = pp.flist;
+  kp.fcount = pp.fcount;
+  kp.forder = sf.order;
+  kp.counter2 = sf.counter;
+  kp.n_items2 = (int)s.n_q_items;
   kp.lse2 = bp.lse2;
   kp.dsum = bp.dsum;
-  kp.dqacc = bp.dqacc;
+  kp.dq = static_cast<__nv_bfloat16*>(dq);
   kp.dk = static_cast<__nv_bfloat16*>(dk);
   kp.dv = static_cast<__nv_bfloat16*>(dv);
   kp.status = di.status;
   kp.wait_limit_ns = (uint64_t)g_wait_limit_ns.load();
-  const int grid = kp.n_items < di.sm_count ? kp.n_items : di.sm_count;
-  if (grid > 0) FM_CUDA(launch_bwd(kp, tq, tk, tv, tdo, grid, st));
-
-  if (has_q) {
-    DqFinParams fp{};
-    fp.dqacc = bp.dqacc;
-    fp.dq = static_cast<__nv_bfloat16*>(dq);
-    fp.scale = sc;
-    fp.n = (int64_t)s.B * s.Nq * s.Hq * s.d;
-    FM_CUDA(launch_dq_finalize(fp, st));
-  }
+  const int grid_kv = kp.n_items < di.sm_count ? kp.n_items : di.sm_count;
+  if (grid_kv > 0) FM_CUDA(launch_bwd_dkdv(kp, tq, tk, tv, tdo, grid_kv, st));
+  const int grid_q = kp.n_items2 < di.sm_count ? kp.n_items2 : di.sm_count;
+  if (has_q && grid_q > 0) FM_CUDA(launch_bwd_dq(kp, tq, tk, tv, tdo, grid_q, st));
   return FLASHMASK_OK;
 }
 
@@ -483,10 +515,10 @@ int flashmask_profiler_enable(int on) {
   return FLASHMASK_OK;
 }
 
-int flashmask_profiler_read(double* fwd_ms, int64_t* fwd_launches, double* bwd_ms, int64_t* bwd_launches) {
+int flashmask_profiler_read(double* ms_out, int64_t* launches_out) {
   std::lock_guard<std::mutex> lock(g_mu);
-  double ms[2] = {0.0, 0.0};
-  int64_t cnt[2] = {0, 0};
+  double ms[3] = {0.0, 0.0, 0.0};
+  int64_t cnt[3] = {0, 0, 0};
   int rc = FLASHMASK_OK;
   for (size_t i = 0; i < g_prof_used; ++i) {
     ProfRec& r = g_prof_pool[i];
@@ -495,14 +527,15 @@ int flashmask_profiler_read(double* fwd_ms, int64_t* fwd_launches, double* bwd_m
       rc = FLASHMASK_ERR_CUDA;
       continue;
     }
-    ms[r.kind & 1] += t;
-    cnt[r.kind & 1] += 1;
+    const int kd = (r.kind >= 0 && r.kind < 3) ? r.kind : 0;
+    ms[kd] += t;
+    cnt[kd] += 1;
   }
   g_prof_used = 0;
-  if (fwd_ms) *fwd_ms = ms[0];
-  if (fwd_launches) *fwd_launches = cnt[0];
-  if (bwd_ms) *bwd_ms = ms[1];
-  if (bwd_launches) *bwd_launches = cnt[1];
+  for (int kd = 0; kd < 3; ++kd) {
+    if (ms_out) ms_out[kd] = ms[kd];
+    if (launches_out) launches_out[kd] = cnt[kd];
+  }
   return rc;
 }
 

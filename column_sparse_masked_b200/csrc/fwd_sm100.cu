@@ -168,13 +168,10 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
     __syncthreads();
     const int item = s.item;
     if (item >= p.n_items) break;
-    const int unit = p.order[item / sh.Ef];
-    const int hsub = item % sh.Ef;
-    const int qb = unit % sh.nQB;
-    const int hm = (unit / sh.nQB) % sh.Hm;
-    const int b = unit / (sh.nQB * sh.Hm);
-    const int h = hm * sh.Ef + hsub;
-    const int hkv = h / sh.G;
+    const ItemCoord c = decode_fwd_item(sh, p.order[item]);
+    const int b = c.b, qb = c.t, hkv = c.hkv;
+    const int h = hkv * sh.G + c.hg;
+    const int hm = (sh.Hm == 1) ? 0 : h;
     const size_t lrow = ((size_t)b * sh.Hm + hm) * sh.nQB + qb;
     const int* list = p.flist + lrow * sh.nKt;
     const int n = p.fcount[lrow];

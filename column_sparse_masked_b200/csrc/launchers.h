@@ -22,12 +22,15 @@ cudaError_t launch_wait_timeout(int* status, uint64_t limit_ns, cudaStream_t st)
 cudaError_t launch_fwd(const FwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        int grid, cudaStream_t st);
 cudaError_t launch_bwd_pre(const BwdPreParams& p, cudaStream_t st);
-cudaError_t launch_bwd(const BwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                       const CUtensorMap& tdo, int grid, cudaStream_t st);
-cudaError_t launch_dq_finalize(const DqFinParams& p, cudaStream_t st);
+// Backward, key side (dK, dV) and query side (dQ); both persistent, grid CTAs.
+cudaError_t launch_bwd_dkdv(const BwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const CUtensorMap& tdo, int grid, cudaStream_t st);
+cudaError_t launch_bwd_dq(const BwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                          const CUtensorMap& tdo, int grid, cudaStream_t st);
 
 // Launch bookkeeping: counts every launch; brackets the attention kernels
-// with profiler events when profiling is enabled (kind 0 forward, 1 backward).
+// with profiler events when profiling is enabled (kind 0 forward, 1 backward
+// dK/dV, 2 backward dQ).
 void note_launch();
 void profile_begin(int kind, cudaStream_t st);
 void profile_end(int kind, cudaStream_t st);

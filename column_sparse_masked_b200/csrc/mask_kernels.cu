@@ -91,6 +91,8 @@ __global__ void __launch_bounds__(128) plan_fwd_kernel(PlanParams p) {
   int* list = p.flist + (row * s.nQB + qb) * s.nKt;
   __shared__ int warp_tot[4];
   __shared__ int total;
+  __shared__ int qc[2];
+  if (threadIdx.x < 2) qc[threadIdx.x] = 0;
   int count = 0;
   for (int base = 0; base < s.nKt; base += kTile) {
     const int kt = base + threadIdx.x;
@@ -104,12 +106,19 @@ __global__ void __launch_bounds__(128) plan_fwd_kernel(PlanParams p) {
       if (qt1 < s.nQt) c1 = classify_tile(sm, r10, r11);
     }
     const bool keep = (c0 != kClsSkip) || (c1 != kClsSkip);
+    const unsigned b0 = __ballot_sync(0xffffffffu, c0 != kClsSkip);
+    const unsigned b1 = __ballot_sync(0xffffffffu, c1 != kClsSkip);
+    if ((threadIdx.x & 31) == 0) {
+      atomicAdd(&qc[0], __popc(b0));
+      atomicAdd(&qc[1], __popc(b1));
+    }
     const int pos = block_compact128(keep, warp_tot, &total);
     if (keep) list[count + pos] = fwd_entry(kt, c0, c1, (ragged_k && kt == s.nKt - 1) ? 1 : 0);
     count += total;
     __syncthreads();
   }
   if (threadIdx.x == 0) p.fcount[row * s.nQB + qb] = count;
+  if (threadIdx.x < 2) p.qcount[(row * s.nQB + qb) * 2 + threadIdx.x] = qc[threadIdx.x];
 }
 
 // ----------------------------------------------------------------------------
@@ -158,19 +167,42 @@ __global__ void __launch_bounds__(128) classify_export_kernel(PlanParams p) {
 }
 
 // ----------------------------------------------------------------------------
-// 3. longest-first order of scheduling units (one CTA, bitonic sort in smem).
-//    Key = (~cost << 32) | unit: descending cost, ascending unit id on ties.
+// 3. work order of the persistent kernels (one CTA, bitonic sort in smem).
+//    Items are indexed group-major ((batch, KV head) groups), so the natural
+//    order keeps one group's data together in L2.  With wave > 0 the items of
+//    `wave` consecutive groups are taken longest-first:
+//      key = wave index << 48 | (0xFFFF - cost) << 32 | item.
 //    Also zeroes the work counter of the persistent kernel that follows.
 // ----------------------------------------------------------------------------
-constexpr int kSortMax = 8192;
+constexpr int kSortMax = 16384;
+
+__device__ __forceinline__ unsigned item_cost(const SortParams& p, int i) {
+  const Shape& s = p.s;
+  if (p.mode == 0) {
+    const ItemCoord c = decode_fwd_item(s, i);
+    const int h = c.hkv * s.G + c.hg, hm = (s.Hm == 1) ? 0 : h;
+    return (unsigned)p.count[((size_t)c.b * s.Hm + hm) * s.nQB + c.t];
+  }
+  if (p.mode == 1) {
+    const ItemCoord c = decode_kv_item_coord(s, i);
+    unsigned cost = 0;
+    for (int g = 0; g < s.G; ++g) {
+      const int h = c.hkv * s.G + g, hm = (s.Hm == 1) ? 0 : h;
+      cost += (unsigned)p.count[((size_t)c.b * s.Hm + hm) * s.nKt + c.t];
+    }
+    return cost;
+  }
+  const ItemCoord c = decode_q_item_coord(s, i);
+  const int h = c.hkv * s.G + c.hg, hm = (s.Hm == 1) ? 0 : h;
+  return (unsigned)p.count[((size_t)c.b * s.Hm + hm) * (s.nQB * 2) + c.t];
+}
 
 __global__ void __launch_bounds__(1024) sort_units_kernel(SortParams p) {
   extern __shared__ unsigned long long keys[];
-  const Shape& s = p.s;
-  const int n = p.n_units;
+  const int n = p.n_items;
   const int t = threadIdx.x;
   if (t == 0) p.counter[0] = 0;
-  if (n > kSortMax) {  // too many units for the in-smem sort: identity order
+  if (p.wave <= 0 || n > kSortMax) {  // natural group-major order
     for (int u = t; u < n; u += blockDim.x) p.order[u] = u;
     return;
   }
@@ -179,21 +211,9 @@ __global__ void __launch_bounds__(1024) sort_units_kernel(SortParams p) {
   for (int u = t; u < np2; u += blockDim.x) {
     unsigned long long key = ~0ull;
     if (u < n) {
-      unsigned cost;
-      if (p.mode == 0) {
-        cost = (unsigned)p.count[u];
-      } else {
-        // unit u = (b, mu, kt); its q-heads' lists live at mask heads
-        // [mu*Gm, mu*Gm + Gm) with Gm = 1 for a shared mask.
-        const int kt = u % s.nKt, mu = (u / s.nKt) % s.Mu, b = u / (s.nKt * s.Mu);
-        if (s.Hm == 1) {
-          cost = (unsigned)p.count[(size_t)b * s.nKt + kt] * (unsigned)s.G;
-        } else {
-          cost = 0;
-          for (int g = 0; g < s.G; ++g) cost += (unsigned)p.count[((size_t)b * s.Hm + mu * s.G + g) * s.nKt + kt];
-        }
-      }
-      key = ((unsigned long long)(~cost) << 32) | (unsigned)u;
+      const unsigned cost = min(item_cost(p, u), 0xFFFFu);
+      const unsigned long long wv = (unsigned long long)((u / p.items_per_group) / p.wave);
+      key = (wv << 48) | ((unsigned long long)(0xFFFFu - cost) << 32) | (unsigned)u;
     }
     keys[u] = key;
   }
@@ -324,10 +344,10 @@ cudaError_t launch_classify_export(const PlanParams& p, cudaStream_t st) {
 }
 
 cudaError_t launch_sort_units(const SortParams& p, cudaStream_t st) {
-  const int n = p.n_units;
+  const int n = p.n_items;
   int np2 = 1;
   while (np2 < n) np2 <<= 1;
-  const size_t smem = (n <= kSortMax) ? (size_t)np2 * sizeof(unsigned long long) : 0;
+  const size_t smem = (p.wave > 0 && n <= kSortMax) ? (size_t)np2 * sizeof(unsigned long long) : 0;
   cudaError_t e = ensure_smem_limit((const void*)sort_units_kernel, (int)(kSortMax * sizeof(unsigned long long)));
   if (e != cudaSuccess) return e;
   { note_launch(); sort_units_kernel<<<1, 1024, smem, st>>>(p);

@@ -117,7 +117,8 @@ int flashmask_fwd_noalloc(const void* q, const void* k, const void* v, const int
                           void* o, float* lse, void* stream);
 
 /* Bytes of workspace flashmask_bwd needs (forward's plus the backward lists,
- * per-row D = rowsum(dO*O), and an fp32 dQ accumulator [B, Nq, Hq, d]). */
+ * and per-row D = rowsum(dO*O) and LSE in log2 units over whole 128-row
+ * tiles). */
 size_t flashmask_bwd_workspace_size(const flashmask_dims* dims);
 
 /*
@@ -125,7 +126,8 @@ size_t flashmask_bwd_workspace_size(const flashmask_dims* dims);
  * "forward+backward"): dQ, dK, dV.  dK and dV sum the contributions of the
  * Hq/Hkv q-heads that share a KV head.  `o` and `lse` must be the forward's
  * outputs for the same inputs.  Key columns that no row sees get dK = dV = 0;
- * fully masked rows get dQ = 0.  Outputs are written in full.
+ * fully masked rows get dQ = 0.  Outputs are written in full, each element by
+ * exactly one CTA (no atomics): results are deterministic.
  */
 int flashmask_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
                   const int32_t* lts, const int32_t* lte, const int32_t* uts, const int32_t* ute, float scale,
@@ -190,15 +192,16 @@ void flashmask_set_wait_limit_ns(int64_t ns);
 int flashmask_test_wait_timeout(int64_t limit_ns, void* stream);
 
 /*
- * Kernel timing for benchmarks.  While enabled (on != 0), every launch of the
- * forward or backward attention kernel is bracketed by a CUDA event pair
- * recorded on the call's stream.  flashmask_profiler_read() waits for the
- * recorded events, returns the summed kernel milliseconds and launch counts
- * of each kind (either output pointer may be NULL) and clears them.  Event
- * pairs are pooled (at most 4096 outstanding).  Host-side, process-wide.
+ * Kernel timing for benchmarks.  While enabled (on != 0), every launch of an
+ * attention kernel is bracketed by a CUDA event pair recorded on the call's
+ * stream.  flashmask_profiler_read() waits for the recorded events and fills
+ * ms[3] / launches[3] (either may be NULL) with the summed milliseconds and
+ * launch counts of kind 0 = forward, 1 = backward key side (dK, dV),
+ * 2 = backward query side (dQ), then clears them.  Event pairs are pooled (at
+ * most 4096 outstanding).  Host-side, process-wide.
  */
 int flashmask_profiler_enable(int on);
-int flashmask_profiler_read(double* fwd_ms, int64_t* fwd_launches, double* bwd_ms, int64_t* bwd_launches);
+int flashmask_profiler_read(double* ms, int64_t* launches);
 
 /* Number of kernels this library has launched since the process started
  * (every kind: summary, lists, ordering, attention, preprocess, finalise). */
