@@ -7,16 +7,24 @@
 // (TMA/WGMMA with three warp roles); this one is written for Blackwell:
 //
 //   * persistent CTAs (one per SM) take work items -- (batch, q-head, block of
-//     two 128-row q-tiles) -- from a longest-first list through an atomic
-//     counter;
+//     two 128-row q-tiles) -- from a locality-aware longest-first order through
+//     an atomic counter; the producer warp hands each item to the other roles
+//     through a ring of mbarriers, so consecutive items overlap (the next
+//     item's Q load and first QK^T run while the softmax warps write O);
 //   * warp 8 issues TMA loads (Q once per item; K, V and, for tiles that need
 //     it, the 2 KiB boundary records through a multi-stage ring);
 //   * warp 9 issues tcgen05 MMAs: S_g = Q_g K^T into TMEM, O_g += P_g V with
-//     P_g read from TMEM (bf16, written over S_g);
+//     P_g read from TMEM (bf16, written over S_g), ping-pong between the two
+//     q-tiles: S0 S1 | PV0 S0' PV1 S1' | ...;
 //   * warps 0-3 and 4-7 are the softmax groups of q-tiles 0 and 1: one thread
-//     per query row, S read with tcgen05.ld, online softmax in the exp2
-//     domain, O rescaled in TMEM only when a row maximum grows by more than
-//     2^8 (otherwise the stale maximum is kept, exact after the final 1/l).
+//     per query row; online softmax in the exp2 domain with the scale folded
+//     into one FMA per element, O rescaled in TMEM
+//     only when a row maximum grows by more than 2^8.
+//
+// The element mask of a partial tile is built per key column: each lane turns
+// the boundaries of 4 columns into 32-bit words over its warp's 32 rows
+// (interval arithmetic), and a 5-step shuffle transpose of each 32x32 bit
+// block hands every row its mask bits.
 //
 // TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+d), O1 after O0.
 #include <cuda.h>
@@ -38,6 +46,7 @@ struct FwdCfg {
   static constexpr int kThreads = 320;
   static constexpr int kProducerWarp = 8;
   static constexpr int kMmaWarp = 9;
+  static constexpr int kRing = 4;
 };
 
 template <int D>
@@ -46,19 +55,42 @@ struct __align__(1024) FwdSmem {
   uint8_t k[FwdCfg<D>::kStages][FwdCfg<D>::kTileBytes];
   uint8_t v[FwdCfg<D>::kStages][FwdCfg<D>::kTileBytes];
   int4 mask[FwdCfg<D>::kStages][kTile];
-  uint64_t q_full;
+  int ring_item[FwdCfg<D>::kRing];
+  uint64_t ring_full[FwdCfg<D>::kRing], ring_empty[FwdCfg<D>::kRing];
+  uint64_t q_full, q_empty;
   uint64_t k_full[FwdCfg<D>::kStages];
   uint64_t v_full[FwdCfg<D>::kStages];
   uint64_t kv_empty[FwdCfg<D>::kStages];
   uint64_t s_full[2];
   uint64_t p_full[2];
   uint64_t o_full[2];
+  uint64_t o_free[2];
   uint64_t teardown;
   uint32_t tmem_base;
   int abort_flag;
   int no_abort;
-  int item;
 };
+
+struct FwdItem {
+  int b, h, hm, hkv, qb;
+  const int* list;
+  int n;
+};
+
+__device__ __forceinline__ FwdItem decode_fwd(const FwdParams& p, int item) {
+  const Shape& sh = p.s;
+  const ItemCoord c = decode_fwd_item(sh, p.order[item]);
+  FwdItem it;
+  it.b = c.b;
+  it.qb = c.t;
+  it.hkv = c.hkv;
+  it.h = c.hkv * sh.G + c.hg;
+  it.hm = (sh.Hm == 1) ? 0 : it.h;
+  const size_t lrow = ((size_t)it.b * sh.Hm + it.hm) * sh.nQB + it.qb;
+  it.list = p.flist + lrow * sh.nKt;
+  it.n = p.fcount[lrow];
+  return it;
+}
 
 // S = Q K^T: M = 128 rows, N = 128 keys, K = D; both operands K-major SW128.
 template <int D>
@@ -84,29 +116,39 @@ __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, const
            (accumulate || kk > 0) ? 1u : 0u);
 }
 
-__device__ __forceinline__ void tmem_ld32p(uint32_t taddr, uint32_t* r) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
-      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
-        "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
-        "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
-        "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
+// Bits [lo, hi) of a 32-bit word (0 <= lo, hi <= 32).
+__device__ __forceinline__ uint32_t bit_range(int lo, int hi) {
+  const uint32_t up = hi >= 32 ? 0xffffffffu : ((1u << hi) - 1u);
+  const uint32_t dn = lo >= 32 ? 0xffffffffu : ((1u << lo) - 1u);
+  return hi > lo ? (up & ~dn) : 0u;
 }
 
-__device__ __forceinline__ void tmem_st32p(uint32_t taddr, const uint32_t* r) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
-      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
-      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
-      "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
-      "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
-      : "memory");
+// Rows [r0, r0+32) hidden by one key column's intervals, as a 32-bit word.
+__device__ __forceinline__ uint32_t column_row_bits(const int4 r, int r0) {
+  const int a0 = min(max(r.x - r0, 0), 32), a1 = min(max(r.y - r0, 0), 32);
+  const int b0 = min(max(r.z - r0, 0), 32), b1 = min(max(r.w - r0, 0), 32);
+  return bit_range(a0, a1) | bit_range(b0, b1);
+}
+
+// 32x32 bit-matrix transpose across a warp: lane l holds word l on entry
+// (bit r = element (l, r)); on exit lane r holds bit l = element (l, r).
+template <int J, uint32_t M>
+__device__ __forceinline__ uint32_t transpose_step(uint32_t a, int lane) {
+  const uint32_t b = __shfl_xor_sync(0xffffffffu, a, J);
+  return (lane & J) ? ((a & ~M) | ((b & ~M) >> J)) : ((a & M) | ((b & M) << J));
+}
+__device__ __forceinline__ uint32_t warp_transpose32(uint32_t a, int lane) {
+  a = transpose_step<16, 0x0000FFFFu>(a, lane);
+  a = transpose_step<8, 0x00FF00FFu>(a, lane);
+  a = transpose_step<4, 0x0F0F0F0Fu>(a, lane);
+  a = transpose_step<2, 0x33333333u>(a, lane);
+  return transpose_step<1, 0x55555555u>(a, lane);
+}
+
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float m;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(m) : "f"(a), "f"(b), "f"(c));
+  return m;
 }
 
 template <int D>
@@ -115,6 +157,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
                   const __grid_constant__ CUtensorMap tv, const FwdParams p) {
   using Cfg = FwdCfg<D>;
   constexpr int kStages = Cfg::kStages;
+  constexpr int kRing = Cfg::kRing;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   FwdSmem<D>& s = *reinterpret_cast<FwdSmem<D>*>(smem_raw);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -129,7 +172,12 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
     tmem_relinquish();
   }
   if (tid == 0) {
+    for (int i = 0; i < kRing; ++i) {
+      mbar_init(&s.ring_full[i], 1);
+      mbar_init(&s.ring_empty[i], 9);  // MMA lane 0 + lane 0 of the 8 softmax warps
+    }
     mbar_init(&s.q_full, 1);
+    mbar_init(&s.q_empty, 1);
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&s.k_full[i], 1);
       mbar_init(&s.v_full[i], 1);
@@ -139,6 +187,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
       mbar_init(&s.s_full[g], 1);
       mbar_init(&s.p_full[g], 128);
       mbar_init(&s.o_full[g], 1);
+      mbar_init(&s.o_free[g], 128);
     }
     mbar_init(&s.teardown, 1);
     s.abort_flag = 0;
@@ -155,65 +204,70 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
   const WaitCtx w{&s.abort_flag, p.status, p.wait_limit_ns};
+  uint32_t q_par = 0, q_armed = 0, k_par[kStages] = {}, k_armed = 0;
 
-  // Per-role counters; every role walks the same tiles in the same order.
-  uint32_t kv_iter = 0;    // position in the K/V ring
-  uint32_t tile_cnt = 0;   // tiles processed (parity of s_full / p_full)
-  uint32_t act_cnt = 0;    // items with at least one tile (parity of q_full / o_full)
-  uint32_t q_par = 0, k_par[kStages] = {}, v_par[kStages] = {};  // producer: last armed phases
-  uint32_t k_armed = 0, q_armed = 0;
-
-  for (;;) {
-    if (tid == 0) s.item = s.abort_flag ? INT_MAX : atomicAdd(p.counter, 1);
-    __syncthreads();
-    const int item = s.item;
-    if (item >= p.n_items) break;
-    const ItemCoord c = decode_fwd_item(sh, p.order[item]);
-    const int b = c.b, qb = c.t, hkv = c.hkv;
-    const int h = hkv * sh.G + c.hg;
-    const int hm = (sh.Hm == 1) ? 0 : h;
-    const size_t lrow = ((size_t)b * sh.Hm + hm) * sh.nQB + qb;
-    const int* list = p.flist + lrow * sh.nKt;
-    const int n = p.fcount[lrow];
-
-    if (warp == Cfg::kProducerWarp) {
-      if (lane == 0 && n > 0) {
+  if (warp == Cfg::kProducerWarp) {
+    if (lane == 0) {
+      uint32_t kv_iter = 0, act = 0;
+      bool ok = true;
+      for (uint32_t k = 0; ok; ++k) {
+        const int slot = k % kRing;
+        if (!(ok = mbar_wait(&s.ring_empty[slot], ((k / kRing) & 1) ^ 1, w))) break;
+        const int item = s.abort_flag ? INT_MAX : atomicAdd(p.counter, 1);
+        s.ring_item[slot] = item;
+        mbar_arrive(&s.ring_full[slot]);
+        if (item >= p.n_items) break;
+        const FwdItem it = decode_fwd(p, item);
+        if (it.n == 0) continue;
+        if (!(ok = mbar_wait(&s.q_empty, (act & 1) ^ 1, w))) break;
         mbar_arrive_expect_tx(&s.q_full, 2 * Cfg::kTileBytes);
-        q_par = act_cnt & 1;
+        q_par = act & 1;
         q_armed = 1;
 #pragma unroll
         for (int g = 0; g < 2; ++g)
 #pragma unroll
           for (int bx = 0; bx < Cfg::kBoxes; ++bx)
-            tma_load_4d(s.q[g] + bx * 16384, &tq, &s.q_full, bx * 64, h, qb * 256 + g * kTile, b);
-        for (int t = 0; t < n; ++t, ++kv_iter) {
-          const int e = list[t];
+            tma_load_4d(s.q[g] + bx * 16384, &tq, &s.q_full, bx * 64, it.h, it.qb * 256 + g * kTile, it.b);
+        ++act;
+        for (int t = 0; t < it.n; ++t, ++kv_iter) {
+          const int e = it.list[t];
           const int kt = e >> 8;
           const bool need = ((e & 3) != kClsFull) || (((e >> 2) & 3) != kClsFull) || ((e >> 4) & 1);
           const int st = kv_iter % kStages;
           const uint32_t ph = (kv_iter / kStages) & 1;
-          if (!mbar_wait(&s.kv_empty[st], ph ^ 1, w)) break;
+          if (!(ok = mbar_wait(&s.kv_empty[st], ph ^ 1, w))) break;
           mbar_arrive_expect_tx(&s.k_full[st], Cfg::kTileBytes + (need ? kTile * 16 : 0));
 #pragma unroll
           for (int bx = 0; bx < Cfg::kBoxes; ++bx)
-            tma_load_4d(s.k[st] + bx * 16384, &tk, &s.k_full[st], bx * 64, hkv, kt * kTile, b);
+            tma_load_4d(s.k[st] + bx * 16384, &tk, &s.k_full[st], bx * 64, it.hkv, kt * kTile, it.b);
           if (need)
-            bulk_load(s.mask[st], p.rec + (((size_t)b * sh.Hm + hm) * sh.nKt + kt) * kTile, kTile * 16,
+            bulk_load(s.mask[st], p.rec + (((size_t)it.b * sh.Hm + it.hm) * sh.nKt + kt) * kTile, kTile * 16,
                       &s.k_full[st]);
           mbar_arrive_expect_tx(&s.v_full[st], Cfg::kTileBytes);
 #pragma unroll
           for (int bx = 0; bx < Cfg::kBoxes; ++bx)
-            tma_load_4d(s.v[st] + bx * 16384, &tv, &s.v_full[st], bx * 64, hkv, kt * kTile, b);
+            tma_load_4d(s.v[st] + bx * 16384, &tv, &s.v_full[st], bx * 64, it.hkv, kt * kTile, it.b);
           k_par[st] = ph;
-          v_par[st] = ph;
           k_armed |= 1u << st;
         }
       }
-    } else if (warp == Cfg::kMmaWarp) {
-      if (lane == 0 && n > 0) {
-        bool ok = mbar_wait(&s.q_full, act_cnt & 1, w);
+    }
+  } else if (warp == Cfg::kMmaWarp) {
+    if (lane == 0) {
+      uint32_t kv_iter = 0, tile_cnt = 0, act = 0;
+      bool ok = true;
+      for (uint32_t k = 0; ok; ++k) {
+        const int slot = k % kRing;
+        if (!(ok = mbar_wait(&s.ring_full[slot], (k / kRing) & 1, w))) break;
+        const int item = s.ring_item[slot];
+        mbar_arrive(&s.ring_empty[slot]);
+        if (item >= p.n_items) break;
+        const FwdItem it = decode_fwd(p, item);
+        const int n = it.n;
+        if (n == 0) continue;
+        if (!(ok = mbar_wait(&s.q_full, act & 1, w))) break;
         tc_fence_after();
-        for (int t = 0; ok && t < n; ++t) {
+        for (int t = 0; t < n; ++t) {
           const int st = kv_iter % kStages;
           const uint32_t ph = (kv_iter / kStages) & 1;
           const int st2 = (kv_iter + 1) % kStages;
@@ -225,8 +279,10 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
             mma_commit(&s.s_full[0]);
             issue_qk<D>(tmem + 128, s.q[1], s.k[st]);
             mma_commit(&s.s_full[1]);
+            if (n == 1) mma_commit(&s.q_empty);
           }
           if (!(ok = mbar_wait(&s.v_full[st], ph, w) && mbar_wait(&s.p_full[0], tile_cnt & 1, w))) break;
+          if (t == 0 && !(ok = mbar_wait(&s.o_free[0], (act & 1) ^ 1, w))) break;  // previous O0 read out
           tc_fence_after();
           issue_pv<D>(tmem + 256, tmem + 0, s.v[st], t > 0);
           if (t == n - 1) mma_commit(&s.o_full[0]);
@@ -237,6 +293,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
             mma_commit(&s.s_full[0]);
           }
           if (!(ok = mbar_wait(&s.p_full[1], tile_cnt & 1, w))) break;
+          if (t == 0 && !(ok = mbar_wait(&s.o_free[1], (act & 1) ^ 1, w))) break;
           tc_fence_after();
           issue_pv<D>(tmem + 256 + D, tmem + 128, s.v[st], t > 0);
           if (t == n - 1) mma_commit(&s.o_full[1]);
@@ -244,21 +301,37 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
           if (t + 1 < n) {
             issue_qk<D>(tmem + 128, s.q[1], s.k[st2]);
             mma_commit(&s.s_full[1]);
+            if (t + 2 == n) mma_commit(&s.q_empty);  // last QK^T of the item issued
           }
           ++kv_iter;
           ++tile_cnt;
         }
+        if (!ok) break;
+        ++act;
       }
-    } else {
-      // ---------------- softmax groups ----------------
-      const int g = warp >> 2, wq = warp & 3;
-      const int row = qb * 256 + g * kTile + wq * 32 + lane;
-      const uint32_t tb = tmem + ((uint32_t)(wq * 32) << 16);
-      const uint32_t s_col = g * 128, o_col = 256 + g * D;
-      float m_run = -INFINITY, l_run = 0.f;
-      bool ok = true;
+    }
+  } else {
+    // ---------------- softmax groups: thread = query row ----------------
+    const int g = warp >> 2, wq = warp & 3;
+    const uint32_t tb = tmem + ((uint32_t)(wq * 32) << 16);
+    const uint32_t s_col = g * 128, o_col = 256 + g * D;
+    const float sl2 = p.scale_log2;
+    uint32_t kv_iter = 0, tile_cnt = 0, act = 0;
+    bool ok = true;
+    for (uint32_t k = 0; ok; ++k) {
+      const int slot = k % kRing;
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(&s.ring_full[slot], (k / kRing) & 1, w)))) break;
+      const int item = s.ring_item[slot];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.ring_empty[slot]);
+      if (item >= p.n_items) break;
+      const FwdItem it = decode_fwd(p, item);
+      const int n = it.n;
+      const int rbase = it.qb * 256 + g * kTile + wq * 32;  // first row of this warp
+      const int row = rbase + lane;
+      float m_run = -INFINITY, l_run = 0.f;  // m_run in scaled log2 units
       for (int t = 0; t < n; ++t) {
-        const int e = list[t];
+        const int e = it.list[t];
         const int cls = (e >> (2 * g)) & 3;
         const bool need = (cls != kClsFull) || ((e >> 4) & 1);
         const int st = kv_iter % kStages;
@@ -267,40 +340,35 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
         if (need && ok) ok = __all_sync(0xffffffffu, mbar_wait(&s.k_full[st], ph, w));
         if (!ok) break;
         tc_fence_after();
-        uint32_t raw[128];
-        tmem_ld32p(tb + s_col + 0, raw + 0);
-        tmem_ld32p(tb + s_col + 32, raw + 32);
-        tmem_ld32p(tb + s_col + 64, raw + 64);
-        tmem_ld32p(tb + s_col + 96, raw + 96);
-        tmem_ld_wait();
         float x[128];
-#pragma unroll
-        for (int i = 0; i < 128; ++i) x[i] = __uint_as_float(raw[i]) * p.scale_log2;
+        uint32_t* raw = reinterpret_cast<uint32_t*>(x);
+        tmem_ld32x(tb + s_col + 0, raw + 0);
+        tmem_ld32x(tb + s_col + 32, raw + 32);
+        tmem_ld32x(tb + s_col + 64, raw + 64);
+        tmem_ld32x(tb + s_col + 96, raw + 96);
+        uint32_t mw[4] = {0u, 0u, 0u, 0u};
         if (need) {
-          // Bit j of word c: column 32c + j is masked for this row.  Built with
-          // a rolled loop (the boundary records are smem broadcasts), then
-          // applied with bit tests on the unrolled register array.
+          // column words (this lane's 4 columns) -> row words by transposition
           const int4* mrec = s.mask[st];
 #pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t bits = 0;
-#pragma unroll 4
-            for (int j = 0; j < 32; ++j) {
-              const int4 r = mrec[c * 32 + j];
-              const bool masked = (r.x <= row && row < r.y) || (r.z <= row && row < r.w);
-              bits |= (masked ? 1u : 0u) << j;
-            }
-#pragma unroll
-            for (int j = 0; j < 32; ++j) x[c * 32 + j] = ((bits >> j) & 1u) ? -INFINITY : x[c * 32 + j];
-          }
+          for (int c = 0; c < 4; ++c) mw[c] = warp_transpose32(column_row_bits(mrec[c * 32 + lane], rbase), lane);
         }
-        float mx8[8];
+        tmem_ld_wait();
+        if (need) {
 #pragma unroll
-        for (int j = 0; j < 8; ++j) mx8[j] = x[j];
+          for (int i = 0; i < 128; ++i) x[i] = ((mw[i >> 5] >> (i & 31)) & 1u) ? -INFINITY : x[i];
+        }
+        // row maximum of the raw logits (the scale is positive)
+        float m4[4];
 #pragma unroll
-        for (int i = 8; i < 128; ++i) mx8[i & 7] = fmaxf(mx8[i & 7], x[i]);
-        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        for (int j = 0; j < 4; ++j) m4[j] = max3f(x[j], x[4 + j], x[8 + j]);
+#pragma unroll
+        for (int i = 12; i + 7 < 128; i += 8)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) m4[j] = max3f(m4[j], x[i + j], x[i + 4 + j]);
+        m4[0] = max3f(m4[0], x[124], x[125]);
+        m4[1] = max3f(m4[1], x[126], x[127]);
+        const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl2;
         // Lazy rescale: only when the maximum grows by more than 8 (log2 units).
         float alpha = 1.f;
         bool rescale = false;
@@ -310,32 +378,33 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
           m_run = mx;
           l_run *= alpha;
         }
-        const float mref = (m_run == -INFINITY) ? 0.f : m_run;
-        float sum4[4] = {0.f, 0.f, 0.f, 0.f};
+        const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
+        float sa = 0.f, sb = 0.f;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {  // 32 columns -> 16 packed bf16 pairs per store
           uint32_t pk[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const float a0 = fast_exp2(x[c * 32 + 2 * i] - mref);
-            const float a1 = fast_exp2(x[c * 32 + 2 * i + 1] - mref);
-            sum4[i & 3] += a0 + a1;
+            const float a0 = fast_exp2(fmaf(x[c * 32 + 2 * i], sl2, neg_m));
+            const float a1 = fast_exp2(fmaf(x[c * 32 + 2 * i + 1], sl2, neg_m));
+            sa += a0;
+            sb += a1;
             pk[i] = pack_bf16x2(a0, a1);
           }
           tmem_st16(tb + s_col + c * 16, pk);
         }
-        l_run += (sum4[0] + sum4[1]) + (sum4[2] + sum4[3]);
+        l_run += sa + sb;
         // O correction (the previous P V of this q-tile has completed: the
         // commit that signalled this S was issued after it).
         if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             uint32_t o[32];
-            tmem_ld32p(tb + o_col + c * 32, o);
+            tmem_ld32x(tb + o_col + c * 32, o);
             tmem_ld_wait();
 #pragma unroll
             for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st32p(tb + o_col + c * 32, o);
+            tmem_st32x(tb + o_col + c * 32, o);
           }
         }
         tmem_st_wait();
@@ -344,46 +413,46 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
         ++kv_iter;
         ++tile_cnt;
       }
+      if (!ok) break;
       // ---------------- epilogue ----------------
-      if (ok && n > 0) ok = __all_sync(0xffffffffu, mbar_wait(&s.o_full[g], act_cnt & 1, w));
-      if (ok) {
-        tc_fence_after();
-        const bool valid = row < sh.Nq;
-        const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
-        __nv_bfloat16* orow = p.o + (((size_t)b * sh.Nq + (valid ? row : 0)) * sh.Hq + h) * D;
+      if (n > 0 && !(ok = __all_sync(0xffffffffu, mbar_wait(&s.o_full[g], act & 1, w)))) break;
+      tc_fence_after();
+      const bool valid = row < sh.Nq;
+      const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
+      __nv_bfloat16* orow = p.o + (((size_t)it.b * sh.Nq + (valid ? row : 0)) * sh.Hq + it.h) * D;
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          if (n > 0) {
-            tmem_ld32p(tb + o_col + c * 32, o);
-            tmem_ld_wait();
-          } else {
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        if (n > 0) {
+          tmem_ld32x(tb + o_col + c * 32, o);
+          tmem_ld_wait();
+        } else {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = 0u;
-          }
-          uint32_t pkd[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i)
-            pkd[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
-          if (valid) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-              dst[i] = make_uint4(pkd[4 * i], pkd[4 * i + 1], pkd[4 * i + 2], pkd[4 * i + 3]);
-          }
+          for (int i = 0; i < 32; ++i) o[i] = 0u;
         }
-        if (valid)
-          p.lse[((size_t)b * sh.Hq + h) * sh.Nq + row] =
-              (l_run > 0.f) ? (m_run + log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+        uint32_t pkd[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          pkd[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
+        if (valid) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pkd[4 * i], pkd[4 * i + 1], pkd[4 * i + 2], pkd[4 * i + 3]);
+        }
       }
+      if (n > 0) {
+        tc_fence_before();
+        mbar_arrive(&s.o_free[g]);
+        ++act;
+      }
+      if (valid)
+        p.lse[((size_t)it.b * sh.Hq + it.h) * sh.Nq + row] =
+            (l_run > 0.f) ? (m_run + log2f(l_run)) * 0.69314718055994531f : -INFINITY;
     }
-    if (n > 0) ++act_cnt;
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
   }
 
   // ---------------- teardown ----------------
+  __syncthreads();
   if (s.abort_flag) {
     // Let copies and MMAs that are still in flight land before the CTA's
     // shared memory and tensor memory are released.
@@ -397,7 +466,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
       for (int st = 0; st < kStages; ++st)
         if (k_armed & (1u << st)) {
           (void)mbar_wait(&s.k_full[st], k_par[st], w2);
-          (void)mbar_wait(&s.v_full[st], v_par[st], w2);
+          (void)mbar_wait(&s.v_full[st], k_par[st], w2);
         }
     }
   }
