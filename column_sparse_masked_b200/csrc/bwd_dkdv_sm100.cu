@@ -16,6 +16,9 @@
 // The MMA warp issues, per q-tile t:
 //   ... dV(t) = P^T(t) dO(t) ; S^T(t+1) = K Q(t+1)^T ; dK(t) = dS^T(t) Q(t) ;
 //   dP^T(t+1) = V dO(t+1)^T ...
+// Q tiles (3-deep ring, freed after dK), dO tiles (2-deep, freed after dV)
+// and the rows' LSE2 / D (2-deep, freed by the compute warps) stream through
+// separate rings, so each is refilled as soon as its last reader is done.
 // Tensor-core instructions of one thread execute in issue order, so S^T(t+1)
 // may overwrite the S^T region right after dV(t) (which reads P^T(t) from it)
 // and dP^T(t+1) right after dK(t).  While the tensor core runs dV(t)+S^T(t+1)
@@ -41,7 +44,9 @@ namespace kvb {
 constexpr int kThreads = 320;
 constexpr int kProducerWarp = 8, kMmaWarp = 9;
 constexpr int kRing = 4;
-constexpr int kStages = 2;
+constexpr int kQStages = 3;   // Q tiles: last read by dK(t)
+constexpr int kDoStages = 2;  // dO tiles: last read by dV(t), freed earlier
+constexpr int kLStages = 2;   // LSE2 / D rows: last read by the compute warps
 constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256;
 }  // namespace kvb
 
@@ -49,14 +54,16 @@ template <int D>
 struct __align__(1024) DkdvSmem {
   uint8_t k[kTile * D * 2];
   uint8_t v[kTile * D * 2];
-  uint8_t q[kvb::kStages][kTile * D * 2];
-  uint8_t dout[kvb::kStages][kTile * D * 2];
-  float lse2[kvb::kStages][kTile];
-  float dsum[kvb::kStages][kTile];
+  uint8_t q[kvb::kQStages][kTile * D * 2];
+  uint8_t dout[kvb::kDoStages][kTile * D * 2];
+  float lse2[kvb::kLStages][kTile];
+  float dsum[kvb::kLStages][kTile];
   int ring_item[kvb::kRing];
   uint64_t ring_full[kvb::kRing], ring_empty[kvb::kRing];
   uint64_t kv_full, kv_empty;
-  uint64_t qd_full[kvb::kStages], qd_empty[kvb::kStages];
+  uint64_t q_full[kvb::kQStages], q_empty[kvb::kQStages];
+  uint64_t do_full[kvb::kDoStages], do_empty[kvb::kDoStages];
+  uint64_t l_full[kvb::kLStages], l_empty[kvb::kLStages];
   uint64_t s_full, dp_full, p_full, ds_full;
   uint64_t s_read, dp_read;  // both compute warpgroups have loaded S^T / dP^T (bf16 results overlap them)
   uint64_t dkdv_full, dkdv_free;
@@ -65,6 +72,9 @@ struct __align__(1024) DkdvSmem {
   int abort_flag;
   int no_abort;
 };
+
+static_assert(sizeof(DkdvSmem<128>) <= 232448, "key-side shared memory exceeds the per-CTA limit");
+static_assert(sizeof(DkdvSmem<64>) <= 232448, "key-side shared memory exceeds the per-CTA limit");
 
 struct KvItem {
   int b, hkv, kt, total;  // total = q-tiles over all q-heads of the group
@@ -157,9 +167,17 @@ __global__ void __launch_bounds__(kvb::kThreads, 1)
     }
     mbar_init(&s.kv_full, 1);
     mbar_init(&s.kv_empty, 1);
-    for (int i = 0; i < kStages; ++i) {
-      mbar_init(&s.qd_full[i], 1);
-      mbar_init(&s.qd_empty[i], 1);
+    for (int i = 0; i < kQStages; ++i) {
+      mbar_init(&s.q_full[i], 1);
+      mbar_init(&s.q_empty[i], 1);
+    }
+    for (int i = 0; i < kDoStages; ++i) {
+      mbar_init(&s.do_full[i], 1);
+      mbar_init(&s.do_empty[i], 1);
+    }
+    for (int i = 0; i < kLStages; ++i) {
+      mbar_init(&s.l_full[i], 1);
+      mbar_init(&s.l_empty[i], 256);
     }
     mbar_init(&s.s_full, 1);
     mbar_init(&s.dp_full, 1);
@@ -185,7 +203,8 @@ __global__ void __launch_bounds__(kvb::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
   const WaitCtx w{&s.abort_flag, p.status, p.wait_limit_ns};
-  uint32_t kv_par = 0, kv_armed = 0, qd_par[kStages] = {}, qd_armed = 0;
+  uint32_t kv_par = 0, kv_armed = 0, q_par[kQStages] = {}, do_par[kDoStages] = {}, l_par[kLStages] = {};
+  uint32_t q_armed = 0, do_armed = 0, l_armed = 0;
 
   if (warp == kProducerWarp) {
     if (lane == 0) {
@@ -211,20 +230,29 @@ __global__ void __launch_bounds__(kvb::kThreads, 1)
         }
         ++act;
         ok = for_each_qtile(p, it, [&](int, int h, int, int qt, int) {
-          const int st = sq % kStages;
-          const uint32_t ph = (sq / kStages) & 1;
-          if (!mbar_wait(&s.qd_empty[st], ph ^ 1, w)) return false;
-          mbar_arrive_expect_tx(&s.qd_full[st], 2 * kTileBytes + 2 * kTile * 4);
+          const int sqi = sq % kQStages, sdo = sq % kDoStages, sl = sq % kLStages;
+          const uint32_t pq = (sq / kQStages) & 1, pd = (sq / kDoStages) & 1, pl = (sq / kLStages) & 1;
+          if (!mbar_wait(&s.q_empty[sqi], pq ^ 1, w)) return false;
+          mbar_arrive_expect_tx(&s.q_full[sqi], kTileBytes);
 #pragma unroll
-          for (int bx = 0; bx < kBoxes; ++bx) {
-            tma_load_4d(s.q[st] + bx * 16384, &tq, &s.qd_full[st], bx * 64, h, qt * kTile, it.b);
-            tma_load_4d(s.dout[st] + bx * 16384, &tdo, &s.qd_full[st], bx * 64, h, qt * kTile, it.b);
-          }
+          for (int bx = 0; bx < kBoxes; ++bx)
+            tma_load_4d(s.q[sqi] + bx * 16384, &tq, &s.q_full[sqi], bx * 64, h, qt * kTile, it.b);
+          q_par[sqi] = pq;
+          q_armed |= 1u << sqi;
+          if (!mbar_wait(&s.do_empty[sdo], pd ^ 1, w)) return false;
+          mbar_arrive_expect_tx(&s.do_full[sdo], kTileBytes);
+#pragma unroll
+          for (int bx = 0; bx < kBoxes; ++bx)
+            tma_load_4d(s.dout[sdo] + bx * 16384, &tdo, &s.do_full[sdo], bx * 64, h, qt * kTile, it.b);
+          do_par[sdo] = pd;
+          do_armed |= 1u << sdo;
+          if (!mbar_wait(&s.l_empty[sl], pl ^ 1, w)) return false;
+          mbar_arrive_expect_tx(&s.l_full[sl], 2 * kTile * 4);
           const size_t roff = ((size_t)it.b * sh.Hq + h) * sh.nQt * kTile + (size_t)qt * kTile;
-          bulk_load(s.lse2[st], p.lse2 + roff, kTile * 4, &s.qd_full[st]);
-          bulk_load(s.dsum[st], p.dsum + roff, kTile * 4, &s.qd_full[st]);
-          qd_par[st] = ph;
-          qd_armed |= 1u << st;
+          bulk_load(s.lse2[sl], p.lse2 + roff, kTile * 4, &s.l_full[sl]);
+          bulk_load(s.dsum[sl], p.dsum + roff, kTile * 4, &s.l_full[sl]);
+          l_par[sl] = pl;
+          l_armed |= 1u << sl;
           ++sq;
           return true;
         });
@@ -246,34 +274,40 @@ __global__ void __launch_bounds__(kvb::kThreads, 1)
         if (!(ok = mbar_wait(&s.kv_full, act & 1, w))) break;
         // first q-tile: S^T and dP^T
         {
-          const int st = sq % kStages;
-          if (!(ok = mbar_wait(&s.qd_full[st], (sq / kStages) & 1, w))) break;
+          const int sqi = sq % kQStages, sdo = sq % kDoStages;
+          if (!(ok = mbar_wait(&s.q_full[sqi], (sq / kQStages) & 1, w))) break;
           tc_fence_after();
-          kv_issue_ss<D>(tmem + kColS, s.k, s.q[st]);
+          kv_issue_ss<D>(tmem + kColS, s.k, s.q[sqi]);
           mma_commit(&s.s_full);
-          kv_issue_ss<D>(tmem + kColDP, s.v, s.dout[st]);
+          if (!(ok = mbar_wait(&s.do_full[sdo], (sq / kDoStages) & 1, w))) break;
+          tc_fence_after();
+          kv_issue_ss<D>(tmem + kColDP, s.v, s.dout[sdo]);
           mma_commit(&s.dp_full);
         }
         for (int j = 0; j < n; ++j) {
           const uint32_t sj = sq + j, tj = tc + j;
-          const int st = sj % kStages, st2 = (sj + 1) % kStages;
+          const int sqi = sj % kQStages, sdo = sj % kDoStages;
+          const int sqi2 = (sj + 1) % kQStages, sdo2 = (sj + 1) % kDoStages;
           const uint32_t par = tj & 1;
           if (j == 0 && !(ok = mbar_wait(&s.dkdv_free, (act & 1) ^ 1, w))) break;  // previous item read out
           if (!(ok = mbar_wait(&s.p_full, par, w))) break;
           tc_fence_after();
-          kv_issue_ts<D>(tmem + kColDV, tmem + kColS, s.dout[st], j > 0);  // dV += P^T dO
+          kv_issue_ts<D>(tmem + kColDV, tmem + kColS, s.dout[sdo], j > 0);  // dV += P^T dO
+          mma_commit(&s.do_empty[sdo]);                                     // dO(j) read for the last time
           if (j + 1 < n) {
-            if (!(ok = mbar_wait(&s.qd_full[st2], ((sj + 1) / kStages) & 1, w))) break;
+            if (!(ok = mbar_wait(&s.q_full[sqi2], ((sj + 1) / kQStages) & 1, w))) break;
             tc_fence_after();
-            kv_issue_ss<D>(tmem + kColS, s.k, s.q[st2]);  // S^T(j+1), after dV(j) read P^T(j)
+            kv_issue_ss<D>(tmem + kColS, s.k, s.q[sqi2]);  // S^T(j+1), after dV(j) read P^T(j)
             mma_commit(&s.s_full);
           }
           if (!(ok = mbar_wait(&s.ds_full, par, w))) break;
           tc_fence_after();
-          kv_issue_ts<D>(tmem + kColDK, tmem + kColDP, s.q[st], j > 0);  // dK += dS^T Q
-          mma_commit(&s.qd_empty[st]);
+          kv_issue_ts<D>(tmem + kColDK, tmem + kColDP, s.q[sqi], j > 0);  // dK += dS^T Q
+          mma_commit(&s.q_empty[sqi]);                                     // Q(j) read for the last time
           if (j + 1 < n) {
-            kv_issue_ss<D>(tmem + kColDP, s.v, s.dout[st2]);  // dP^T(j+1), after dK(j) read dS^T(j)
+            if (!(ok = mbar_wait(&s.do_full[sdo2], ((sj + 1) / kDoStages) & 1, w))) break;
+            tc_fence_after();
+            kv_issue_ss<D>(tmem + kColDP, s.v, s.dout[sdo2]);  // dP^T(j+1), after dK(j) read dS^T(j)
             mma_commit(&s.dp_full);
           }
         }
@@ -310,13 +344,13 @@ __global__ void __launch_bounds__(kvb::kThreads, 1)
             rec = p.rec[(((size_t)it.b * sh.Hm + hm) * sh.nKt + it.kt) * kTile + jl];
             cur_hm = hm;
           }
-          const int st = sq % kStages;
+          const int sl = sq % kLStages;
           const uint32_t par = tc & 1;
           if (!__all_sync(0xffffffffu, mbar_wait(&s.s_full, par, w))) return false;
-          if (!__all_sync(0xffffffffu, mbar_wait(&s.qd_full[st], (sq / kStages) & 1, w))) return false;
+          if (!__all_sync(0xffffffffu, mbar_wait(&s.l_full[sl], (sq / kLStages) & 1, w))) return false;
           tc_fence_after();
-          const float* l2 = s.lse2[st] + c0;
-          const float* dsm = s.dsum[st] + c0;
+          const float* l2 = s.lse2[sl] + c0;
+          const float* dsm = s.dsum[sl] + c0;
           const bool need = cls == kClsPartial;
           const int row0 = qt * kTile + c0;
           // P^T for 64 query columns, in place over the loaded S^T values
@@ -378,6 +412,7 @@ __global__ void __launch_bounds__(kvb::kThreads, 1)
           tmem_st_wait();
           tc_fence_before();
           mbar_arrive(&s.ds_full);
+          mbar_arrive(&s.l_empty[sl]);  // LSE2 / D of this q-tile no longer read
           ++sq;
           ++tc;
           return true;
@@ -429,8 +464,12 @@ __global__ void __launch_bounds__(kvb::kThreads, 1)
     }
     if (warp == kProducerWarp && lane == 0) {
       if (kv_armed) (void)mbar_wait(&s.kv_full, kv_par, w2);
-      for (int st = 0; st < kStages; ++st)
-        if (qd_armed & (1u << st)) (void)mbar_wait(&s.qd_full[st], qd_par[st], w2);
+      for (int st = 0; st < kQStages; ++st)
+        if (q_armed & (1u << st)) (void)mbar_wait(&s.q_full[st], q_par[st], w2);
+      for (int st = 0; st < kDoStages; ++st)
+        if (do_armed & (1u << st)) (void)mbar_wait(&s.do_full[st], do_par[st], w2);
+      for (int st = 0; st < kLStages; ++st)
+        if (l_armed & (1u << st)) (void)mbar_wait(&s.l_full[st], l_par[st], w2);
     }
   }
   tc_fence_before();

@@ -16,6 +16,10 @@
 // TMEM (512 columns): S[0] [0,128), S[1] [128,256) (dS bf16 written over the
 // S buffer of its tile), dP [256,384), dQ [384, 384+d).
 // MMA issue order: S(0) dP(0) | S(t+1) , dQ += dS(t) K(t) , dP(t+1) | ...
+// K tiles (3-deep ring, freed after dQ) and V tiles (2-deep, freed after dP)
+// stream through separate rings; the element mask of a partial tile is built
+// from the boundary records read straight from global memory (L2-resident),
+// turned into per-row bit words by a warp bit-transpose.
 // While the tensor core runs S(t+1) and dQ(t) the compute warps turn
 // S(t+1)/dP(t+1) into dS(t+1).
 //
@@ -38,7 +42,8 @@ namespace qb {
 constexpr int kThreads = 320;
 constexpr int kProducerWarp = 8, kMmaWarp = 9;
 constexpr int kRing = 4;
-constexpr int kStages = 2;
+constexpr int kKStages = 3;  // K tiles: last read by dQ(t)
+constexpr int kVStages = 2;  // V tiles: last read by dP(t), freed earlier
 constexpr uint32_t kColS = 0, kColDP = 256, kColDQ = 384;
 }  // namespace qb
 
@@ -46,13 +51,13 @@ template <int D>
 struct __align__(1024) DqSmem {
   uint8_t q[kTile * D * 2];
   uint8_t dout[kTile * D * 2];
-  uint8_t k[qb::kStages][kTile * D * 2];
-  uint8_t v[qb::kStages][kTile * D * 2];
-  int4 mask[qb::kStages][kTile];
+  uint8_t k[qb::kKStages][kTile * D * 2];
+  uint8_t v[qb::kVStages][kTile * D * 2];
   int ring_item[qb::kRing];
   uint64_t ring_full[qb::kRing], ring_empty[qb::kRing];
   uint64_t q_full, q_empty;
-  uint64_t k_full[qb::kStages], v_full[qb::kStages], kv_empty[qb::kStages];
+  uint64_t k_full[qb::kKStages], k_empty[qb::kKStages];
+  uint64_t v_full[qb::kVStages], v_empty[qb::kVStages];
   uint64_t s_full[2], dp_full, sd_read, ds_full;
   uint64_t dq_full, dq_free;
   uint64_t teardown;
@@ -60,6 +65,9 @@ struct __align__(1024) DqSmem {
   int abort_flag;
   int no_abort;
 };
+
+static_assert(sizeof(DqSmem<128>) <= 232448, "query-side shared memory exceeds the per-CTA limit");
+static_assert(sizeof(DqSmem<64>) <= 232448, "query-side shared memory exceeds the per-CTA limit");
 
 struct QItem {
   int b, h, hm, qt, g;
@@ -149,10 +157,13 @@ __global__ void __launch_bounds__(qb::kThreads, 1)
     }
     mbar_init(&s.q_full, 1);
     mbar_init(&s.q_empty, 1);
-    for (int i = 0; i < kStages; ++i) {
+    for (int i = 0; i < kKStages; ++i) {
       mbar_init(&s.k_full[i], 1);
+      mbar_init(&s.k_empty[i], 1);
+    }
+    for (int i = 0; i < kVStages; ++i) {
       mbar_init(&s.v_full[i], 1);
-      mbar_init(&s.kv_empty[i], 1);
+      mbar_init(&s.v_empty[i], 1);
     }
     mbar_init(&s.s_full[0], 1);
     mbar_init(&s.s_full[1], 1);
@@ -177,7 +188,7 @@ __global__ void __launch_bounds__(qb::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
   const WaitCtx w{&s.abort_flag, p.status, p.wait_limit_ns};
-  uint32_t q_par = 0, q_armed = 0, k_par[kStages] = {}, kv_armed = 0;
+  uint32_t q_par = 0, q_armed = 0, k_par[kKStages] = {}, v_par[kVStages] = {}, k_armed = 0, v_armed = 0;
 
   if (warp == kProducerWarp) {
     if (lane == 0) {
@@ -202,25 +213,24 @@ __global__ void __launch_bounds__(qb::kThreads, 1)
           tma_load_4d(s.dout + bx * 16384, &tdo, &s.q_full, bx * 64, it.h, it.qt * kTile, it.b);
         }
         ++act;
-        ok = for_each_ktile(it, [&](int kt, int cls) {
-          const int st = kv_iter % kStages;
-          const uint32_t ph = (kv_iter / kStages) & 1;
-          if (!mbar_wait(&s.kv_empty[st], ph ^ 1, w)) return false;
-          const bool need = cls == kClsPartial;
+        ok = for_each_ktile(it, [&](int kt, int) {
+          const int sk = kv_iter % kKStages, sv = kv_iter % kVStages;
+          const uint32_t pk = (kv_iter / kKStages) & 1, pv = (kv_iter / kVStages) & 1;
           const int hkv = it.h / sh.G;
-          mbar_arrive_expect_tx(&s.k_full[st], kTileBytes + (need ? kTile * 16 : 0));
+          if (!mbar_wait(&s.k_empty[sk], pk ^ 1, w)) return false;
+          mbar_arrive_expect_tx(&s.k_full[sk], kTileBytes);
 #pragma unroll
           for (int bx = 0; bx < kBoxes; ++bx)
-            tma_load_4d(s.k[st] + bx * 16384, &tk, &s.k_full[st], bx * 64, hkv, kt * kTile, it.b);
-          if (need)
-            bulk_load(s.mask[st], p.rec + (((size_t)it.b * sh.Hm + it.hm) * sh.nKt + kt) * kTile, kTile * 16,
-                      &s.k_full[st]);
-          mbar_arrive_expect_tx(&s.v_full[st], kTileBytes);
+            tma_load_4d(s.k[sk] + bx * 16384, &tk, &s.k_full[sk], bx * 64, hkv, kt * kTile, it.b);
+          k_par[sk] = pk;
+          k_armed |= 1u << sk;
+          if (!mbar_wait(&s.v_empty[sv], pv ^ 1, w)) return false;
+          mbar_arrive_expect_tx(&s.v_full[sv], kTileBytes);
 #pragma unroll
           for (int bx = 0; bx < kBoxes; ++bx)
-            tma_load_4d(s.v[st] + bx * 16384, &tv, &s.v_full[st], bx * 64, hkv, kt * kTile, it.b);
-          k_par[st] = ph;
-          kv_armed |= 1u << st;
+            tma_load_4d(s.v[sv] + bx * 16384, &tv, &s.v_full[sv], bx * 64, hkv, kt * kTile, it.b);
+          v_par[sv] = pv;
+          v_armed |= 1u << sv;
           ++kv_iter;
           return true;
         });
@@ -240,40 +250,41 @@ __global__ void __launch_bounds__(qb::kThreads, 1)
         const int n = it.n;
         if (n == 0) continue;
         if (!(ok = mbar_wait(&s.q_full, act & 1, w))) break;
-        // tile j uses K/V stage (kv_iter + j) % kStages and S buffer (tc + j) & 1
+        // tile j uses K stage (kv_iter + j) % kKStages, V stage (kv_iter + j) % kVStages
+        // and S buffer (tc + j) & 1
         {
-          const int st = kv_iter % kStages;
-          const uint32_t ph = (kv_iter / kStages) & 1;
-          if (!(ok = mbar_wait(&s.k_full[st], ph, w))) break;
+          const int sk = kv_iter % kKStages, sv = kv_iter % kVStages;
+          if (!(ok = mbar_wait(&s.k_full[sk], (kv_iter / kKStages) & 1, w))) break;
           tc_fence_after();
-          q_issue_ss<D>(tmem + kColS + (tc & 1) * 128, s.q, s.k[st]);
+          q_issue_ss<D>(tmem + kColS + (tc & 1) * 128, s.q, s.k[sk]);
           mma_commit(&s.s_full[tc & 1]);
-          if (!(ok = mbar_wait(&s.v_full[st], ph, w))) break;
+          if (!(ok = mbar_wait(&s.v_full[sv], (kv_iter / kVStages) & 1, w))) break;
           tc_fence_after();
-          q_issue_ss<D>(tmem + kColDP, s.dout, s.v[st]);
+          q_issue_ss<D>(tmem + kColDP, s.dout, s.v[sv]);
           mma_commit(&s.dp_full);
+          mma_commit(&s.v_empty[sv]);
         }
         for (int j = 0; j < n; ++j) {
           const uint32_t kj = kv_iter + j, tj = tc + j;
-          const int st = kj % kStages, st2 = (kj + 1) % kStages;
-          const uint32_t ph2 = ((kj + 1) / kStages) & 1;
+          const int sk = kj % kKStages, sk2 = (kj + 1) % kKStages, sv2 = (kj + 1) % kVStages;
           const int bf = tj & 1;
           if (j + 1 < n) {
-            if (!(ok = mbar_wait(&s.k_full[st2], ph2, w))) break;
+            if (!(ok = mbar_wait(&s.k_full[sk2], ((kj + 1) / kKStages) & 1, w))) break;
             tc_fence_after();
-            q_issue_ss<D>(tmem + kColS + (bf ^ 1) * 128, s.q, s.k[st2]);  // S(j+1): its buffer held dS(j-1)
+            q_issue_ss<D>(tmem + kColS + (bf ^ 1) * 128, s.q, s.k[sk2]);  // S(j+1): its buffer held dS(j-1)
             mma_commit(&s.s_full[bf ^ 1]);
           }
           if (j == 0 && !(ok = mbar_wait(&s.dq_free, (act & 1) ^ 1, w))) break;  // previous dQ read out
           if (!(ok = mbar_wait(&s.ds_full, tj & 1, w))) break;
           tc_fence_after();
-          q_issue_dq<D>(tmem + kColDQ, tmem + kColS + bf * 128, s.k[st], j > 0);  // dQ += dS K
-          mma_commit(&s.kv_empty[st]);
+          q_issue_dq<D>(tmem + kColDQ, tmem + kColS + bf * 128, s.k[sk], j > 0);  // dQ += dS K
+          mma_commit(&s.k_empty[sk]);
           if (j + 1 < n) {
-            if (!(ok = mbar_wait(&s.v_full[st2], ph2, w))) break;
+            if (!(ok = mbar_wait(&s.v_full[sv2], ((kj + 1) / kVStages) & 1, w))) break;
             tc_fence_after();
-            q_issue_ss<D>(tmem + kColDP, s.dout, s.v[st2]);  // dP(j+1): dP(j) was read before ds_full(j)
+            q_issue_ss<D>(tmem + kColDP, s.dout, s.v[sv2]);  // dP(j+1): dP(j) was read before ds_full(j)
             mma_commit(&s.dp_full);
+            mma_commit(&s.v_empty[sv2]);
           }
         }
         if (!ok) break;
@@ -290,7 +301,7 @@ __global__ void __launch_bounds__(qb::kThreads, 1)
     const int rl = wq * 32 + lane;  // row within the q-tile
     const uint32_t tb = tmem + ((uint32_t)(wq * 32) << 16);
     const uint32_t c0 = wg * 64;
-    uint32_t kv_iter = 0, tc = 0, act = 0;
+    uint32_t tc = 0, act = 0;
     bool ok = true;
     for (uint32_t k = 0; ok; ++k) {
       const int slot = k % kRing;
@@ -315,38 +326,35 @@ __global__ void __launch_bounds__(qb::kThreads, 1)
       const size_t roff = ((size_t)it.b * sh.Hq + it.h) * sh.nQt * kTile + (size_t)it.qt * kTile + rl;
       const float lse2 = p.lse2[roff];
       const float drow = p.dsum[roff];
-      ok = for_each_ktile(it, [&](int, int cls) {
-        const int st = kv_iter % kStages;
+      const int4* recs = p.rec + ((size_t)it.b * sh.Hm + it.hm) * sh.nKt * kTile;
+      const int rbase = it.qt * kTile + wq * 32;  // first row of this warp
+      ok = for_each_ktile(it, [&](int kt, int cls) {
         const int bf = tc & 1;
+        const bool need = cls == kClsPartial;
+        // this lane's two key columns of the warpgroup's half (read early; L2-resident)
+        int4 ra = make_int4(0, 0, 0, 0), rb = ra;
+        if (need) {
+          ra = recs[(size_t)kt * kTile + c0 + lane];
+          rb = recs[(size_t)kt * kTile + c0 + 32 + lane];
+        }
         if (!__all_sync(0xffffffffu, mbar_wait(&s.s_full[bf], (tc >> 1) & 1, w))) return false;
         if (!__all_sync(0xffffffffu, mbar_wait(&s.dp_full, tc & 1, w))) return false;
-        const bool need = cls == kClsPartial;
-        if (need && !__all_sync(0xffffffffu, mbar_wait(&s.k_full[st], (kv_iter / kStages) & 1, w))) return false;
         tc_fence_after();
         uint32_t sv[64], dv[64];
         tmem_ld32x(tb + kColS + bf * 128 + c0, sv);
         tmem_ld32x(tb + kColS + bf * 128 + c0 + 32, sv + 32);
         tmem_ld32x(tb + kColDP + c0, dv);
         tmem_ld32x(tb + kColDP + c0 + 32, dv + 32);
+        uint32_t mbits0 = 0, mbits1 = 0;
+        if (need) {  // per-column row words, transposed to per-row column words
+          mbits0 = warp_transpose32(column_row_bits(ra, rbase), lane);
+          mbits1 = warp_transpose32(column_row_bits(rb, rbase), lane);
+        }
         tmem_ld_wait();
         // dS of key columns 64-127 is written into TMEM columns 32-63 of the S
         // buffer (S of columns 32-63): both warpgroups must have loaded first.
         tc_fence_before();
         mbar_arrive(&s.sd_read);
-        uint32_t mbits0 = 0, mbits1 = 0;
-        if (need) {
-          const int4* mrec = s.mask[st] + c0;
-#pragma unroll 4
-          for (int j = 0; j < 32; ++j) {
-            const int4 r = mrec[j];
-            mbits0 |= (((r.x <= row && row < r.y) || (r.z <= row && row < r.w)) ? 1u : 0u) << j;
-          }
-#pragma unroll 4
-          for (int j = 0; j < 32; ++j) {
-            const int4 r = mrec[32 + j];
-            mbits1 |= (((r.x <= row && row < r.y) || (r.z <= row && row < r.w)) ? 1u : 0u) << j;
-          }
-        }
 #pragma unroll
         for (int i = 0; i < 64; ++i) {
           float pv = fast_exp2(__uint_as_float(sv[i]) * p.scale_log2 - lse2);
@@ -363,7 +371,6 @@ __global__ void __launch_bounds__(qb::kThreads, 1)
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&s.ds_full);
-        ++kv_iter;
         ++tc;
         return true;
       });
@@ -402,11 +409,10 @@ __global__ void __launch_bounds__(qb::kThreads, 1)
     }
     if (warp == kProducerWarp && lane == 0) {
       if (q_armed) (void)mbar_wait(&s.q_full, q_par, w2);
-      for (int st = 0; st < kStages; ++st)
-        if (kv_armed & (1u << st)) {
-          (void)mbar_wait(&s.k_full[st], k_par[st], w2);
-          (void)mbar_wait(&s.v_full[st], k_par[st], w2);
-        }
+      for (int st = 0; st < kKStages; ++st)
+        if (k_armed & (1u << st)) (void)mbar_wait(&s.k_full[st], k_par[st], w2);
+      for (int st = 0; st < kVStages; ++st)
+        if (v_armed & (1u << st)) (void)mbar_wait(&s.v_full[st], v_par[st], w2);
     }
   }
   tc_fence_before();

@@ -71,6 +71,9 @@ struct __align__(1024) FwdSmem {
   int no_abort;
 };
 
+static_assert(sizeof(FwdSmem<128>) <= 232448, "forward shared memory exceeds the per-CTA limit");
+static_assert(sizeof(FwdSmem<64>) <= 232448, "forward shared memory exceeds the per-CTA limit");
+
 struct FwdItem {
   int b, h, hm, hkv, qb;
   const int* list;
@@ -114,41 +117,6 @@ __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, const
   for (int kk = 0; kk < kTile / 16; ++kk)
     mma_ts(d_tmem, p_tmem + kk * 8, sdesc_sw128(va + kk * 2048, 16384, 1024), idesc,
            (accumulate || kk > 0) ? 1u : 0u);
-}
-
-// Bits [lo, hi) of a 32-bit word (0 <= lo, hi <= 32).
-__device__ __forceinline__ uint32_t bit_range(int lo, int hi) {
-  const uint32_t up = hi >= 32 ? 0xffffffffu : ((1u << hi) - 1u);
-  const uint32_t dn = lo >= 32 ? 0xffffffffu : ((1u << lo) - 1u);
-  return hi > lo ? (up & ~dn) : 0u;
-}
-
-// Rows [r0, r0+32) hidden by one key column's intervals, as a 32-bit word.
-__device__ __forceinline__ uint32_t column_row_bits(const int4 r, int r0) {
-  const int a0 = min(max(r.x - r0, 0), 32), a1 = min(max(r.y - r0, 0), 32);
-  const int b0 = min(max(r.z - r0, 0), 32), b1 = min(max(r.w - r0, 0), 32);
-  return bit_range(a0, a1) | bit_range(b0, b1);
-}
-
-// 32x32 bit-matrix transpose across a warp: lane l holds word l on entry
-// (bit r = element (l, r)); on exit lane r holds bit l = element (l, r).
-template <int J, uint32_t M>
-__device__ __forceinline__ uint32_t transpose_step(uint32_t a, int lane) {
-  const uint32_t b = __shfl_xor_sync(0xffffffffu, a, J);
-  return (lane & J) ? ((a & ~M) | ((b & ~M) >> J)) : ((a & M) | ((b & M) << J));
-}
-__device__ __forceinline__ uint32_t warp_transpose32(uint32_t a, int lane) {
-  a = transpose_step<16, 0x0000FFFFu>(a, lane);
-  a = transpose_step<8, 0x00FF00FFu>(a, lane);
-  a = transpose_step<4, 0x0F0F0F0Fu>(a, lane);
-  a = transpose_step<2, 0x33333333u>(a, lane);
-  return transpose_step<1, 0x55555555u>(a, lane);
-}
-
-__device__ __forceinline__ float max3f(float a, float b, float c) {
-  float m;
-  asm("max.f32 %0, %1, %2, %3;" : "=f"(m) : "f"(a), "f"(b), "f"(c));
-  return m;
 }
 
 template <int D>
