@@ -12,6 +12,8 @@
 // over every q-head of the GQA group and every non-skipped 128-row q-tile.
 // TMEM (512 columns at d = 128):
 //   S^T [0,128) (P^T bf16 written over it)   dP^T [128,256) (dS^T bf16 over it)
+// (bf16 pairs of query columns 0-63 at the region's [0,32), of 64-127 at
+// [64,96): each compute warpgroup overwrites only TMEM columns it has read)
 //   dV [256, 256+d)                          dK [256+d, 256+2d)
 // The MMA warp issues, per q-tile t:
 //   ... dV(t) = P^T(t) dO(t) ; S^T(t+1) = K Q(t+1)^T ; dK(t) = dS^T(t) Q(t) ;
@@ -25,9 +27,12 @@
 // the compute warps turn dP^T(t) into dS^T(t); while it runs dK(t)+dP^T(t+1)
 // they turn S^T(t+1) into P^T(t+1).
 //
-// Roles (320 threads): warps 0-7 compute (two warpgroups; thread = key lane,
+// Roles (352 threads): warps 0-7 compute (two warpgroups; thread = key lane,
 // warpgroup 0 takes query columns 0-63 of the tile, warpgroup 1 columns
-// 64-127), warp 8 TMA producer, warp 9 MMA issuer.  Work items reach every
+// 64-127), warp 8 TMA producer of K and Q, warp 10 TMA producer of V, dO and
+// the LSE2 / D rows, warp 9 MMA issuer.  K is released after the item's last
+// S^T and V after its last dP^T, so the next item's K/V load overlaps the
+// current item's last q-tile.  Work items reach every
 // role through a ring of mbarriers (no CTA-wide barrier between items).
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -41,8 +46,8 @@
 namespace fm {
 
 namespace kvb {
-constexpr int kThreads = 320;
-constexpr int kProducerWarp = 8, kMmaWarp = 9;
+constexpr int kThreads = 352;
+constexpr int kProducerWarp = 8, kMmaWarp = 9, kProducer2Warp = 10;
 constexpr int kRing = 4;
 constexpr int kQStages = 3;   // Q tiles: last read by dK(t)
 constexpr int kDoStages = 2;  // dO tiles: last read by dV(t), freed earlier
@@ -60,12 +65,11 @@ struct __align__(1024) DkdvSmem {
   float dsum[kvb::kLStages][kTile];
   int ring_item[kvb::kRing];
   uint64_t ring_full[kvb::kRing], ring_empty[kvb::kRing];
-  uint64_t kv_full, kv_empty;
+  uint64_t k_full, k_empty, v_full, v_empty;
   uint64_t q_full[kvb::kQStages], q_empty[kvb::kQStages];
   uint64_t do_full[kvb::kDoStages], do_empty[kvb::kDoStages];
   uint64_t l_full[kvb::kLStages], l_empty[kvb::kLStages];
   uint64_t s_full, dp_full, p_full, ds_full;
-  uint64_t s_read, dp_read;  // both compute warpgroups have loaded S^T / dP^T (bf16 results overlap them)
   uint64_t dkdv_full, dkdv_free;
   uint64_t teardown;
   uint32_t tmem_base;
@@ -127,15 +131,17 @@ __device__ __forceinline__ void kv_issue_ss(uint32_t d_tmem, const uint8_t* as, 
   }
 }
 
-// D[tmem] (+)= A[tmem] B, B = [128 rows (K) x D] tile read MN-major.
+// D[tmem] (+)= A[tmem] B, B = [128 rows (K) x D] tile read MN-major.  A (bf16
+// pairs) holds K-columns 0-63 at a_tmem + [0,32) and 64-127 at a_tmem + [64,96):
+// each compute warpgroup writes its half inside the TMEM columns it read.
 template <int D>
 __device__ __forceinline__ void kv_issue_ts(uint32_t d_tmem, uint32_t a_tmem, const uint8_t* bs, bool accumulate) {
   constexpr uint32_t idesc = idesc_bf16(128, D, false, true);
   const uint32_t ba = smem_addr(bs);
 #pragma unroll
   for (int kk = 0; kk < kTile / 16; ++kk)
-    mma_ts(d_tmem, a_tmem + kk * 8, sdesc_sw128(ba + kk * 2048, 16384, 1024), idesc,
-           (accumulate || kk > 0) ? 1u : 0u);
+    mma_ts(d_tmem, a_tmem + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8), sdesc_sw128(ba + kk * 2048, 16384, 1024),
+           idesc, (accumulate || kk > 0) ? 1u : 0u);
 }
 
 template <int D>
@@ -163,10 +169,12 @@ __global__ void __launch_bounds__(kvb::kThreads, 1)
   if (tid == 0) {
     for (int i = 0; i < kRing; ++i) {
       mbar_init(&s.ring_full[i], 1);
-      mbar_init(&s.ring_empty[i], 9);  // MMA lane 0 + lane 0 of the 8 compute warps
+      mbar_init(&s.ring_empty[i], 10);  // MMA + second producer + lane 0 of the 8 compute warps
     }
-    mbar_init(&s.kv_full, 1);
-    mbar_init(&s.kv_empty, 1);
+    mbar_init(&s.k_full, 1);
+    mbar_init(&s.k_empty, 1);
+    mbar_init(&s.v_full, 1);
+    mbar_init(&s.v_empty, 1);
     for (int i = 0; i < kQStages; ++i) {
       mbar_init(&s.q_full[i], 1);
       mbar_init(&s.q_empty[i], 1);
@@ -183,8 +191,6 @@ __global__ void __launch_bounds__(kvb::kThreads, 1)
     mbar_init(&s.dp_full, 1);
     mbar_init(&s.p_full, 256);
     mbar_init(&s.ds_full, 256);
-    mbar_init(&s.s_read, 256);
-    mbar_init(&s.dp_read, 256);
     mbar_init(&s.dkdv_full, 1);
     mbar_init(&s.dkdv_free, 256);
     mbar_init(&s.teardown, 1);
@@ -203,10 +209,12 @@ __global__ void __launch_bounds__(kvb::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
   const WaitCtx w{&s.abort_flag, p.status, p.wait_limit_ns};
-  uint32_t kv_par = 0, kv_armed = 0, q_par[kQStages] = {}, do_par[kDoStages] = {}, l_par[kLStages] = {};
+  uint32_t kv_par = 0, kv_armed = 0, vv_par = 0, vv_armed = 0;
+  uint32_t q_par[kQStages] = {}, do_par[kDoStages] = {}, l_par[kLStages] = {};
   uint32_t q_armed = 0, do_armed = 0, l_armed = 0;
 
   if (warp == kProducerWarp) {
+    // first producer: the item's K tile and every q-tile's Q
     if (lane == 0) {
       uint32_t sq = 0, act = 0;
       bool ok = true;
@@ -219,19 +227,17 @@ __global__ void __launch_bounds__(kvb::kThreads, 1)
         if (item >= p.n_items) break;
         const KvItem it = decode_kv_item(p, item);
         if (it.total == 0) continue;
-        if (!(ok = mbar_wait(&s.kv_empty, (act & 1) ^ 1, w))) break;
-        mbar_arrive_expect_tx(&s.kv_full, 2 * kTileBytes);
+        if (!(ok = mbar_wait(&s.k_empty, (act & 1) ^ 1, w))) break;  // last S^T of the previous item done
+        mbar_arrive_expect_tx(&s.k_full, kTileBytes);
         kv_par = act & 1;
         kv_armed = 1;
 #pragma unroll
-        for (int bx = 0; bx < kBoxes; ++bx) {
-          tma_load_4d(s.k + bx * 16384, &tk, &s.kv_full, bx * 64, it.hkv, it.kt * kTile, it.b);
-          tma_load_4d(s.v + bx * 16384, &tv, &s.kv_full, bx * 64, it.hkv, it.kt * kTile, it.b);
-        }
+        for (int bx = 0; bx < kBoxes; ++bx)
+          tma_load_4d(s.k + bx * 16384, &tk, &s.k_full, bx * 64, it.hkv, it.kt * kTile, it.b);
         ++act;
         ok = for_each_qtile(p, it, [&](int, int h, int, int qt, int) {
-          const int sqi = sq % kQStages, sdo = sq % kDoStages, sl = sq % kLStages;
-          const uint32_t pq = (sq / kQStages) & 1, pd = (sq / kDoStages) & 1, pl = (sq / kLStages) & 1;
+          const int sqi = sq % kQStages;
+          const uint32_t pq = (sq / kQStages) & 1;
           if (!mbar_wait(&s.q_empty[sqi], pq ^ 1, w)) return false;
           mbar_arrive_expect_tx(&s.q_full[sqi], kTileBytes);
 #pragma unroll
@@ -239,6 +245,35 @@ __global__ void __launch_bounds__(kvb::kThreads, 1)
             tma_load_4d(s.q[sqi] + bx * 16384, &tq, &s.q_full[sqi], bx * 64, h, qt * kTile, it.b);
           q_par[sqi] = pq;
           q_armed |= 1u << sqi;
+          ++sq;
+          return true;
+        });
+      }
+    }
+  } else if (warp == kProducer2Warp) {
+    // second producer: the item's V tile, every q-tile's dO and LSE2 / D rows
+    if (lane == 0) {
+      uint32_t sq = 0, act = 0;
+      bool ok = true;
+      for (uint32_t k = 0; ok; ++k) {
+        const int slot = k % kRing;
+        if (!(ok = mbar_wait(&s.ring_full[slot], (k / kRing) & 1, w))) break;
+        const int item = s.ring_item[slot];
+        mbar_arrive(&s.ring_empty[slot]);
+        if (item >= p.n_items) break;
+        const KvItem it = decode_kv_item(p, item);
+        if (it.total == 0) continue;
+        if (!(ok = mbar_wait(&s.v_empty, (act & 1) ^ 1, w))) break;  // last dP^T of the previous item done
+        mbar_arrive_expect_tx(&s.v_full, kTileBytes);
+        vv_par = act & 1;
+        vv_armed = 1;
+#pragma unroll
+        for (int bx = 0; bx < kBoxes; ++bx)
+          tma_load_4d(s.v + bx * 16384, &tv, &s.v_full, bx * 64, it.hkv, it.kt * kTile, it.b);
+        ++act;
+        ok = for_each_qtile(p, it, [&](int, int h, int, int qt, int) {
+          const int sdo = sq % kDoStages, sl = sq % kLStages;
+          const uint32_t pd = (sq / kDoStages) & 1, pl = (sq / kLStages) & 1;
           if (!mbar_wait(&s.do_empty[sdo], pd ^ 1, w)) return false;
           mbar_arrive_expect_tx(&s.do_full[sdo], kTileBytes);
 #pragma unroll
@@ -271,18 +306,19 @@ __global__ void __launch_bounds__(kvb::kThreads, 1)
         const KvItem it = decode_kv_item(p, item);
         const int n = it.total;
         if (n == 0) continue;
-        if (!(ok = mbar_wait(&s.kv_full, act & 1, w))) break;
         // first q-tile: S^T and dP^T
         {
           const int sqi = sq % kQStages, sdo = sq % kDoStages;
-          if (!(ok = mbar_wait(&s.q_full[sqi], (sq / kQStages) & 1, w))) break;
+          if (!(ok = mbar_wait(&s.k_full, act & 1, w) && mbar_wait(&s.q_full[sqi], (sq / kQStages) & 1, w))) break;
           tc_fence_after();
           kv_issue_ss<D>(tmem + kColS, s.k, s.q[sqi]);
           mma_commit(&s.s_full);
-          if (!(ok = mbar_wait(&s.do_full[sdo], (sq / kDoStages) & 1, w))) break;
+          if (n == 1) mma_commit(&s.k_empty);  // K read for the last time
+          if (!(ok = mbar_wait(&s.v_full, act & 1, w) && mbar_wait(&s.do_full[sdo], (sq / kDoStages) & 1, w))) break;
           tc_fence_after();
           kv_issue_ss<D>(tmem + kColDP, s.v, s.dout[sdo]);
           mma_commit(&s.dp_full);
+          if (n == 1) mma_commit(&s.v_empty);  // V read for the last time
         }
         for (int j = 0; j < n; ++j) {
           const uint32_t sj = sq + j, tj = tc + j;
@@ -299,6 +335,7 @@ __global__ void __launch_bounds__(kvb::kThreads, 1)
             tc_fence_after();
             kv_issue_ss<D>(tmem + kColS, s.k, s.q[sqi2]);  // S^T(j+1), after dV(j) read P^T(j)
             mma_commit(&s.s_full);
+            if (j + 2 == n) mma_commit(&s.k_empty);  // K read for the last time
           }
           if (!(ok = mbar_wait(&s.ds_full, par, w))) break;
           tc_fence_after();
@@ -309,6 +346,7 @@ __global__ void __launch_bounds__(kvb::kThreads, 1)
             tc_fence_after();
             kv_issue_ss<D>(tmem + kColDP, s.v, s.dout[sdo2]);  // dP^T(j+1), after dK(j) read dS^T(j)
             mma_commit(&s.dp_full);
+            if (j + 2 == n) mma_commit(&s.v_empty);  // V read for the last time
           }
         }
         if (!ok) break;
@@ -316,7 +354,6 @@ __global__ void __launch_bounds__(kvb::kThreads, 1)
         tc += n;
         ++act;
         mma_commit(&s.dkdv_full);
-        mma_commit(&s.kv_empty);
       }
     }
   } else {
@@ -358,13 +395,9 @@ __global__ void __launch_bounds__(kvb::kThreads, 1)
           tmem_ld32x(tb + kColS + c0, pr);
           tmem_ld32x(tb + kColS + c0 + 32, pr + 32);
           tmem_ld_wait();
-          // P^T of query columns 64-127 is written into TMEM columns 32-63, which
-          // hold S^T of columns 32-63: write only after both warpgroups loaded S^T.
-          tc_fence_before();
-          mbar_arrive(&s.s_read);
 #pragma unroll
           for (int i = 0; i < 64; ++i) {
-            float pv = fast_exp2(__uint_as_float(pr[i]) * p.scale_log2 - l2[i]);
+            float pv = fast_exp2(fmaf(__uint_as_float(pr[i]), p.scale_log2, -l2[i]));
             if (need) {
               const int row = row0 + i;
               const bool masked = (rec.x <= row && row < rec.y) || (rec.z <= row && row < rec.w);
@@ -372,14 +405,12 @@ __global__ void __launch_bounds__(kvb::kThreads, 1)
             }
             pr[i] = __float_as_uint(pv);
           }
-          if (!__all_sync(0xffffffffu, mbar_wait(&s.s_read, par, w))) return false;
-          tc_fence_after();
           {
             uint32_t pk[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i)
               pk[i] = pack_bf16x2(__uint_as_float(pr[2 * i]), __uint_as_float(pr[2 * i + 1]));
-            tmem_st32x(tb + kColS + c0 / 2, pk);  // bf16 pairs: columns [c0/2, c0/2 + 32)
+            tmem_st32x(tb + kColS + c0, pk);  // bf16 pairs over this warpgroup's own S^T columns
           }
           tmem_st_wait();
           tc_fence_before();
@@ -392,22 +423,16 @@ __global__ void __launch_bounds__(kvb::kThreads, 1)
             tmem_ld32x(tb + kColDP + c0, r);
             tmem_ld32x(tb + kColDP + c0 + 32, r + 32);
             tmem_ld_wait();
-            // dS^T of columns 64-127 lands in TMEM columns 160-191 = dP^T of columns
-            // 32-63: write only after both warpgroups loaded dP^T.
-            tc_fence_before();
-            mbar_arrive(&s.dp_read);
 #pragma unroll
             for (int i = 0; i < 64; ++i)
               pr[i] = __float_as_uint(__uint_as_float(pr[i]) * (__uint_as_float(r[i]) - dsm[i]));
           }
-          if (!__all_sync(0xffffffffu, mbar_wait(&s.dp_read, par, w))) return false;
-          tc_fence_after();
           {
             uint32_t pk[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i)
               pk[i] = pack_bf16x2(__uint_as_float(pr[2 * i]), __uint_as_float(pr[2 * i + 1]));
-            tmem_st32x(tb + kColDP + c0 / 2, pk);
+            tmem_st32x(tb + kColDP + c0, pk);  // bf16 pairs over this warpgroup's own dP^T columns
           }
           tmem_st_wait();
           tc_fence_before();
@@ -463,9 +488,12 @@ __global__ void __launch_bounds__(kvb::kThreads, 1)
       (void)mbar_wait(&s.teardown, 0, w2);
     }
     if (warp == kProducerWarp && lane == 0) {
-      if (kv_armed) (void)mbar_wait(&s.kv_full, kv_par, w2);
+      if (kv_armed) (void)mbar_wait(&s.k_full, kv_par, w2);
       for (int st = 0; st < kQStages; ++st)
         if (q_armed & (1u << st)) (void)mbar_wait(&s.q_full[st], q_par[st], w2);
+    }
+    if (warp == kProducer2Warp && lane == 0) {
+      if (vv_armed) (void)mbar_wait(&s.v_full, vv_par, w2);
       for (int st = 0; st < kDoStages; ++st)
         if (do_armed & (1u << st)) (void)mbar_wait(&s.do_full[st], do_par[st], w2);
       for (int st = 0; st < kLStages; ++st)

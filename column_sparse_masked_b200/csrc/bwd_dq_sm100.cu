@@ -14,7 +14,9 @@
 // key-stationary kernel.)
 //
 // TMEM (512 columns): S[0] [0,128), S[1] [128,256) (dS bf16 written over the
-// S buffer of its tile), dP [256,384), dQ [384, 384+d).
+// S buffer of its tile: key columns 0-63 as pairs at [0,32), 64-127 at
+// [64,96), so each warpgroup overwrites only columns it has read), dP
+// [256,384), dQ [384, 384+d).
 // MMA issue order: S(0) dP(0) | S(t+1) , dQ += dS(t) K(t) , dP(t+1) | ...
 // K tiles (3-deep ring, freed after dQ) and V tiles (2-deep, freed after dP)
 // stream through separate rings; the element mask of a partial tile is built
@@ -23,10 +25,12 @@
 // While the tensor core runs S(t+1) and dQ(t) the compute warps turn
 // S(t+1)/dP(t+1) into dS(t+1).
 //
-// Roles (320 threads): warps 0-7 compute (thread = query row; warpgroup 0
+// Roles (352 threads): warps 0-7 compute (thread = query row; warpgroup 0
 // takes key columns 0-63 of a tile, warpgroup 1 columns 64-127), warp 8 TMA
-// producer, warp 9 MMA issuer; work items reach every role through a ring of
-// mbarriers.
+// producer of Q/dO and the K ring, warp 10 TMA producer of the V ring, warp 9
+// MMA issuer; work items reach every role through a ring of mbarriers.  Q and
+// dO are released after the item's last S and dP (one tile before its end), so
+// the next item's Q/dO load overlaps the current item's last dQ step.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <climits>
@@ -39,8 +43,8 @@
 namespace fm {
 
 namespace qb {
-constexpr int kThreads = 320;
-constexpr int kProducerWarp = 8, kMmaWarp = 9;
+constexpr int kThreads = 352;
+constexpr int kProducerWarp = 8, kMmaWarp = 9, kProducer2Warp = 10;
 constexpr int kRing = 4;
 constexpr int kKStages = 3;  // K tiles: last read by dQ(t)
 constexpr int kVStages = 2;  // V tiles: last read by dP(t), freed earlier
@@ -58,7 +62,7 @@ struct __align__(1024) DqSmem {
   uint64_t q_full, q_empty;
   uint64_t k_full[qb::kKStages], k_empty[qb::kKStages];
   uint64_t v_full[qb::kVStages], v_empty[qb::kVStages];
-  uint64_t s_full[2], dp_full, sd_read, ds_full;
+  uint64_t s_full[2], dp_full, ds_full;
   uint64_t dq_full, dq_free;
   uint64_t teardown;
   uint32_t tmem_base;
@@ -124,9 +128,9 @@ __device__ __forceinline__ void q_issue_dq(uint32_t d_tmem, uint32_t a_tmem, con
   constexpr uint32_t idesc = idesc_bf16(128, D, false, true);
   const uint32_t ka = smem_addr(ks);
 #pragma unroll
-  for (int kk = 0; kk < kTile / 16; ++kk)
-    mma_ts(d_tmem, a_tmem + kk * 8, sdesc_sw128(ka + kk * 2048, 16384, 1024), idesc,
-           (accumulate || kk > 0) ? 1u : 0u);
+  for (int kk = 0; kk < kTile / 16; ++kk)  // dS pairs: keys 0-63 at [0,32), 64-127 at [64,96)
+    mma_ts(d_tmem, a_tmem + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8), sdesc_sw128(ka + kk * 2048, 16384, 1024),
+           idesc, (accumulate || kk > 0) ? 1u : 0u);
 }
 
 template <int D>
@@ -153,7 +157,7 @@ __global__ void __launch_bounds__(qb::kThreads, 1)
   if (tid == 0) {
     for (int i = 0; i < kRing; ++i) {
       mbar_init(&s.ring_full[i], 1);
-      mbar_init(&s.ring_empty[i], 9);
+      mbar_init(&s.ring_empty[i], 10);  // MMA + second producer + lane 0 of the 8 compute warps
     }
     mbar_init(&s.q_full, 1);
     mbar_init(&s.q_empty, 1);
@@ -168,7 +172,6 @@ __global__ void __launch_bounds__(qb::kThreads, 1)
     mbar_init(&s.s_full[0], 1);
     mbar_init(&s.s_full[1], 1);
     mbar_init(&s.dp_full, 1);
-    mbar_init(&s.sd_read, 256);
     mbar_init(&s.ds_full, 256);
     mbar_init(&s.dq_full, 1);
     mbar_init(&s.dq_free, 256);
@@ -214,8 +217,8 @@ __global__ void __launch_bounds__(qb::kThreads, 1)
         }
         ++act;
         ok = for_each_ktile(it, [&](int kt, int) {
-          const int sk = kv_iter % kKStages, sv = kv_iter % kVStages;
-          const uint32_t pk = (kv_iter / kKStages) & 1, pv = (kv_iter / kVStages) & 1;
+          const int sk = kv_iter % kKStages;
+          const uint32_t pk = (kv_iter / kKStages) & 1;
           const int hkv = it.h / sh.G;
           if (!mbar_wait(&s.k_empty[sk], pk ^ 1, w)) return false;
           mbar_arrive_expect_tx(&s.k_full[sk], kTileBytes);
@@ -224,11 +227,32 @@ __global__ void __launch_bounds__(qb::kThreads, 1)
             tma_load_4d(s.k[sk] + bx * 16384, &tk, &s.k_full[sk], bx * 64, hkv, kt * kTile, it.b);
           k_par[sk] = pk;
           k_armed |= 1u << sk;
+          ++kv_iter;
+          return true;
+        });
+      }
+    }
+  } else if (warp == kProducer2Warp) {
+    // second producer: the V ring
+    if (lane == 0) {
+      uint32_t kv_iter = 0;
+      bool ok = true;
+      for (uint32_t k = 0; ok; ++k) {
+        const int slot = k % kRing;
+        if (!(ok = mbar_wait(&s.ring_full[slot], (k / kRing) & 1, w))) break;
+        const int item = s.ring_item[slot];
+        mbar_arrive(&s.ring_empty[slot]);
+        if (item >= p.n_items2) break;
+        const QItem it = decode_q_item(p, item);
+        if (it.n == 0) continue;
+        ok = for_each_ktile(it, [&](int kt, int) {
+          const int sv = kv_iter % kVStages;
+          const uint32_t pv = (kv_iter / kVStages) & 1;
           if (!mbar_wait(&s.v_empty[sv], pv ^ 1, w)) return false;
           mbar_arrive_expect_tx(&s.v_full[sv], kTileBytes);
 #pragma unroll
           for (int bx = 0; bx < kBoxes; ++bx)
-            tma_load_4d(s.v[sv] + bx * 16384, &tv, &s.v_full[sv], bx * 64, hkv, kt * kTile, it.b);
+            tma_load_4d(s.v[sv] + bx * 16384, &tv, &s.v_full[sv], bx * 64, it.h / sh.G, kt * kTile, it.b);
           v_par[sv] = pv;
           v_armed |= 1u << sv;
           ++kv_iter;
@@ -263,6 +287,7 @@ __global__ void __launch_bounds__(qb::kThreads, 1)
           q_issue_ss<D>(tmem + kColDP, s.dout, s.v[sv]);
           mma_commit(&s.dp_full);
           mma_commit(&s.v_empty[sv]);
+          if (n == 1) mma_commit(&s.q_empty);  // Q and dO read for the last time
         }
         for (int j = 0; j < n; ++j) {
           const uint32_t kj = kv_iter + j, tj = tc + j;
@@ -285,6 +310,7 @@ __global__ void __launch_bounds__(qb::kThreads, 1)
             q_issue_ss<D>(tmem + kColDP, s.dout, s.v[sv2]);  // dP(j+1): dP(j) was read before ds_full(j)
             mma_commit(&s.dp_full);
             mma_commit(&s.v_empty[sv2]);
+            if (j + 2 == n) mma_commit(&s.q_empty);  // last S and dP of the item issued
           }
         }
         if (!ok) break;
@@ -292,7 +318,6 @@ __global__ void __launch_bounds__(qb::kThreads, 1)
         tc += n;
         ++act;
         mma_commit(&s.dq_full);
-        mma_commit(&s.q_empty);
       }
     }
   } else {
@@ -351,13 +376,9 @@ __global__ void __launch_bounds__(qb::kThreads, 1)
           mbits1 = warp_transpose32(column_row_bits(rb, rbase), lane);
         }
         tmem_ld_wait();
-        // dS of key columns 64-127 is written into TMEM columns 32-63 of the S
-        // buffer (S of columns 32-63): both warpgroups must have loaded first.
-        tc_fence_before();
-        mbar_arrive(&s.sd_read);
 #pragma unroll
         for (int i = 0; i < 64; ++i) {
-          float pv = fast_exp2(__uint_as_float(sv[i]) * p.scale_log2 - lse2);
+          float pv = fast_exp2(fmaf(__uint_as_float(sv[i]), p.scale_log2, -lse2));
           const uint32_t bits = (i < 32) ? mbits0 : mbits1;
           pv = ((bits >> (i & 31)) & 1u) ? 0.f : pv;
           sv[i] = __float_as_uint(pv * (__uint_as_float(dv[i]) - drow));
@@ -365,9 +386,7 @@ __global__ void __launch_bounds__(qb::kThreads, 1)
         uint32_t pk[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) pk[i] = pack_bf16x2(__uint_as_float(sv[2 * i]), __uint_as_float(sv[2 * i + 1]));
-        if (!__all_sync(0xffffffffu, mbar_wait(&s.sd_read, tc & 1, w))) return false;
-        tc_fence_after();
-        tmem_st32x(tb + kColS + bf * 128 + c0 / 2, pk);
+        tmem_st32x(tb + kColS + bf * 128 + c0, pk);  // bf16 pairs over this warpgroup's own S columns
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&s.ds_full);
@@ -411,6 +430,8 @@ __global__ void __launch_bounds__(qb::kThreads, 1)
       if (q_armed) (void)mbar_wait(&s.q_full, q_par, w2);
       for (int st = 0; st < kKStages; ++st)
         if (k_armed & (1u << st)) (void)mbar_wait(&s.k_full[st], k_par[st], w2);
+    }
+    if (warp == kProducer2Warp && lane == 0) {
       for (int st = 0; st < kVStages; ++st)
         if (v_armed & (1u << st)) (void)mbar_wait(&s.v_full[st], v_par[st], w2);
     }
