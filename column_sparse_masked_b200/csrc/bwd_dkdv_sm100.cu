@@ -389,7 +389,14 @@ __global__ void __launch_bounds__(kvb::kThreads, 1)
           const float* l2 = s.lse2[sl] + c0;
           const float* dsm = s.dsum[sl] + c0;
           const bool need = cls == kClsPartial;
-          const int row0 = qt * kTile + c0;
+          // this key's masked rows among the warpgroup's 64 query rows, as two
+          // 32-bit words (interval arithmetic on the column's boundaries)
+          uint32_t mw0 = 0u, mw1 = 0u;
+          if (need) {
+            const int row0 = qt * kTile + c0;
+            mw0 = column_row_bits(rec, row0);
+            mw1 = column_row_bits(rec, row0 + 32);
+          }
           // P^T for 64 query columns, in place over the loaded S^T values
           uint32_t pr[64];
           tmem_ld32x(tb + kColS + c0, pr);
@@ -397,13 +404,9 @@ __global__ void __launch_bounds__(kvb::kThreads, 1)
           tmem_ld_wait();
 #pragma unroll
           for (int i = 0; i < 64; ++i) {
-            float pv = fast_exp2(fmaf(__uint_as_float(pr[i]), p.scale_log2, -l2[i]));
-            if (need) {
-              const int row = row0 + i;
-              const bool masked = (rec.x <= row && row < rec.y) || (rec.z <= row && row < rec.w);
-              pv = masked ? 0.f : pv;
-            }
-            pr[i] = __float_as_uint(pv);
+            const float pv = fast_exp2(fmaf(__uint_as_float(pr[i]), p.scale_log2, -l2[i]));
+            const uint32_t bit = ((i < 32 ? mw0 : mw1) >> (i & 31)) & 1u;
+            pr[i] = bit ? 0u : __float_as_uint(pv);
           }
           {
             uint32_t pk[32];

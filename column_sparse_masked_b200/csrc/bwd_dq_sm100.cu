@@ -17,13 +17,16 @@
 // S buffer of its tile: key columns 0-63 as pairs at [0,32), 64-127 at
 // [64,96), so each warpgroup overwrites only columns it has read), dP
 // [256,384), dQ [384, 384+d).
-// MMA issue order: S(0) dP(0) | S(t+1) , dQ += dS(t) K(t) , dP(t+1) | ...
+// MMA issue order: S(0) dP(0) | S(t+1) , dP(t+1) , dQ += dS(t) K(t) | ...
+// where dP(t+1) waits only until the compute warps have loaded dP(t) into
+// registers (dS(t) is written over S(t), not over dP), so the next tile's dP
+// is computed while the compute warps evaluate the current tile.
 // K tiles (3-deep ring, freed after dQ) and V tiles (2-deep, freed after dP)
 // stream through separate rings; the element mask of a partial tile is built
 // from the boundary records read straight from global memory (L2-resident),
 // turned into per-row bit words by a warp bit-transpose.
-// While the tensor core runs S(t+1) and dQ(t) the compute warps turn
-// S(t+1)/dP(t+1) into dS(t+1).
+// While the tensor core runs S(t+1), dP(t+1) and dQ(t) the compute warps turn
+// S(t)/dP(t) into dS(t).
 //
 // Roles (352 threads): warps 0-7 compute (thread = query row; warpgroup 0
 // takes key columns 0-63 of a tile, warpgroup 1 columns 64-127), warp 8 TMA
@@ -62,7 +65,7 @@ struct __align__(1024) DqSmem {
   uint64_t q_full, q_empty;
   uint64_t k_full[qb::kKStages], k_empty[qb::kKStages];
   uint64_t v_full[qb::kVStages], v_empty[qb::kVStages];
-  uint64_t s_full[2], dp_full, ds_full;
+  uint64_t s_full[2], dp_full, dp_read, ds_full;
   uint64_t dq_full, dq_free;
   uint64_t teardown;
   uint32_t tmem_base;
@@ -172,6 +175,7 @@ __global__ void __launch_bounds__(qb::kThreads, 1)
     mbar_init(&s.s_full[0], 1);
     mbar_init(&s.s_full[1], 1);
     mbar_init(&s.dp_full, 1);
+    mbar_init(&s.dp_read, 256);
     mbar_init(&s.ds_full, 256);
     mbar_init(&s.dq_full, 1);
     mbar_init(&s.dq_free, 256);
@@ -299,19 +303,21 @@ __global__ void __launch_bounds__(qb::kThreads, 1)
             q_issue_ss<D>(tmem + kColS + (bf ^ 1) * 128, s.q, s.k[sk2]);  // S(j+1): its buffer held dS(j-1)
             mma_commit(&s.s_full[bf ^ 1]);
           }
+          if (j + 1 < n) {
+            // dP(j+1) as soon as the compute warps hold dP(j) in registers
+            if (!(ok = mbar_wait(&s.dp_read, tj & 1, w) && mbar_wait(&s.v_full[sv2], ((kj + 1) / kVStages) & 1, w)))
+              break;
+            tc_fence_after();
+            q_issue_ss<D>(tmem + kColDP, s.dout, s.v[sv2]);
+            mma_commit(&s.dp_full);
+            mma_commit(&s.v_empty[sv2]);
+            if (j + 2 == n) mma_commit(&s.q_empty);  // last S and dP of the item issued
+          }
           if (j == 0 && !(ok = mbar_wait(&s.dq_free, (act & 1) ^ 1, w))) break;  // previous dQ read out
           if (!(ok = mbar_wait(&s.ds_full, tj & 1, w))) break;
           tc_fence_after();
           q_issue_dq<D>(tmem + kColDQ, tmem + kColS + bf * 128, s.k[sk], j > 0);  // dQ += dS K
           mma_commit(&s.k_empty[sk]);
-          if (j + 1 < n) {
-            if (!(ok = mbar_wait(&s.v_full[sv2], ((kj + 1) / kVStages) & 1, w))) break;
-            tc_fence_after();
-            q_issue_ss<D>(tmem + kColDP, s.dout, s.v[sv2]);  // dP(j+1): dP(j) was read before ds_full(j)
-            mma_commit(&s.dp_full);
-            mma_commit(&s.v_empty[sv2]);
-            if (j + 2 == n) mma_commit(&s.q_empty);  // last S and dP of the item issued
-          }
         }
         if (!ok) break;
         kv_iter += n;
@@ -376,6 +382,8 @@ __global__ void __launch_bounds__(qb::kThreads, 1)
           mbits1 = warp_transpose32(column_row_bits(rb, rbase), lane);
         }
         tmem_ld_wait();
+        tc_fence_before();
+        mbar_arrive(&s.dp_read);  // dP(j) is in registers: the tensor core may overwrite it
 #pragma unroll
         for (int i = 0; i < 64; ++i) {
           float pv = fast_exp2(fmaf(__uint_as_float(sv[i]), p.scale_log2, -lse2));

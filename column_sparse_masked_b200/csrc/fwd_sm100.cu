@@ -11,8 +11,10 @@
 //     an atomic counter; the producer warp hands each item to the other roles
 //     through a ring of mbarriers, so consecutive items overlap (the next
 //     item's Q load and first QK^T run while the softmax warps write O);
-//   * warp 8 issues TMA loads (Q once per item; K, V and, for tiles that need
-//     it, the 2 KiB boundary records through a multi-stage ring);
+//   * warp 8 issues TMA loads: Q once per item, and K(0), V(0), K(1), V(1), ...
+//     through one ring of tile-sized slots; a K slot is released after the
+//     second q-tile's QK^T, a V slot after its P V, so V tiles are requested
+//     about two key steps before they are used;
 //   * warp 9 issues tcgen05 MMAs: S_g = Q_g K^T into TMEM, O_g += P_g V with
 //     P_g read from TMEM (bf16, written over S_g), ping-pong between the two
 //     q-tiles: S0 S1 | PV0 S0' PV1 S1' | ...;
@@ -21,10 +23,11 @@
 //     into one FMA per element, O rescaled in TMEM
 //     only when a row maximum grows by more than 2^8.
 //
-// The element mask of a partial tile is built per key column: each lane turns
-// the boundaries of 4 columns into 32-bit words over its warp's 32 rows
-// (interval arithmetic), and a 5-step shuffle transpose of each 32x32 bit
-// block hands every row its mask bits.
+// The element mask of a partial tile is built per key column: each lane reads
+// the boundary records of 4 columns (L2-resident), turns them into 32-bit words
+// over its warp's 32 rows (interval arithmetic), and a 5-step shuffle transpose
+// of each 32x32 bit block hands every row its mask bits.  This runs before the
+// wait for S, off the softmax critical path.
 //
 // TMEM (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+d), O1 after O0.
 #include <cuda.h>
@@ -40,7 +43,7 @@ namespace fm {
 
 template <int D>
 struct FwdCfg {
-  static constexpr int kStages = (D == 128) ? 2 : 4;
+  static constexpr int kSlots = (D == 128) ? 5 : 10;  // K/V ring slots of one tile each
   static constexpr int kTileBytes = kTile * D * 2;  // one 128-row bf16 tile
   static constexpr int kBoxes = D / 64;             // 64-column (128-byte) TMA boxes per tile
   static constexpr int kThreads = 320;
@@ -49,18 +52,43 @@ struct FwdCfg {
   static constexpr int kRing = 4;
 };
 
+// A decoded work item.  The producer decodes each item once (three dependent
+// global reads) and publishes it in the shared-memory ring; the other roles
+// read it from there.  item = INT_MAX ends the work.
+struct __align__(16) FwdItem {
+  int item, b, h, hm, hkv, qb, n, e0;  // e0: first entry of the item's tile list
+  __device__ __forceinline__ const int* list(const FwdParams& p) const {
+    const Shape& sh = p.s;
+    return p.flist + (((size_t)b * sh.Hm + hm) * sh.nQB + qb) * sh.nKt;
+  }
+};
+
+__device__ __forceinline__ FwdItem decode_fwd(const FwdParams& p, int item) {
+  const Shape& sh = p.s;
+  FwdItem it{};
+  it.item = item;
+  if (item >= p.n_items) return it;
+  const ItemCoord c = decode_fwd_item(sh, p.order[item]);
+  it.b = c.b;
+  it.qb = c.t;
+  it.hkv = c.hkv;
+  it.h = c.hkv * sh.G + c.hg;
+  it.hm = (sh.Hm == 1) ? 0 : it.h;
+  const size_t lrow = ((size_t)it.b * sh.Hm + it.hm) * sh.nQB + it.qb;
+  it.n = p.fcount[lrow];
+  it.e0 = it.n > 0 ? p.flist[lrow * sh.nKt] : 0;
+  return it;
+}
+
 template <int D>
 struct __align__(1024) FwdSmem {
   uint8_t q[2][FwdCfg<D>::kTileBytes];
-  uint8_t k[FwdCfg<D>::kStages][FwdCfg<D>::kTileBytes];
-  uint8_t v[FwdCfg<D>::kStages][FwdCfg<D>::kTileBytes];
-  int4 mask[FwdCfg<D>::kStages][kTile];
-  int ring_item[FwdCfg<D>::kRing];
+  uint8_t slot[FwdCfg<D>::kSlots][FwdCfg<D>::kTileBytes];  // K(t) in ring position 2t, V(t) in 2t+1
+  FwdItem ring[FwdCfg<D>::kRing];
   uint64_t ring_full[FwdCfg<D>::kRing], ring_empty[FwdCfg<D>::kRing];
   uint64_t q_full, q_empty;
-  uint64_t k_full[FwdCfg<D>::kStages];
-  uint64_t v_full[FwdCfg<D>::kStages];
-  uint64_t kv_empty[FwdCfg<D>::kStages];
+  uint64_t slot_full[FwdCfg<D>::kSlots];
+  uint64_t slot_empty[FwdCfg<D>::kSlots];
   uint64_t s_full[2];
   uint64_t p_full[2];
   uint64_t o_full[2];
@@ -73,27 +101,6 @@ struct __align__(1024) FwdSmem {
 
 static_assert(sizeof(FwdSmem<128>) <= 232448, "forward shared memory exceeds the per-CTA limit");
 static_assert(sizeof(FwdSmem<64>) <= 232448, "forward shared memory exceeds the per-CTA limit");
-
-struct FwdItem {
-  int b, h, hm, hkv, qb;
-  const int* list;
-  int n;
-};
-
-__device__ __forceinline__ FwdItem decode_fwd(const FwdParams& p, int item) {
-  const Shape& sh = p.s;
-  const ItemCoord c = decode_fwd_item(sh, p.order[item]);
-  FwdItem it;
-  it.b = c.b;
-  it.qb = c.t;
-  it.hkv = c.hkv;
-  it.h = c.hkv * sh.G + c.hg;
-  it.hm = (sh.Hm == 1) ? 0 : it.h;
-  const size_t lrow = ((size_t)it.b * sh.Hm + it.hm) * sh.nQB + it.qb;
-  it.list = p.flist + lrow * sh.nKt;
-  it.n = p.fcount[lrow];
-  return it;
-}
 
 // S = Q K^T: M = 128 rows, N = 128 keys, K = D; both operands K-major SW128.
 template <int D>
@@ -124,7 +131,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
     fm_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                   const __grid_constant__ CUtensorMap tv, const FwdParams p) {
   using Cfg = FwdCfg<D>;
-  constexpr int kStages = Cfg::kStages;
+  constexpr int kSlots = Cfg::kSlots;
   constexpr int kRing = Cfg::kRing;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   FwdSmem<D>& s = *reinterpret_cast<FwdSmem<D>*>(smem_raw);
@@ -146,10 +153,9 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
     }
     mbar_init(&s.q_full, 1);
     mbar_init(&s.q_empty, 1);
-    for (int i = 0; i < kStages; ++i) {
-      mbar_init(&s.k_full[i], 1);
-      mbar_init(&s.v_full[i], 1);
-      mbar_init(&s.kv_empty[i], 1);
+    for (int i = 0; i < kSlots; ++i) {
+      mbar_init(&s.slot_full[i], 1);
+      mbar_init(&s.slot_empty[i], 1);
     }
     for (int g = 0; g < 2; ++g) {
       mbar_init(&s.s_full[g], 1);
@@ -172,21 +178,22 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
   const WaitCtx w{&s.abort_flag, p.status, p.wait_limit_ns};
-  uint32_t q_par = 0, q_armed = 0, k_par[kStages] = {}, k_armed = 0;
+  uint32_t q_par = 0, q_armed = 0, slot_par = 0, slot_armed = 0;  // producer: copies that may be in flight
 
   if (warp == Cfg::kProducerWarp) {
     if (lane == 0) {
-      uint32_t kv_iter = 0, act = 0;
+      uint32_t pos = 0, act = 0;  // ring position of the next K/V tile
       bool ok = true;
       for (uint32_t k = 0; ok; ++k) {
         const int slot = k % kRing;
         if (!(ok = mbar_wait(&s.ring_empty[slot], ((k / kRing) & 1) ^ 1, w))) break;
         const int item = s.abort_flag ? INT_MAX : atomicAdd(p.counter, 1);
-        s.ring_item[slot] = item;
+        const FwdItem it = decode_fwd(p, item);
+        s.ring[slot] = it;
         mbar_arrive(&s.ring_full[slot]);
         if (item >= p.n_items) break;
-        const FwdItem it = decode_fwd(p, item);
         if (it.n == 0) continue;
+        const int* list = it.list(p);
         if (!(ok = mbar_wait(&s.q_empty, (act & 1) ^ 1, w))) break;
         mbar_arrive_expect_tx(&s.q_full, 2 * Cfg::kTileBytes);
         q_par = act & 1;
@@ -197,81 +204,77 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
           for (int bx = 0; bx < Cfg::kBoxes; ++bx)
             tma_load_4d(s.q[g] + bx * 16384, &tq, &s.q_full, bx * 64, it.h, it.qb * 256 + g * kTile, it.b);
         ++act;
-        for (int t = 0; t < it.n; ++t, ++kv_iter) {
-          const int e = it.list[t];
-          const int kt = e >> 8;
-          const bool need = ((e & 3) != kClsFull) || (((e >> 2) & 3) != kClsFull) || ((e >> 4) & 1);
-          const int st = kv_iter % kStages;
-          const uint32_t ph = (kv_iter / kStages) & 1;
-          if (!(ok = mbar_wait(&s.kv_empty[st], ph ^ 1, w))) break;
-          mbar_arrive_expect_tx(&s.k_full[st], Cfg::kTileBytes + (need ? kTile * 16 : 0));
+        for (int t = 0; t < it.n && ok; ++t) {
+          const int kt = (t == 0 ? it.e0 : list[t]) >> 8;
 #pragma unroll
-          for (int bx = 0; bx < Cfg::kBoxes; ++bx)
-            tma_load_4d(s.k[st] + bx * 16384, &tk, &s.k_full[st], bx * 64, it.hkv, kt * kTile, it.b);
-          if (need)
-            bulk_load(s.mask[st], p.rec + (((size_t)it.b * sh.Hm + it.hm) * sh.nKt + kt) * kTile, kTile * 16,
-                      &s.k_full[st]);
-          mbar_arrive_expect_tx(&s.v_full[st], Cfg::kTileBytes);
+          for (int kv = 0; kv < 2; ++kv, ++pos) {  // K(t), then V(t)
+            const int sl = pos % kSlots;
+            const uint32_t ph = (pos / kSlots) & 1;
+            if (!(ok = mbar_wait(&s.slot_empty[sl], ph ^ 1, w))) break;
+            mbar_arrive_expect_tx(&s.slot_full[sl], Cfg::kTileBytes);
 #pragma unroll
-          for (int bx = 0; bx < Cfg::kBoxes; ++bx)
-            tma_load_4d(s.v[st] + bx * 16384, &tv, &s.v_full[st], bx * 64, it.hkv, kt * kTile, it.b);
-          k_par[st] = ph;
-          k_armed |= 1u << st;
+            for (int bx = 0; bx < Cfg::kBoxes; ++bx)
+              tma_load_4d(s.slot[sl] + bx * 16384, kv ? &tv : &tk, &s.slot_full[sl], bx * 64, it.hkv, kt * kTile, it.b);
+            slot_par = (slot_par & ~(1u << sl)) | (ph << sl);
+            slot_armed |= 1u << sl;
+          }
         }
       }
     }
   } else if (warp == Cfg::kMmaWarp) {
     if (lane == 0) {
-      uint32_t kv_iter = 0, tile_cnt = 0, act = 0;
+      uint32_t pos = 0, tile_cnt = 0, act = 0;
       bool ok = true;
       for (uint32_t k = 0; ok; ++k) {
         const int slot = k % kRing;
         if (!(ok = mbar_wait(&s.ring_full[slot], (k / kRing) & 1, w))) break;
-        const int item = s.ring_item[slot];
+        const FwdItem it = s.ring[slot];
         mbar_arrive(&s.ring_empty[slot]);
-        if (item >= p.n_items) break;
-        const FwdItem it = decode_fwd(p, item);
+        if (it.item >= p.n_items) break;
         const int n = it.n;
         if (n == 0) continue;
         if (!(ok = mbar_wait(&s.q_full, act & 1, w))) break;
         tc_fence_after();
-        for (int t = 0; t < n; ++t) {
-          const int st = kv_iter % kStages;
-          const uint32_t ph = (kv_iter / kStages) & 1;
-          const int st2 = (kv_iter + 1) % kStages;
-          const uint32_t ph2 = ((kv_iter + 1) / kStages) & 1;
+        for (int t = 0; t < n; ++t, pos += 2) {
+          // ring slots of K(t+1) and V(t)
+          const int sv = (pos + 1) % kSlots;
+          const uint32_t pv_ph = ((pos + 1) / kSlots) & 1;
+          const int sk2 = (pos + 2) % kSlots;
+          const uint32_t k2_ph = ((pos + 2) / kSlots) & 1;
           if (t == 0) {
-            if (!(ok = mbar_wait(&s.k_full[st], ph, w))) break;
+            const int sk = pos % kSlots;
+            if (!(ok = mbar_wait(&s.slot_full[sk], (pos / kSlots) & 1, w))) break;
             tc_fence_after();
-            issue_qk<D>(tmem + 0, s.q[0], s.k[st]);
+            issue_qk<D>(tmem + 0, s.q[0], s.slot[sk]);
             mma_commit(&s.s_full[0]);
-            issue_qk<D>(tmem + 128, s.q[1], s.k[st]);
+            issue_qk<D>(tmem + 128, s.q[1], s.slot[sk]);
             mma_commit(&s.s_full[1]);
+            mma_commit(&s.slot_empty[sk]);
             if (n == 1) mma_commit(&s.q_empty);
           }
-          if (!(ok = mbar_wait(&s.v_full[st], ph, w) && mbar_wait(&s.p_full[0], tile_cnt & 1, w))) break;
+          if (!(ok = mbar_wait(&s.slot_full[sv], pv_ph, w) && mbar_wait(&s.p_full[0], tile_cnt & 1, w))) break;
           if (t == 0 && !(ok = mbar_wait(&s.o_free[0], (act & 1) ^ 1, w))) break;  // previous O0 read out
           tc_fence_after();
-          issue_pv<D>(tmem + 256, tmem + 0, s.v[st], t > 0);
+          issue_pv<D>(tmem + 256, tmem + 0, s.slot[sv], t > 0);
           if (t == n - 1) mma_commit(&s.o_full[0]);
           if (t + 1 < n) {
-            if (!(ok = mbar_wait(&s.k_full[st2], ph2, w))) break;
+            if (!(ok = mbar_wait(&s.slot_full[sk2], k2_ph, w))) break;
             tc_fence_after();
-            issue_qk<D>(tmem + 0, s.q[0], s.k[st2]);
+            issue_qk<D>(tmem + 0, s.q[0], s.slot[sk2]);
             mma_commit(&s.s_full[0]);
           }
           if (!(ok = mbar_wait(&s.p_full[1], tile_cnt & 1, w))) break;
           if (t == 0 && !(ok = mbar_wait(&s.o_free[1], (act & 1) ^ 1, w))) break;
           tc_fence_after();
-          issue_pv<D>(tmem + 256 + D, tmem + 128, s.v[st], t > 0);
+          issue_pv<D>(tmem + 256 + D, tmem + 128, s.slot[sv], t > 0);
           if (t == n - 1) mma_commit(&s.o_full[1]);
-          mma_commit(&s.kv_empty[st]);
+          mma_commit(&s.slot_empty[sv]);
           if (t + 1 < n) {
-            issue_qk<D>(tmem + 128, s.q[1], s.k[st2]);
+            issue_qk<D>(tmem + 128, s.q[1], s.slot[sk2]);
             mma_commit(&s.s_full[1]);
+            mma_commit(&s.slot_empty[sk2]);
             if (t + 2 == n) mma_commit(&s.q_empty);  // last QK^T of the item issued
           }
-          ++kv_iter;
           ++tile_cnt;
         }
         if (!ok) break;
@@ -284,29 +287,42 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
     const uint32_t tb = tmem + ((uint32_t)(wq * 32) << 16);
     const uint32_t s_col = g * 128, o_col = 256 + g * D;
     const float sl2 = p.scale_log2;
-    uint32_t kv_iter = 0, tile_cnt = 0, act = 0;
+    // O rows go out as 32-byte stores when the output allows it (rows are
+    // Hq * D * 2 bytes apart, a multiple of 32).
+    const bool o_v8 = (reinterpret_cast<uintptr_t>(p.o) & 31u) == 0;
+    uint32_t tile_cnt = 0, act = 0, k = 0;
     bool ok = true;
-    for (uint32_t k = 0; ok; ++k) {
-      const int slot = k % kRing;
-      if (!(ok = __all_sync(0xffffffffu, mbar_wait(&s.ring_full[slot], (k / kRing) & 1, w)))) break;
-      const int item = s.ring_item[slot];
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s.ring_empty[slot]);
-      if (item >= p.n_items) break;
-      const FwdItem it = decode_fwd(p, item);
+    // The item loop is software-pipelined: the next item is taken from the
+    // ring and decoded (dependent global reads) before this item's epilogue.
+    FwdItem it{};
+    it.item = INT_MAX;
+    if ((ok = __all_sync(0xffffffffu, mbar_wait(&s.ring_full[0], 0, w)))) it = s.ring[0];
+    __syncwarp();
+    if (ok && lane == 0) mbar_arrive(&s.ring_empty[0]);
+    k = 1;
+    int e = it.e0;
+    while (ok && it.item < p.n_items) {
       const int n = it.n;
+      const int* list = it.list(p);
       const int rbase = it.qb * 256 + g * kTile + wq * 32;  // first row of this warp
       const int row = rbase + lane;
+      const int4* recs = p.rec + ((size_t)it.b * sh.Hm + it.hm) * sh.nKt * kTile;
       float m_run = -INFINITY, l_run = 0.f;  // m_run in scaled log2 units
       for (int t = 0; t < n; ++t) {
-        const int e = it.list[t];
+        const int e_next = (t + 1 < n) ? list[t + 1] : 0;  // in flight during this tile
         const int cls = (e >> (2 * g)) & 3;
         const bool need = (cls != kClsFull) || ((e >> 4) & 1);
-        const int st = kv_iter % kStages;
-        const uint32_t ph = (kv_iter / kStages) & 1;
-        ok = __all_sync(0xffffffffu, mbar_wait(&s.s_full[g], tile_cnt & 1, w));
-        if (need && ok) ok = __all_sync(0xffffffffu, mbar_wait(&s.k_full[st], ph, w));
-        if (!ok) break;
+        uint32_t mw[4] = {0u, 0u, 0u, 0u};
+        if (need) {
+          // column words (this lane's 4 columns) -> row words by transposition
+          const int4* mrec = recs + (size_t)(e >> 8) * kTile;
+          int4 r4[4];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) r4[c] = __ldg(mrec + c * 32 + lane);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) mw[c] = warp_transpose32(column_row_bits(r4[c], rbase), lane);
+        }
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(&s.s_full[g], tile_cnt & 1, w)))) break;
         tc_fence_after();
         float x[128];
         uint32_t* raw = reinterpret_cast<uint32_t*>(x);
@@ -314,13 +330,6 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
         tmem_ld32x(tb + s_col + 32, raw + 32);
         tmem_ld32x(tb + s_col + 64, raw + 64);
         tmem_ld32x(tb + s_col + 96, raw + 96);
-        uint32_t mw[4] = {0u, 0u, 0u, 0u};
-        if (need) {
-          // column words (this lane's 4 columns) -> row words by transposition
-          const int4* mrec = s.mask[st];
-#pragma unroll
-          for (int c = 0; c < 4; ++c) mw[c] = warp_transpose32(column_row_bits(mrec[c * 32 + lane], rbase), lane);
-        }
         tmem_ld_wait();
         if (need) {
 #pragma unroll
@@ -378,34 +387,51 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
         tmem_st_wait();
         tc_fence_before();
         mbar_arrive(&s.p_full[g]);
-        ++kv_iter;
         ++tile_cnt;
+        e = e_next;
       }
       if (!ok) break;
-      // ---------------- epilogue ----------------
+      // next item: take it from the ring and decode it now
+      const FwdItem cur = it;
+      {
+        const int slot = k % kRing;
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(&s.ring_full[slot], (k / kRing) & 1, w)))) break;
+        it = s.ring[slot];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s.ring_empty[slot]);
+        ++k;
+        e = it.e0;
+      }
+      // ---------------- epilogue of the current item ----------------
       if (n > 0 && !(ok = __all_sync(0xffffffffu, mbar_wait(&s.o_full[g], act & 1, w)))) break;
       tc_fence_after();
       const bool valid = row < sh.Nq;
       const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
-      __nv_bfloat16* orow = p.o + (((size_t)it.b * sh.Nq + (valid ? row : 0)) * sh.Hq + it.h) * D;
+      __nv_bfloat16* orow = p.o + (((size_t)cur.b * sh.Nq + (valid ? row : 0)) * sh.Hq + cur.h) * D;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t o[32];
+      for (int c = 0; c < D / 64; ++c) {
+        uint32_t o[64];
         if (n > 0) {
-          tmem_ld32x(tb + o_col + c * 32, o);
+          tmem_ld32x(tb + o_col + c * 64, o);
+          tmem_ld32x(tb + o_col + c * 64 + 32, o + 32);
           tmem_ld_wait();
         } else {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = 0u;
+          for (int i = 0; i < 64; ++i) o[i] = 0u;
         }
-        uint32_t pkd[16];
+        uint32_t pkd[32];
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
+        for (int i = 0; i < 32; ++i)
           pkd[i] = pack_bf16x2(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
         if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+          if (o_v8) {
 #pragma unroll
-          for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pkd[4 * i], pkd[4 * i + 1], pkd[4 * i + 2], pkd[4 * i + 3]);
+            for (int i = 0; i < 4; ++i) st_global_v8(orow + c * 64 + i * 16, pkd + 8 * i);
+          } else {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c * 64);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) dst[i] = make_uint4(pkd[4 * i], pkd[4 * i + 1], pkd[4 * i + 2], pkd[4 * i + 3]);
+          }
         }
       }
       if (n > 0) {
@@ -414,7 +440,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
         ++act;
       }
       if (valid)
-        p.lse[((size_t)it.b * sh.Hq + it.h) * sh.Nq + row] =
+        p.lse[((size_t)cur.b * sh.Hq + cur.h) * sh.Nq + row] =
             (l_run > 0.f) ? (m_run + log2f(l_run)) * 0.69314718055994531f : -INFINITY;
     }
   }
@@ -431,11 +457,8 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
     }
     if (warp == Cfg::kProducerWarp && lane == 0) {
       if (q_armed) (void)mbar_wait(&s.q_full, q_par, w2);
-      for (int st = 0; st < kStages; ++st)
-        if (k_armed & (1u << st)) {
-          (void)mbar_wait(&s.k_full[st], k_par[st], w2);
-          (void)mbar_wait(&s.v_full[st], k_par[st], w2);
-        }
+      for (int sl = 0; sl < kSlots; ++sl)
+        if (slot_armed & (1u << sl)) (void)mbar_wait(&s.slot_full[sl], (slot_par >> sl) & 1, w2);
     }
   }
   tc_fence_before();
