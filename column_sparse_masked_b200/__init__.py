@@ -25,6 +25,7 @@ from ._binding import (  # noqa: F401
     fwd,
     bwd,
     get_status,
+    get_timeout_info,
     launch_count,
     lib_path,
     load_library,
@@ -39,7 +40,7 @@ from ._binding import (  # noqa: F401
 )
 
 __all__ = [
-    "FlashMaskError", "classify", "count_unmasked", "flashmask_attention", "fwd", "bwd", "get_status",
+    "FlashMaskError", "classify", "count_unmasked", "flashmask_attention", "fwd", "bwd", "get_status", "get_timeout_info",
     "launch_count", "lib_path", "load_library", "localize", "localize_multi", "profiler_enable", "profiler_read", "set_wait_limit_ns", "test_wait_timeout",
     "version", "workspace_size",
 ]

@@ -25,6 +25,7 @@ _SIGS = {
     "flashmask_localize": (ctypes.c_int, [_P, _P, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, _P]),
     "flashmask_localize_multi": (ctypes.c_int, [_P, _P, ctypes.c_int64, _P, _P, ctypes.c_int32, _P]),
     "flashmask_count_unmasked": (ctypes.c_int, [_P, _P, _P, _P, _DIMS, _P, _P]),
+    "flashmask_get_timeout_info": (ctypes.c_int, [_P]),
     "flashmask_get_status": (ctypes.c_int, []),
     "flashmask_set_wait_limit_ns": (None, [ctypes.c_int64]),
     "flashmask_test_wait_timeout": (ctypes.c_int, [ctypes.c_int64, _P]),
@@ -227,6 +228,18 @@ def get_status() -> int:
     return int(load_library().flashmask_get_status())
 
 
+_TIMEOUT_KERNELS = ("forward", "backward key side", "backward query side", "wait self-test")
+
+
+def get_timeout_info() -> dict:
+    """The bounded wait behind the first timeout since the status word was last cleared."""
+    info = (ctypes.c_int32 * 5)()
+    _check(load_library().flashmask_get_timeout_info(info), "flashmask_get_timeout_info")
+    k = int(info[0])
+    return {"kernel": _TIMEOUT_KERNELS[k] if 0 <= k < len(_TIMEOUT_KERNELS) else k,
+            "barrier_offset": int(info[1]), "parity": int(info[2]), "block": int(info[3]), "thread": int(info[4])}
+
+
 def set_wait_limit_ns(ns: int) -> None:
     load_library().flashmask_set_wait_limit_ns(ctypes.c_int64(int(ns)))
 
@@ -244,12 +257,13 @@ def profiler_enable(on: bool = True) -> None:
 
 
 def profiler_read():
-    """{'fwd_ms', 'fwd_launches', 'bwd_kv_ms', 'bwd_kv_launches', 'bwd_q_ms', 'bwd_q_launches'} since the last read."""
-    ms = (ctypes.c_double * 3)()
-    cnt = (ctypes.c_int64 * 3)()
+    """{'<kind>_ms', '<kind>_launches'} since the last read, kinds fwd, bwd_kv, bwd_q and bwd_pair
+    (the two backward kernels run concurrently; bwd_pair is their joint duration)."""
+    ms = (ctypes.c_double * 4)()
+    cnt = (ctypes.c_int64 * 4)()
     _check(load_library().flashmask_profiler_read(ms, cnt), "flashmask_profiler_read")
     out = {}
-    for i, k in enumerate(("fwd", "bwd_kv", "bwd_q")):
+    for i, k in enumerate(("fwd", "bwd_kv", "bwd_q", "bwd_pair")):
         out[f"{k}_ms"] = ms[i]
         out[f"{k}_launches"] = cnt[i]
     return out

@@ -208,7 +208,7 @@ __global__ void __launch_bounds__(kvb::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
-  const WaitCtx w{&s.abort_flag, p.status, p.wait_limit_ns};
+  const WaitCtx w{&s.abort_flag, p.status, p.wait_limit_ns, smem_addr(smem_raw), 1};
   uint32_t kv_par = 0, kv_armed = 0, vv_par = 0, vv_armed = 0;
   uint32_t q_par[kQStages] = {}, do_par[kDoStages] = {}, l_par[kLStages] = {};
   uint32_t q_armed = 0, do_armed = 0, l_armed = 0;
@@ -403,10 +403,16 @@ __global__ void __launch_bounds__(kvb::kThreads, 1)
           tmem_ld32x(tb + kColS + c0 + 32, pr + 32);
           tmem_ld_wait();
 #pragma unroll
-          for (int i = 0; i < 64; ++i) {
-            const float pv = fast_exp2(fmaf(__uint_as_float(pr[i]), p.scale_log2, -l2[i]));
-            const uint32_t bit = ((i < 32 ? mw0 : mw1) >> (i & 31)) & 1u;
-            pr[i] = bit ? 0u : __float_as_uint(pv);
+          for (int i4 = 0; i4 < 16; ++i4) {  // 16-byte broadcast reads of the rows' LSE2
+            const float4 lv = reinterpret_cast<const float4*>(l2)[i4];
+            const float lq[4] = {lv.x, lv.y, lv.z, lv.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              const int i = i4 * 4 + u;
+              const float pv = fast_exp2(fmaf(__uint_as_float(pr[i]), p.scale_log2, -lq[u]));
+              const uint32_t bit = ((i < 32 ? mw0 : mw1) >> (i & 31)) & 1u;
+              pr[i] = bit ? 0u : __float_as_uint(pv);
+            }
           }
           {
             uint32_t pk[32];
@@ -427,8 +433,15 @@ __global__ void __launch_bounds__(kvb::kThreads, 1)
             tmem_ld32x(tb + kColDP + c0 + 32, r + 32);
             tmem_ld_wait();
 #pragma unroll
-            for (int i = 0; i < 64; ++i)
-              pr[i] = __float_as_uint(__uint_as_float(pr[i]) * (__uint_as_float(r[i]) - dsm[i]));
+            for (int i4 = 0; i4 < 16; ++i4) {  // 16-byte broadcast reads of the rows' D
+              const float4 dv4 = reinterpret_cast<const float4*>(dsm)[i4];
+              const float dq4[4] = {dv4.x, dv4.y, dv4.z, dv4.w};
+#pragma unroll
+              for (int u = 0; u < 4; ++u) {
+                const int i = i4 * 4 + u;
+                pr[i] = __float_as_uint(__uint_as_float(pr[i]) * (__uint_as_float(r[i]) - dq4[u]));
+              }
+            }
           }
           {
             uint32_t pk[32];
@@ -485,7 +498,7 @@ __global__ void __launch_bounds__(kvb::kThreads, 1)
   // ---------------- teardown ----------------
   __syncthreads();
   if (s.abort_flag) {
-    const WaitCtx w2{&s.no_abort, p.status, p.wait_limit_ns};
+    const WaitCtx w2{&s.no_abort, p.status, p.wait_limit_ns, smem_addr(smem_raw), 1};
     if (warp == kMmaWarp && lane == 0) {
       mma_commit(&s.teardown);
       (void)mbar_wait(&s.teardown, 0, w2);
@@ -517,10 +530,10 @@ static cudaError_t launch_dkdv_d(const BwdParams& p, const CUtensorMap& tq, cons
   const int smem = (int)sizeof(DkdvSmem<D>);
   cudaError_t e = ensure_smem_limit((const void*)fm_bwd_dkdv_kernel<D>, smem);
   if (e != cudaSuccess) return e;
-  profile_begin(1, st);
+  const int prof = profile_begin(1, st);
   note_launch();
   fm_bwd_dkdv_kernel<D><<<grid, kvb::kThreads, smem, st>>>(tq, tk, tv, tdo, p);
-  profile_end(1, st);
+  profile_end(prof, st);
   return cudaGetLastError();
 }
 

@@ -20,7 +20,11 @@
 // MMA issue order: S(0) dP(0) | S(t+1) , dP(t+1) , dQ += dS(t) K(t) | ...
 // where dP(t+1) waits only until the compute warps have loaded dP(t) into
 // registers (dS(t) is written over S(t), not over dP), so the next tile's dP
-// is computed while the compute warps evaluate the current tile.
+// is computed while the compute warps evaluate the current tile.  The compute
+// warps can then complete tile t+1 before the MMA warp has seen "dS(t)
+// written", so that signal alternates between two barriers by tile parity: a
+// parity wait never sees its barrier two phases ahead (tile t+2 needs S(t+2),
+// issued only after dQ(t)).
 // K tiles (3-deep ring, freed after dQ) and V tiles (2-deep, freed after dP)
 // stream through separate rings; the element mask of a partial tile is built
 // from the boundary records read straight from global memory (L2-resident),
@@ -65,7 +69,7 @@ struct __align__(1024) DqSmem {
   uint64_t q_full, q_empty;
   uint64_t k_full[qb::kKStages], k_empty[qb::kKStages];
   uint64_t v_full[qb::kVStages], v_empty[qb::kVStages];
-  uint64_t s_full[2], dp_full, dp_read, ds_full;
+  uint64_t s_full[2], dp_full, dp_read, ds_full[2];
   uint64_t dq_full, dq_free;
   uint64_t teardown;
   uint32_t tmem_base;
@@ -176,7 +180,8 @@ __global__ void __launch_bounds__(qb::kThreads, 1)
     mbar_init(&s.s_full[1], 1);
     mbar_init(&s.dp_full, 1);
     mbar_init(&s.dp_read, 256);
-    mbar_init(&s.ds_full, 256);
+    mbar_init(&s.ds_full[0], 256);
+    mbar_init(&s.ds_full[1], 256);
     mbar_init(&s.dq_full, 1);
     mbar_init(&s.dq_free, 256);
     mbar_init(&s.teardown, 1);
@@ -194,7 +199,7 @@ __global__ void __launch_bounds__(qb::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
-  const WaitCtx w{&s.abort_flag, p.status, p.wait_limit_ns};
+  const WaitCtx w{&s.abort_flag, p.status, p.wait_limit_ns, smem_addr(smem_raw), 2};
   uint32_t q_par = 0, q_armed = 0, k_par[kKStages] = {}, v_par[kVStages] = {}, k_armed = 0, v_armed = 0;
 
   if (warp == kProducerWarp) {
@@ -314,7 +319,7 @@ __global__ void __launch_bounds__(qb::kThreads, 1)
             if (j + 2 == n) mma_commit(&s.q_empty);  // last S and dP of the item issued
           }
           if (j == 0 && !(ok = mbar_wait(&s.dq_free, (act & 1) ^ 1, w))) break;  // previous dQ read out
-          if (!(ok = mbar_wait(&s.ds_full, tj & 1, w))) break;
+          if (!(ok = mbar_wait(&s.ds_full[tj & 1], (tj >> 1) & 1, w))) break;
           tc_fence_after();
           q_issue_dq<D>(tmem + kColDQ, tmem + kColS + bf * 128, s.k[sk], j > 0);  // dQ += dS K
           mma_commit(&s.k_empty[sk]);
@@ -397,7 +402,7 @@ __global__ void __launch_bounds__(qb::kThreads, 1)
         tmem_st32x(tb + kColS + bf * 128 + c0, pk);  // bf16 pairs over this warpgroup's own S columns
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(&s.ds_full);
+        mbar_arrive(&s.ds_full[tc & 1]);
         ++tc;
         return true;
       });
@@ -429,7 +434,7 @@ __global__ void __launch_bounds__(qb::kThreads, 1)
   // ---------------- teardown ----------------
   __syncthreads();
   if (s.abort_flag) {
-    const WaitCtx w2{&s.no_abort, p.status, p.wait_limit_ns};
+    const WaitCtx w2{&s.no_abort, p.status, p.wait_limit_ns, smem_addr(smem_raw), 2};
     if (warp == kMmaWarp && lane == 0) {
       mma_commit(&s.teardown);
       (void)mbar_wait(&s.teardown, 0, w2);
@@ -458,10 +463,10 @@ static cudaError_t launch_dq_d(const BwdParams& p, const CUtensorMap& tq, const 
   const int smem = (int)sizeof(DqSmem<D>);
   cudaError_t e = ensure_smem_limit((const void*)fm_bwd_dq_kernel<D>, smem);
   if (e != cudaSuccess) return e;
-  profile_begin(2, st);
+  const int prof = profile_begin(2, st);
   note_launch();
   fm_bwd_dq_kernel<D><<<grid, qb::kThreads, smem, st>>>(tq, tk, tv, tdo, p);
-  profile_end(2, st);
+  profile_end(prof, st);
   return cudaGetLastError();
 }
 

@@ -22,7 +22,10 @@
 namespace fm {
 
 // Per-device status word written by kernels (bounded-wait timeouts).
-__device__ int g_status_word;
+// [0] status word; [1..5] the wait behind the first timeout since the status
+// was last cleared: kernel, barrier offset in the kernel's shared-memory
+// struct, parity, block, thread.
+__device__ int g_status_word[8];
 
 namespace {
 
@@ -61,6 +64,32 @@ int current_device(DeviceInfo* out) {
   }
   *out = it->second;
   return FLASHMASK_OK;
+}
+
+// The library's second stream of the current device, with the fork/join
+// events of one backward call (the mutex serialises their use between host
+// threads).  Null if it could not be created: the caller's stream alone is used.
+struct AuxStream {
+  cudaStream_t stream = nullptr;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  std::mutex mu;
+};
+AuxStream* aux_stream() {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+  static std::unordered_map<int, AuxStream*> cache;
+  std::lock_guard<std::mutex> lock(g_mu);
+  auto it = cache.find(dev);
+  if (it != cache.end()) return it->second;
+  AuxStream* a = new AuxStream();
+  if (cudaStreamCreateWithFlags(&a->stream, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaEventCreateWithFlags(&a->fork, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&a->join, cudaEventDisableTiming) != cudaSuccess) {
+    delete a;  // handles of a failed set-up are left to the context (none is used)
+    a = nullptr;
+  }
+  cache.emplace(dev, a);
+  return a;
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -157,6 +186,7 @@ std::atomic<int> g_profiling{0};
 struct ProfRec {
   cudaEvent_t start = nullptr, stop = nullptr;
   int kind = 0;
+  bool closed = false;
 };
 std::vector<ProfRec> g_prof_pool;  // guarded by g_mu
 size_t g_prof_used = 0;
@@ -180,35 +210,33 @@ int wave_groups(size_t group_bytes, int n_groups, int64_t n_items, int sm_count)
 
 void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
-// A begin/end pair is recorded only while profiling is on; `end` closes the
-// record opened by the matching `begin` of the same thread (launches of the
-// library are issued from one thread per call).
-thread_local ProfRec* t_open_rec = nullptr;
+// A begin/end pair is recorded only while profiling is on.
+constexpr int kProfKinds = 4;
 
-void profile_begin(int kind, cudaStream_t st) {
-  t_open_rec = nullptr;
-  if (!g_profiling.load(std::memory_order_relaxed)) return;
+int profile_begin(int kind, cudaStream_t st) {
+  if (!g_profiling.load(std::memory_order_relaxed)) return -1;
   std::lock_guard<std::mutex> lock(g_mu);
-  if (g_prof_used >= kProfMax) return;
+  if (g_prof_used >= kProfMax) return -1;
   if (g_prof_used == g_prof_pool.size()) {
     ProfRec r;
-    if (cudaEventCreate(&r.start) != cudaSuccess || cudaEventCreate(&r.stop) != cudaSuccess) return;
+    if (cudaEventCreate(&r.start) != cudaSuccess || cudaEventCreate(&r.stop) != cudaSuccess) return -1;
     g_prof_pool.push_back(r);
   }
-  ProfRec* r = &g_prof_pool[g_prof_used++];
+  const size_t h = g_prof_used;
+  ProfRec* r = &g_prof_pool[h];
   r->kind = kind;
-  if (cudaEventRecord(r->start, st) != cudaSuccess) {
-    --g_prof_used;
-    return;
-  }
-  t_open_rec = r;
+  r->closed = false;
+  if (cudaEventRecord(r->start, st) != cudaSuccess) return -1;
+  ++g_prof_used;
+  return (int)h;
 }
 
-void profile_end(int kind, cudaStream_t st) {
-  if (!t_open_rec) return;
+void profile_end(int handle, cudaStream_t st) {
+  if (handle < 0) return;
   std::lock_guard<std::mutex> lock(g_mu);
-  if (t_open_rec->kind == kind) cudaEventRecord(t_open_rec->stop, st);
-  t_open_rec = nullptr;
+  if ((size_t)handle >= g_prof_used) return;
+  ProfRec& r = g_prof_pool[handle];
+  if (cudaEventRecord(r.stop, st) == cudaSuccess) r.closed = true;
 }
 
 cudaError_t ensure_smem_limit(const void* func, int bytes) {
@@ -291,7 +319,7 @@ int flashmask_fwd(const void* q, const void* k, const void* v, const int32_t* lt
   sp.n_items = (int)s.n_fwd_items;
   sp.items_per_group = s.nQB * s.G;
   sp.wave = wave_groups((size_t)s.Nk * s.d * 2 * 2, s.B * s.Hkv, s.n_fwd_items, di.sm_count);
-  FM_CUDA(launch_sort_units(sp, st));
+  FM_CUDA(launch_sort_units(&sp, 1, st));
 
   FwdParams fp{};
   fp.s = s;
@@ -370,7 +398,6 @@ int flashmask_bwd(const void* q, const void* k, const void* v, const void* o, co
   sb.n_items = (int)s.n_kv_items;
   sb.items_per_group = s.nKt;
   sb.wave = wave_groups((size_t)s.G * s.Nq * s.d * 2 * 2, s.B * s.Hkv, s.n_kv_items, di.sm_count);
-  if (sb.n_items > 0) FM_CUDA(launch_sort_units(sb, st));
   // query side: per q-block k-tile lists (the forward's), per q-tile counts
   pp.qcount = reinterpret_cast<int*>(ws + L.qcount);
   FM_CUDA(launch_plan_fwd(pp, st));
@@ -383,7 +410,13 @@ int flashmask_bwd(const void* q, const void* k, const void* v, const void* o, co
   sf.n_items = (int)s.n_q_items;
   sf.items_per_group = s.nQt * s.G;
   sf.wave = wave_groups((size_t)s.Nk * s.d * 2 * 2, s.B * s.Hkv, s.n_q_items, di.sm_count);
-  if (sf.n_items > 0) FM_CUDA(launch_sort_units(sf, st));
+  {
+    SortParams both[2];
+    int nsort = 0;
+    if (sb.n_items > 0) both[nsort++] = sb;
+    if (sf.n_items > 0) both[nsort++] = sf;
+    if (nsort > 0) FM_CUDA(launch_sort_units(both, nsort, st));
+  }
 
   BwdPreParams bp{};
   bp.s = s;
@@ -417,9 +450,28 @@ int flashmask_bwd(const void* q, const void* k, const void* v, const void* o, co
   kp.status = di.status;
   kp.wait_limit_ns = (uint64_t)g_wait_limit_ns.load();
   const int grid_kv = kp.n_items < di.sm_count ? kp.n_items : di.sm_count;
-  if (grid_kv > 0) FM_CUDA(launch_bwd_dkdv(kp, tq, tk, tv, tdo, grid_kv, st));
-  const int grid_q = kp.n_items2 < di.sm_count ? kp.n_items2 : di.sm_count;
-  if (has_q && grid_q > 0) FM_CUDA(launch_bwd_dq(kp, tq, tk, tv, tdo, grid_q, st));
+  const int grid_q = (has_q && kp.n_items2 > 0) ? (kp.n_items2 < di.sm_count ? kp.n_items2 : di.sm_count) : 0;
+  // The key-side and query-side kernels are independent (same inputs,
+  // disjoint outputs).  The query side runs on the library's second stream,
+  // forked from and joined back to the caller's stream, so its CTAs take the
+  // SMs that the key side's CTAs free as they run out of work.
+  AuxStream* ax = (grid_kv > 0 && grid_q > 0) ? aux_stream() : nullptr;
+  if (ax) {
+    std::lock_guard<std::mutex> lock(ax->mu);
+    const int prof = profile_begin(3, st);
+    FM_CUDA(cudaEventRecord(ax->fork, st));
+    FM_CUDA(cudaStreamWaitEvent(ax->stream, ax->fork, 0));
+    FM_CUDA(launch_bwd_dkdv(kp, tq, tk, tv, tdo, grid_kv, st));
+    FM_CUDA(launch_bwd_dq(kp, tq, tk, tv, tdo, grid_q, ax->stream));
+    FM_CUDA(cudaEventRecord(ax->join, ax->stream));
+    FM_CUDA(cudaStreamWaitEvent(st, ax->join, 0));
+    profile_end(prof, st);
+  } else {
+    const int prof = profile_begin(3, st);
+    if (grid_kv > 0) FM_CUDA(launch_bwd_dkdv(kp, tq, tk, tv, tdo, grid_kv, st));
+    if (grid_q > 0) FM_CUDA(launch_bwd_dq(kp, tq, tk, tv, tdo, grid_q, st));
+    profile_end(prof, st);
+  }
   return FLASHMASK_OK;
 }
 
@@ -500,6 +552,17 @@ int flashmask_get_status(void) {
   return v;
 }
 
+int flashmask_get_timeout_info(int32_t* info) {
+  if (!info) return FLASHMASK_ERR_INVALID_ARG;
+  DeviceInfo di;
+  FM_TRY(current_device(&di));
+  if (cudaDeviceSynchronize() != cudaSuccess) return FLASHMASK_ERR_CUDA;
+  int v[8] = {};
+  if (cudaMemcpy(v, di.status, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return FLASHMASK_ERR_CUDA;
+  for (int i = 0; i < 5; ++i) info[i] = v[1 + i];
+  return FLASHMASK_OK;
+}
+
 void flashmask_set_wait_limit_ns(int64_t ns) { g_wait_limit_ns.store(ns > 0 ? ns : 2000000000LL); }
 
 int flashmask_test_wait_timeout(int64_t limit_ns, void* stream) {
@@ -517,22 +580,23 @@ int flashmask_profiler_enable(int on) {
 
 int flashmask_profiler_read(double* ms_out, int64_t* launches_out) {
   std::lock_guard<std::mutex> lock(g_mu);
-  double ms[3] = {0.0, 0.0, 0.0};
-  int64_t cnt[3] = {0, 0, 0};
+  double ms[kProfKinds] = {};
+  int64_t cnt[kProfKinds] = {};
   int rc = FLASHMASK_OK;
   for (size_t i = 0; i < g_prof_used; ++i) {
     ProfRec& r = g_prof_pool[i];
+    if (!r.closed) continue;
     float t = 0.f;
     if (cudaEventSynchronize(r.stop) != cudaSuccess || cudaEventElapsedTime(&t, r.start, r.stop) != cudaSuccess) {
       rc = FLASHMASK_ERR_CUDA;
       continue;
     }
-    const int kd = (r.kind >= 0 && r.kind < 3) ? r.kind : 0;
+    const int kd = (r.kind >= 0 && r.kind < kProfKinds) ? r.kind : 0;
     ms[kd] += t;
     cnt[kd] += 1;
   }
   g_prof_used = 0;
-  for (int kd = 0; kd < 3; ++kd) {
+  for (int kd = 0; kd < kProfKinds; ++kd) {
     if (ms_out) ms_out[kd] = ms[kd];
     if (launches_out) launches_out[kd] = cnt[kd];
   }

@@ -177,7 +177,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
-  const WaitCtx w{&s.abort_flag, p.status, p.wait_limit_ns};
+  const WaitCtx w{&s.abort_flag, p.status, p.wait_limit_ns, smem_addr(smem_raw), 0};
   uint32_t q_par = 0, q_armed = 0, slot_par = 0, slot_armed = 0;  // producer: copies that may be in flight
 
   if (warp == Cfg::kProducerWarp) {
@@ -450,7 +450,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
   if (s.abort_flag) {
     // Let copies and MMAs that are still in flight land before the CTA's
     // shared memory and tensor memory are released.
-    const WaitCtx w2{&s.no_abort, p.status, p.wait_limit_ns};
+    const WaitCtx w2{&s.no_abort, p.status, p.wait_limit_ns, smem_addr(smem_raw), 0};
     if (warp == Cfg::kMmaWarp && lane == 0) {
       mma_commit(&s.teardown);
       (void)mbar_wait(&s.teardown, 0, w2);
@@ -475,10 +475,10 @@ static cudaError_t launch_fwd_d(const FwdParams& p, const CUtensorMap& tq, const
   const int smem = (int)sizeof(FwdSmem<D>);
   cudaError_t e = ensure_smem_limit((const void*)fm_fwd_kernel<D>, smem);
   if (e != cudaSuccess) return e;
-  profile_begin(0, st);
+  const int prof = profile_begin(0, st);
   note_launch();
   fm_fwd_kernel<D><<<grid, FwdCfg<D>::kThreads, smem, st>>>(tq, tk, tv, p);
-  profile_end(0, st);
+  profile_end(prof, st);
   return cudaGetLastError();
 }
 

@@ -11,7 +11,8 @@ cudaError_t launch_mask_prep(const MaskPrepParams& p, cudaStream_t st);
 cudaError_t launch_plan_fwd(const PlanParams& p, cudaStream_t st);
 cudaError_t launch_plan_bwd(const PlanParams& p, cudaStream_t st);
 cudaError_t launch_classify_export(const PlanParams& p, cudaStream_t st);
-cudaError_t launch_sort_units(const SortParams& p, cudaStream_t st);
+// Sorts the work items of count (1 or 2) independent orders, one block each.
+cudaError_t launch_sort_units(const SortParams* ps, int count, cudaStream_t st);
 cudaError_t launch_localize(const int32_t* in, int32_t* out, int64_t n, int32_t a, int32_t b, cudaStream_t st);
 cudaError_t launch_localize_multi(const int32_t* in, int32_t* out, int64_t n, const int32_t* starts,
                                   const int32_t* ends, int nchunks, cudaStream_t st);
@@ -28,12 +29,14 @@ cudaError_t launch_bwd_dkdv(const BwdParams& p, const CUtensorMap& tq, const CUt
 cudaError_t launch_bwd_dq(const BwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                           const CUtensorMap& tdo, int grid, cudaStream_t st);
 
-// Launch bookkeeping: counts every launch; brackets the attention kernels
-// with profiler events when profiling is enabled (kind 0 forward, 1 backward
-// dK/dV, 2 backward dQ).
+// Launch bookkeeping: counts every launch.
 void note_launch();
-void profile_begin(int kind, cudaStream_t st);
-void profile_end(int kind, cudaStream_t st);
+// Kernel timing (while profiling is on): begin records a start event on st and
+// returns a handle (-1 when nothing was recorded); end records the matching
+// stop event.  Kinds: 0 forward, 1 backward key side, 2 backward query side,
+// 3 the backward attention pair (fork to join).
+int profile_begin(int kind, cudaStream_t st);
+void profile_end(int handle, cudaStream_t st);
 
 // Raises a kernel's dynamic shared-memory limit once per (kernel, device).
 cudaError_t ensure_smem_limit(const void* func, int bytes);

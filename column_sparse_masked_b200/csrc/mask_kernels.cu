@@ -197,8 +197,7 @@ __device__ __forceinline__ unsigned item_cost(const SortParams& p, int i) {
   return (unsigned)p.count[((size_t)c.b * s.Hm + hm) * (s.nQB * 2) + c.t];
 }
 
-__global__ void __launch_bounds__(1024) sort_units_kernel(SortParams p) {
-  extern __shared__ unsigned long long keys[];
+__device__ void sort_units_body(const SortParams& p, unsigned long long* keys) {
   const int n = p.n_items;
   const int t = threadIdx.x;
   if (t == 0) p.counter[0] = 0;
@@ -235,6 +234,16 @@ __global__ void __launch_bounds__(1024) sort_units_kernel(SortParams p) {
     }
   }
   for (int u = t; u < n; u += blockDim.x) p.order[u] = (int)(keys[u] & 0xffffffffu);
+}
+
+// One block per order: block b sorts the units of p[b] (two independent sorts
+// share a launch).
+struct SortPair {
+  SortParams p[2];
+};
+__global__ void __launch_bounds__(1024) sort_units_kernel(SortPair sp) {
+  extern __shared__ unsigned long long keys[];
+  sort_units_body(sp.p[blockIdx.x], keys);
 }
 
 // ----------------------------------------------------------------------------
@@ -306,7 +315,7 @@ __global__ void wait_timeout_kernel(int* status, uint64_t limit_ns) {
   }
   __syncthreads();
   if (threadIdx.x == 0) {
-    WaitCtx w{&abort_flag, status, limit_ns};
+    WaitCtx w{&abort_flag, status, limit_ns, smem_addr(&bar), 3};
     (void)mbar_wait(&bar, 0, w);  // gives up after limit_ns, records the timeout
   }
   __syncthreads();
@@ -343,15 +352,24 @@ cudaError_t launch_classify_export(const PlanParams& p, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_sort_units(const SortParams& p, cudaStream_t st) {
-  const int n = p.n_items;
+static size_t sort_smem(const SortParams& p) {
   int np2 = 1;
-  while (np2 < n) np2 <<= 1;
-  const size_t smem = (p.wave > 0 && n <= kSortMax) ? (size_t)np2 * sizeof(unsigned long long) : 0;
+  while (np2 < p.n_items) np2 <<= 1;
+  return (p.wave > 0 && p.n_items <= kSortMax) ? (size_t)np2 * sizeof(unsigned long long) : 0;
+}
+
+cudaError_t launch_sort_units(const SortParams* ps, int count, cudaStream_t st) {
+  if (count < 1 || count > 2) return cudaErrorInvalidValue;
+  SortPair sp{};
+  size_t smem = 0;
+  for (int i = 0; i < count; ++i) {
+    sp.p[i] = ps[i];
+    smem = sort_smem(ps[i]) > smem ? sort_smem(ps[i]) : smem;
+  }
   cudaError_t e = ensure_smem_limit((const void*)sort_units_kernel, (int)(kSortMax * sizeof(unsigned long long)));
   if (e != cudaSuccess) return e;
-  { note_launch(); sort_units_kernel<<<1, 1024, smem, st>>>(p);
-  }
+  note_launch();
+  sort_units_kernel<<<count, 1024, smem, st>>>(sp);
   return cudaGetLastError();
 }
 

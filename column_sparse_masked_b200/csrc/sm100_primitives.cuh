@@ -63,8 +63,10 @@ __device__ __forceinline__ uint32_t mbar_try_wait(uint64_t* bar, uint32_t parity
 // memory: once any role of the CTA gives up, the others stop waiting too.
 struct WaitCtx {
   volatile int* abort;   // shared-memory flag of this CTA
-  int* status;           // per-device status word (global)
+  int* status;           // per-device status word (global), followed by the timeout record
   uint64_t limit_ns;     // wall-clock limit of one wait
+  uint32_t smem_base;    // shared-window address of the CTA's shared-memory struct
+  int kernel;            // 0 forward, 1 backward key side, 2 backward query side, 3 self-test
 };
 
 // Waits for the phase with the given parity to complete.  Returns false
@@ -79,7 +81,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
       if (*w.abort) return false;
       if (global_timer_ns() - t0 > w.limit_ns) {
         *w.abort = 1;
-        atomicCAS(w.status, 0, kDevErrTimeout);
+        if (atomicCAS(w.status, 0, kDevErrTimeout) == 0) {
+          // first timeout since the status was cleared: say which wait it was
+          w.status[1] = w.kernel;
+          w.status[2] = (int)(smem_addr(bar) - w.smem_base);
+          w.status[3] = (int)parity;
+          w.status[4] = (int)blockIdx.x;
+          w.status[5] = (int)threadIdx.x;
+        }
         return false;
       }
     }

@@ -128,6 +128,12 @@ size_t flashmask_bwd_workspace_size(const flashmask_dims* dims);
  * outputs for the same inputs.  Key columns that no row sees get dK = dV = 0;
  * fully masked rows get dQ = 0.  Outputs are written in full, each element by
  * exactly one CTA (no atomics): results are deterministic.
+ * The dK/dV kernel runs on `stream`; the dQ kernel runs alongside it on a
+ * stream the library owns (one per device, created on first use), ordered
+ * after the call's earlier work on `stream` by an event and joined back to
+ * `stream` by another: everything the call writes is complete in `stream`
+ * order when the call's last operation there completes.  Concurrent calls
+ * from several host threads share that stream and are serialised on it.
  */
 int flashmask_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
                   const int32_t* lts, const int32_t* lte, const int32_t* uts, const int32_t* ute, float scale,
@@ -181,6 +187,16 @@ int flashmask_count_unmasked(const int32_t* lts, const int32_t* lte, const int32
  * FLASHMASK_ERR_* code written by a kernel) and resets it to 0. */
 int flashmask_get_status(void);
 
+/* Synchronises the current device and copies into info[5] the description of
+ * the bounded wait that caused the first FLASHMASK_ERR_TIMEOUT since the
+ * status word was last cleared (left unchanged when none occurred since):
+ * info[0] kernel (0 forward, 1 backward key side, 2 backward query side,
+ * 3 the flashmask_test_wait_timeout self-test), info[1] byte offset of the
+ * mbarrier in that kernel's shared-memory block, info[2] the phase parity
+ * waited for, info[3] block index, info[4] thread index.  Returns
+ * FLASHMASK_ERR_INVALID_ARG for a NULL info. */
+int flashmask_get_timeout_info(int32_t* info);
+
 /* Sets the limit of every bounded device-side wait, in nanoseconds (default
  * 2e9).  Values <= 0 restore the default.  Host-side setting, process-wide. */
 void flashmask_set_wait_limit_ns(int64_t ns);
@@ -193,11 +209,14 @@ int flashmask_test_wait_timeout(int64_t limit_ns, void* stream);
 
 /*
  * Kernel timing for benchmarks.  While enabled (on != 0), every launch of an
- * attention kernel is bracketed by a CUDA event pair recorded on the call's
- * stream.  flashmask_profiler_read() waits for the recorded events and fills
- * ms[3] / launches[3] (either may be NULL) with the summed milliseconds and
- * launch counts of kind 0 = forward, 1 = backward key side (dK, dV),
- * 2 = backward query side (dQ), then clears them.  Event pairs are pooled (at
+ * attention kernel is bracketed by a CUDA event pair recorded on the stream it
+ * runs on, and so is the backward's pair of attention kernels as a whole (on
+ * the call's stream, from before the key-side launch to after both kernels
+ * completed).  flashmask_profiler_read() waits for the recorded events and
+ * fills ms[4] / launches[4] (either may be NULL) with the summed milliseconds
+ * and counts of kind 0 = forward, 1 = backward key side (dK, dV), 2 = backward
+ * query side (dQ), 3 = the backward pair (kinds 1 and 2 run concurrently, so
+ * 3 is their joint duration), then clears them.  Event pairs are pooled (at
  * most 4096 outstanding).  Host-side, process-wide.
  */
 int flashmask_profiler_enable(int on);

@@ -150,6 +150,9 @@ def test_bounded_wait_timeout_reports_status():
     assert fm.get_status() == 0
     fm.test_wait_timeout(2_000_000)  # 2 ms
     assert fm.get_status() == -6
+    info = fm.get_timeout_info()
+    assert info["kernel"] == "wait self-test" and info["barrier_offset"] == 0 and info["parity"] == 0
+    assert info["block"] == 0 and info["thread"] == 0
     assert fm.get_status() == 0  # cleared
     q, k, v, do, masks = make_case(1, 256, 256, 2, 2, 1, 128, "causal", 61)
     o, lse = fm.fwd(*cuda(q, k, v), *cuda(*masks))
@@ -166,3 +169,28 @@ def test_autograd_wrapper(oracle_mod):
     check_out("dQ", qg.grad, rdq)
     check_out("dK", kg.grad, rdk)
     check_out("dV", vg.grad, rdv)
+
+
+@pytest.mark.parametrize("name", ["doc8k", "sharequestion32k"])
+def test_repeated_calls_never_time_out(name):
+    """Hundreds of back-to-back calls with a short wait limit: every barrier
+    protocol keeps its waiters within one phase (a lost phase would hang a
+    role until its bounded wait gives up and sets the status word)."""
+    w = wl.CONFIGS[name]
+    d = {k: v.cuda() for k, v in wl.make_inputs(w, with_grad=True).items()}
+    m = [d[n] for n in ("lts", "lte", "uts", "ute")]
+    fm.set_wait_limit_ns(100_000_000)
+    try:
+        o, lse = fm.fwd(d["q"], d["k"], d["v"], *m)
+        dq, dk, dv = fm.bwd(d["q"], d["k"], d["v"], o, lse, d["do"], *m)
+        for i in range(300):
+            if i % 3 == 0:
+                fm.fwd(d["q"], d["k"], d["v"], *m, out=(o, lse))
+            fm.bwd(d["q"], d["k"], d["v"], o, lse, d["do"], *m, out=(dq, dk, dv))
+        st = fm.get_status()
+        assert st == 0, (st, fm.get_timeout_info())
+        # the last results equal a fresh call's (deterministic, no stale state)
+        dq2, dk2, dv2 = fm.bwd(d["q"], d["k"], d["v"], o, lse, d["do"], *m)
+        assert torch.equal(dq, dq2) and torch.equal(dk, dk2) and torch.equal(dv, dv2)
+    finally:
+        fm.set_wait_limit_ns(0)
