@@ -67,12 +67,12 @@ __global__ void __launch_bounds__(256) fm_bwd_pre_kernel(BwdPreParams p) {
   }
 }
 
-cudaError_t launch_bwd_pre(const BwdPreParams& p, cudaStream_t st) {
+cudaError_t launch_bwd_pre(const BwdPreParams& p, int max_blocks, cudaStream_t st) {
   const int64_t rows = (int64_t)p.s.B * p.s.nQt * kTile * p.s.Hq;
   if (rows == 0) return cudaSuccess;
   const int rows_per_block = (p.s.d == 128 ? 2 : 4) * 8;
   int64_t blocks = (rows + rows_per_block - 1) / rows_per_block;
-  if (blocks > 148 * 64) blocks = 148 * 64;
+  if (blocks > max_blocks) blocks = max_blocks;  // grid-stride loop over the rows
   note_launch();
   if (p.s.d == 128)
     fm_bwd_pre_kernel<128><<<(unsigned)blocks, 256, 0, st>>>(p);

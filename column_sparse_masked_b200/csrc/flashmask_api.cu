@@ -71,7 +71,7 @@ int current_device(DeviceInfo* out) {
 // threads).  Null if it could not be created: the caller's stream alone is used.
 struct AuxStream {
   cudaStream_t stream = nullptr;
-  cudaEvent_t fork = nullptr, join = nullptr;
+  cudaEvent_t fork = nullptr, pre = nullptr, plan = nullptr, join = nullptr;
   std::mutex mu;
 };
 AuxStream* aux_stream() {
@@ -84,6 +84,8 @@ AuxStream* aux_stream() {
   AuxStream* a = new AuxStream();
   if (cudaStreamCreateWithFlags(&a->stream, cudaStreamNonBlocking) != cudaSuccess ||
       cudaEventCreateWithFlags(&a->fork, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&a->pre, cudaEventDisableTiming) != cudaSuccess ||
+      cudaEventCreateWithFlags(&a->plan, cudaEventDisableTiming) != cudaSuccess ||
       cudaEventCreateWithFlags(&a->join, cudaEventDisableTiming) != cudaSuccess) {
     delete a;  // handles of a failed set-up are left to the context (none is used)
     a = nullptr;
@@ -376,6 +378,29 @@ int flashmask_bwd(const void* q, const void* k, const void* v, const void* o, co
     FM_TRY(make_map(&tk, workspace, 1, 1, 1, s.d));
     tv = tk;
   }
+  // The preprocess (D, LSE2; HBM-bound) does not depend on the mask: it runs
+  // on the library's second stream while the caller's stream builds the lists
+  // and orders.  The query-side kernel follows it there.
+  AuxStream* ax = aux_stream();
+  std::unique_lock<std::mutex> ax_lock;
+  if (ax) ax_lock = std::unique_lock<std::mutex>(ax->mu);
+  BwdPreParams bp{};
+  bp.s = s;
+  bp.o = static_cast<const __nv_bfloat16*>(o);
+  bp.dout = static_cast<const __nv_bfloat16*>(dout);
+  bp.lse = lse;
+  bp.lse2 = reinterpret_cast<float*>(ws + L.lse2);
+  bp.dsum = reinterpret_cast<float*>(ws + L.dsum);
+  const int pre_blocks = 64 * di.sm_count;
+  if (ax) {
+    FM_CUDA(cudaEventRecord(ax->fork, st));
+    FM_CUDA(cudaStreamWaitEvent(ax->stream, ax->fork, 0));
+    if (has_q) FM_CUDA(launch_bwd_pre(bp, pre_blocks, ax->stream));
+    FM_CUDA(cudaEventRecord(ax->pre, ax->stream));
+  } else if (has_q) {
+    FM_CUDA(launch_bwd_pre(bp, pre_blocks, st));
+  }
+
   const MaskPrepParams mp = prep_params(s, L, ws, lts, lte, uts, ute);
   FM_CUDA(launch_mask_prep(mp, st));
 
@@ -418,15 +443,6 @@ int flashmask_bwd(const void* q, const void* k, const void* v, const void* o, co
     if (nsort > 0) FM_CUDA(launch_sort_units(both, nsort, st));
   }
 
-  BwdPreParams bp{};
-  bp.s = s;
-  bp.o = static_cast<const __nv_bfloat16*>(o);
-  bp.dout = static_cast<const __nv_bfloat16*>(dout);
-  bp.lse = lse;
-  bp.lse2 = reinterpret_cast<float*>(ws + L.lse2);
-  bp.dsum = reinterpret_cast<float*>(ws + L.dsum);
-  if (has_q) FM_CUDA(launch_bwd_pre(bp, st));
-
   BwdParams kp{};
   kp.s = s;
   kp.scale = sc;
@@ -452,17 +468,16 @@ int flashmask_bwd(const void* q, const void* k, const void* v, const void* o, co
   const int grid_kv = kp.n_items < di.sm_count ? kp.n_items : di.sm_count;
   const int grid_q = (has_q && kp.n_items2 > 0) ? (kp.n_items2 < di.sm_count ? kp.n_items2 : di.sm_count) : 0;
   // The key-side and query-side kernels are independent (same inputs,
-  // disjoint outputs).  The query side runs on the library's second stream,
-  // forked from and joined back to the caller's stream, so its CTAs take the
-  // SMs that the key side's CTAs free as they run out of work.
-  AuxStream* ax = (grid_kv > 0 && grid_q > 0) ? aux_stream() : nullptr;
+  // disjoint outputs).  The query side runs on the library's second stream
+  // and is joined back to the caller's stream, so its CTAs take the SMs that
+  // the key side's CTAs free as they run out of work.
   if (ax) {
-    std::lock_guard<std::mutex> lock(ax->mu);
     const int prof = profile_begin(3, st);
-    FM_CUDA(cudaEventRecord(ax->fork, st));
-    FM_CUDA(cudaStreamWaitEvent(ax->stream, ax->fork, 0));
-    FM_CUDA(launch_bwd_dkdv(kp, tq, tk, tv, tdo, grid_kv, st));
-    FM_CUDA(launch_bwd_dq(kp, tq, tk, tv, tdo, grid_q, ax->stream));
+    FM_CUDA(cudaStreamWaitEvent(st, ax->pre, 0));           // key side reads D and LSE2
+    FM_CUDA(cudaEventRecord(ax->plan, st));
+    FM_CUDA(cudaStreamWaitEvent(ax->stream, ax->plan, 0));  // query side reads the lists and orders
+    if (grid_kv > 0) FM_CUDA(launch_bwd_dkdv(kp, tq, tk, tv, tdo, grid_kv, st));
+    if (grid_q > 0) FM_CUDA(launch_bwd_dq(kp, tq, tk, tv, tdo, grid_q, ax->stream));
     FM_CUDA(cudaEventRecord(ax->join, ax->stream));
     FM_CUDA(cudaStreamWaitEvent(st, ax->join, 0));
     profile_end(prof, st);

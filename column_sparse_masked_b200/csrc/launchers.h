@@ -22,7 +22,7 @@ cudaError_t launch_wait_timeout(int* status, uint64_t limit_ns, cudaStream_t st)
 // Forward / backward attention kernels.  `grid` is the persistent CTA count.
 cudaError_t launch_fwd(const FwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                        int grid, cudaStream_t st);
-cudaError_t launch_bwd_pre(const BwdPreParams& p, cudaStream_t st);
+cudaError_t launch_bwd_pre(const BwdPreParams& p, int max_blocks, cudaStream_t st);
 // Backward, key side (dK, dV) and query side (dQ); both persistent, grid CTAs.
 cudaError_t launch_bwd_dkdv(const BwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const CUtensorMap& tdo, int grid, cudaStream_t st);
