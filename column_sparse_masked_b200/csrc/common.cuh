@@ -149,6 +149,8 @@ struct SortParams {
   int n_items;
   int items_per_group;
   int wave;
+  int cost_cap;   // costs are clamped to [0, cost_cap]
+  int n_buckets;  // > 0: counting sort over (wave, cost) buckets; 0: bitonic sort
 };
 
 struct FwdParams {

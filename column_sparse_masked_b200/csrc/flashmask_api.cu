@@ -321,6 +321,7 @@ int flashmask_fwd(const void* q, const void* k, const void* v, const int32_t* lt
   sp.n_items = (int)s.n_fwd_items;
   sp.items_per_group = s.nQB * s.G;
   sp.wave = wave_groups((size_t)s.Nk * s.d * 2 * 2, s.B * s.Hkv, s.n_fwd_items, di.sm_count);
+  finish_sort_params(sp);
   FM_CUDA(launch_sort_units(&sp, 1, st));
 
   FwdParams fp{};
@@ -423,6 +424,7 @@ int flashmask_bwd(const void* q, const void* k, const void* v, const void* o, co
   sb.n_items = (int)s.n_kv_items;
   sb.items_per_group = s.nKt;
   sb.wave = wave_groups((size_t)s.G * s.Nq * s.d * 2 * 2, s.B * s.Hkv, s.n_kv_items, di.sm_count);
+  finish_sort_params(sb);
   // query side: per q-block k-tile lists (the forward's), per q-tile counts
   pp.qcount = reinterpret_cast<int*>(ws + L.qcount);
   FM_CUDA(launch_plan_fwd(pp, st));
@@ -435,6 +437,7 @@ int flashmask_bwd(const void* q, const void* k, const void* v, const void* o, co
   sf.n_items = (int)s.n_q_items;
   sf.items_per_group = s.nQt * s.G;
   sf.wave = wave_groups((size_t)s.Nk * s.d * 2 * 2, s.B * s.Hkv, s.n_q_items, di.sm_count);
+  finish_sort_params(sf);
   {
     SortParams both[2];
     int nsort = 0;

@@ -13,6 +13,8 @@ cudaError_t launch_plan_bwd(const PlanParams& p, cudaStream_t st);
 cudaError_t launch_classify_export(const PlanParams& p, cudaStream_t st);
 // Sorts the work items of count (1 or 2) independent orders, one block each.
 cudaError_t launch_sort_units(const SortParams* ps, int count, cudaStream_t st);
+// Fills cost_cap and n_buckets (chooses the counting sort when it fits).
+void finish_sort_params(SortParams& p);
 cudaError_t launch_localize(const int32_t* in, int32_t* out, int64_t n, int32_t a, int32_t b, cudaStream_t st);
 cudaError_t launch_localize_multi(const int32_t* in, int32_t* out, int64_t n, const int32_t* starts,
                                   const int32_t* ends, int nchunks, cudaStream_t st);

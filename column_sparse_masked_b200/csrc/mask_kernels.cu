@@ -167,12 +167,17 @@ __global__ void __launch_bounds__(128) classify_export_kernel(PlanParams p) {
 }
 
 // ----------------------------------------------------------------------------
-// 3. work order of the persistent kernels (one CTA, bitonic sort in smem).
+// 3. work order of the persistent kernels (one CTA per order, in smem).
 //    Items are indexed group-major ((batch, KV head) groups), so the natural
 //    order keeps one group's data together in L2.  With wave > 0 the items of
-//    `wave` consecutive groups are taken longest-first:
-//      key = wave index << 48 | (0xFFFF - cost) << 32 | item.
-//    Also zeroes the work counter of the persistent kernel that follows.
+//    `wave` consecutive groups are taken longest-first: ascending wave index,
+//    descending cost.  With a single wave the order is a counting sort over
+//    cost buckets (histogram, scan, scatter); the order of equal-cost items is
+//    left to the atomics, which changes which CTA takes an item, never what
+//    any output element is computed from.  With several waves a bitonic sort
+//    of  key = wave index << 48 | (cost_cap - cost) << 32 | item  keeps the
+//    index order of equal-cost items.  Also zeroes the work counter of the
+//    kernel that follows.
 // ----------------------------------------------------------------------------
 constexpr int kSortMax = 16384;
 
@@ -197,6 +202,62 @@ __device__ __forceinline__ unsigned item_cost(const SortParams& p, int i) {
   return (unsigned)p.count[((size_t)c.b * s.Hm + hm) * (s.nQB * 2) + c.t];
 }
 
+// Exclusive scan of one int per thread over the block (blockDim.x <= 1024).
+__device__ int block_exclusive_scan(int v, int* wsum) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) wsum[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < nw ? wsum[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    if (lane < nw) wsum[lane] = w;  // inclusive prefix of warp totals
+  }
+  __syncthreads();
+  const int excl = x - v + (warp > 0 ? wsum[warp - 1] : 0);
+  __syncthreads();
+  return excl;
+}
+
+__device__ void counting_sort_body(const SortParams& p, int* sm) {
+  const int n = p.n_items, nb = p.n_buckets, C = p.cost_cap;
+  const int t = threadIdx.x, nt = blockDim.x;
+  int* bkt = sm;          // [n] bucket of each item
+  int* pos = sm + n;      // [n] rank within its bucket
+  int* hist = sm + 2 * n; // [nb] counts, then start offsets
+  __shared__ int wsum[32];
+  for (int b = t; b < nb; b += nt) hist[b] = 0;
+  __syncthreads();
+  for (int u = t; u < n; u += nt) {
+    const int cost = min((int)item_cost(p, u), C);
+    const int wv = (u / p.items_per_group) / p.wave;
+    const int b = wv * (C + 1) + (C - cost);  // ascending wave, descending cost
+    bkt[u] = b;
+    pos[u] = atomicAdd(&hist[b], 1);
+  }
+  __syncthreads();
+  const int chunk = (nb + nt - 1) / nt, b0 = t * chunk, b1 = min(b0 + chunk, nb);
+  int sum = 0;
+  for (int b = b0; b < b1; ++b) sum += hist[b];
+  int run = block_exclusive_scan(sum, wsum);
+  for (int b = b0; b < b1; ++b) {
+    const int c = hist[b];
+    hist[b] = run;
+    run += c;
+  }
+  __syncthreads();
+  for (int u = t; u < n; u += nt) p.order[hist[bkt[u]] + pos[u]] = u;
+}
+
 __device__ void sort_units_body(const SortParams& p, unsigned long long* keys) {
   const int n = p.n_items;
   const int t = threadIdx.x;
@@ -205,14 +266,18 @@ __device__ void sort_units_body(const SortParams& p, unsigned long long* keys) {
     for (int u = t; u < n; u += blockDim.x) p.order[u] = u;
     return;
   }
+  if (p.n_buckets > 0) {
+    counting_sort_body(p, reinterpret_cast<int*>(keys));
+    return;
+  }
   int np2 = 1;
   while (np2 < n) np2 <<= 1;
   for (int u = t; u < np2; u += blockDim.x) {
     unsigned long long key = ~0ull;
     if (u < n) {
-      const unsigned cost = min(item_cost(p, u), 0xFFFFu);
+      const unsigned cost = min(item_cost(p, u), (unsigned)p.cost_cap);
       const unsigned long long wv = (unsigned long long)((u / p.items_per_group) / p.wave);
-      key = (wv << 48) | ((unsigned long long)(0xFFFFu - cost) << 32) | (unsigned)u;
+      key = (wv << 48) | ((unsigned long long)((unsigned)p.cost_cap - cost) << 32) | (unsigned)u;
     }
     keys[u] = key;
   }
@@ -353,9 +418,30 @@ cudaError_t launch_classify_export(const PlanParams& p, cudaStream_t st) {
 }
 
 static size_t sort_smem(const SortParams& p) {
+  if (p.wave <= 0 || p.n_items > kSortMax) return 0;
+  if (p.n_buckets > 0) return (size_t)(2 * p.n_items + p.n_buckets) * sizeof(int);
   int np2 = 1;
   while (np2 < p.n_items) np2 <<= 1;
-  return (p.wave > 0 && p.n_items <= kSortMax) ? (size_t)np2 * sizeof(unsigned long long) : 0;
+  return (size_t)np2 * sizeof(unsigned long long);
+}
+
+void finish_sort_params(SortParams& p) {
+  // cost bound per mode: k-tiles of a q-block (forward), q-tiles of the group
+  // (key side), k-tiles of a q-tile (query side)
+  const Shape& s = p.s;
+  const int64_t bound = (p.mode == 1) ? (int64_t)s.G * s.nQt : (int64_t)s.nKt;
+  p.cost_cap = (int)(bound < 0xFFFF ? bound : 0xFFFF);
+  p.n_buckets = 0;
+  if (p.wave <= 0 || p.n_items <= 0 || p.n_items > kSortMax || p.items_per_group <= 0) return;
+  const int64_t groups = (p.n_items + p.items_per_group - 1) / p.items_per_group;
+  const int64_t waves = (groups + p.wave - 1) / p.wave;
+  // With several L2 waves the index order of equal-cost items (neighbouring
+  // tiles of one group, which share K/V or Q/dO) is worth keeping: the
+  // bitonic sort keeps it, the counting sort does not.  With one wave (few
+  // items, global longest-first) the counting sort is used.
+  if (waves != 1) return;
+  const int64_t nb = waves * (p.cost_cap + 1);
+  if ((2 * (int64_t)p.n_items + nb) * (int64_t)sizeof(int) <= (int64_t)kSortMax * 8) p.n_buckets = (int)nb;
 }
 
 cudaError_t launch_sort_units(const SortParams* ps, int count, cudaStream_t st) {
