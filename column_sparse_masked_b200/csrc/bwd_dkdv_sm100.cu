@@ -207,6 +207,7 @@ __global__ void __launch_bounds__(kvb::kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  griddep_wait();
   const uint32_t tmem = s.tmem_base;
   const WaitCtx w{&s.abort_flag, p.status, p.wait_limit_ns, smem_addr(smem_raw), 1};
   uint32_t kv_par = 0, kv_armed = 0, vv_par = 0, vv_armed = 0;

@@ -198,6 +198,7 @@ __global__ void __launch_bounds__(qb::kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  griddep_wait();
   const uint32_t tmem = s.tmem_base;
   const WaitCtx w{&s.abort_flag, p.status, p.wait_limit_ns, smem_addr(smem_raw), 2};
   uint32_t q_par = 0, q_armed = 0, k_par[kKStages] = {}, v_par[kVStages] = {}, k_armed = 0, v_armed = 0;

@@ -176,6 +176,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  griddep_wait();  // the lists, orders and records of the planning kernels
   const uint32_t tmem = s.tmem_base;
   const WaitCtx w{&s.abort_flag, p.status, p.wait_limit_ns, smem_addr(smem_raw), 0};
   uint32_t q_par = 0, q_armed = 0, slot_par = 0, slot_armed = 0;  // producer: copies that may be in flight
@@ -476,10 +477,9 @@ static cudaError_t launch_fwd_d(const FwdParams& p, const CUtensorMap& tq, const
   cudaError_t e = ensure_smem_limit((const void*)fm_fwd_kernel<D>, smem);
   if (e != cudaSuccess) return e;
   const int prof = profile_begin(0, st);
-  note_launch();
-  fm_fwd_kernel<D><<<grid, FwdCfg<D>::kThreads, smem, st>>>(tq, tk, tv, p);
+  const cudaError_t le = launch_after(fm_fwd_kernel<D>, dim3(grid), dim3(FwdCfg<D>::kThreads), smem, st, tq, tk, tv, p);
   profile_end(prof, st);
-  return cudaGetLastError();
+  return le;
 }
 
 cudaError_t launch_fwd(const FwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,

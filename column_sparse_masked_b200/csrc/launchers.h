@@ -33,6 +33,28 @@ cudaError_t launch_bwd_dq(const BwdParams& p, const CUtensorMap& tq, const CUten
 
 // Launch bookkeeping: counts every launch.
 void note_launch();
+
+// Launches `kernel` after the previous kernel of the stream with programmatic
+// stream serialisation: the kernel may be scheduled while its predecessor
+// finishes and must call griddep_wait() before reading that kernel's outputs.
+// Used only where the predecessor in the stream is a kernel of this library
+// (not an event wait).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_after(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                         Args... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  note_launch();
+  return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
 // Kernel timing (while profiling is on): begin records a start event on st and
 // returns a handle (-1 when nothing was recorded); end records the matching
 // stop event.  Kinds: 0 forward, 1 backward key side, 2 backward query side,

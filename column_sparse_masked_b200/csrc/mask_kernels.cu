@@ -21,6 +21,8 @@ namespace fm {
 // 1. padded boundary records + block summary, one CTA per (k-tile, hm, b)
 // ----------------------------------------------------------------------------
 __global__ void __launch_bounds__(128) mask_prep_kernel(MaskPrepParams p) {
+  griddep_wait();
+  griddep_launch_dependents();
   const int kt = blockIdx.x, hm = blockIdx.y, b = blockIdx.z;
   const int t = threadIdx.x;
   const int j = kt * kTile + t;
@@ -81,6 +83,8 @@ __device__ __forceinline__ int block_compact128(bool flag, int* warp_tot, int* t
 //     are not skipped for at least one of the two q-tiles, in increasing order
 // ----------------------------------------------------------------------------
 __global__ void __launch_bounds__(128) plan_fwd_kernel(PlanParams p) {
+  griddep_wait();
+  griddep_launch_dependents();
   const Shape& s = p.s;
   const int qb = blockIdx.x, hm = blockIdx.y, b = blockIdx.z;
   const size_t row = (size_t)b * s.Hm + hm;
@@ -125,6 +129,8 @@ __global__ void __launch_bounds__(128) plan_fwd_kernel(PlanParams p) {
 // 2b. backward work lists: per (b, hm, k-tile) the q-tiles that are not skipped
 // ----------------------------------------------------------------------------
 __global__ void __launch_bounds__(128) plan_bwd_kernel(PlanParams p) {
+  griddep_wait();
+  griddep_launch_dependents();
   const Shape& s = p.s;
   const int kt = blockIdx.x, hm = blockIdx.y, b = blockIdx.z;
   const size_t row = (size_t)b * s.Hm + hm;
@@ -307,6 +313,8 @@ struct SortPair {
   SortParams p[2];
 };
 __global__ void __launch_bounds__(1024) sort_units_kernel(SortPair sp) {
+  griddep_wait();
+  griddep_launch_dependents();
   extern __shared__ unsigned long long keys[];
   sort_units_body(sp.p[blockIdx.x], keys);
 }
@@ -398,16 +406,12 @@ cudaError_t launch_mask_prep(const MaskPrepParams& p, cudaStream_t st) {
 
 cudaError_t launch_plan_fwd(const PlanParams& p, cudaStream_t st) {
   if (p.s.B == 0 || p.s.nQB == 0) return cudaSuccess;
-  { note_launch(); plan_fwd_kernel<<<dim3(p.s.nQB, p.s.Hm, p.s.B), 128, 0, st>>>(p);
-  }
-  return cudaGetLastError();
+  return launch_after(plan_fwd_kernel, dim3(p.s.nQB, p.s.Hm, p.s.B), dim3(128), 0, st, p);
 }
 
 cudaError_t launch_plan_bwd(const PlanParams& p, cudaStream_t st) {
   if (p.s.B == 0 || p.s.nKt == 0) return cudaSuccess;
-  { note_launch(); plan_bwd_kernel<<<dim3(p.s.nKt, p.s.Hm, p.s.B), 128, 0, st>>>(p);
-  }
-  return cudaGetLastError();
+  return launch_after(plan_bwd_kernel, dim3(p.s.nKt, p.s.Hm, p.s.B), dim3(128), 0, st, p);
 }
 
 cudaError_t launch_classify_export(const PlanParams& p, cudaStream_t st) {
@@ -454,9 +458,7 @@ cudaError_t launch_sort_units(const SortParams* ps, int count, cudaStream_t st) 
   }
   cudaError_t e = ensure_smem_limit((const void*)sort_units_kernel, (int)(kSortMax * sizeof(unsigned long long)));
   if (e != cudaSuccess) return e;
-  note_launch();
-  sort_units_kernel<<<count, 1024, smem, st>>>(sp);
-  return cudaGetLastError();
+  return launch_after(sort_units_kernel, dim3(count), dim3(1024), smem, st, sp);
 }
 
 cudaError_t launch_localize(const int32_t* in, int32_t* out, int64_t n, int32_t a, int32_t b, cudaStream_t st) {

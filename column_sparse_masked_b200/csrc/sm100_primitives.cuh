@@ -285,6 +285,15 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
+// Programmatic dependent launch.  griddep_wait: returns once the grid this one
+// was launched after (with programmatic stream serialisation) has completed
+// and its memory operations are visible; a no-op for a normal launch.  Every
+// kernel calls it before touching memory that an earlier kernel wrote.
+// griddep_launch_dependents: lets the next grid of the stream be scheduled
+// (its blocks run up to their own griddep_wait).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // 32-byte global store (sm_100 256-bit vector store); p must be 32-byte aligned.
 __device__ __forceinline__ void st_global_v8(void* p, const uint32_t* v) {
   asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(v[0]), "r"(v[1]),
