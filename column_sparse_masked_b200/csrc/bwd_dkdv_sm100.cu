@@ -55,6 +55,31 @@ constexpr int kLStages = 2;   // LSE2 / D rows: last read by the compute warps
 constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256;
 }  // namespace kvb
 
+// A decoded work item (batch, KV head, k-tile).  The first producer decodes
+// each item once and publishes it in the shared-memory ring; the other roles
+// read it there.  item >= n_items ends the work.
+struct __align__(16) KvItem {
+  int item, b, hkv, kt, total;  // total = q-tiles over all q-heads of the group
+};
+
+__device__ __forceinline__ KvItem decode_kv_item(const BwdParams& p, int item) {
+  const Shape& sh = p.s;
+  KvItem it{};
+  it.item = item;
+  if (item >= p.n_items) return it;
+  const ItemCoord c = decode_kv_item_coord(sh, p.order[item]);
+  it.b = c.b;
+  it.hkv = c.hkv;
+  it.kt = c.t;
+  it.total = 0;
+  for (int gi = 0; gi < sh.G; ++gi) {
+    const int h = it.hkv * sh.G + gi;
+    const int hm = (sh.Hm == 1) ? 0 : h;
+    it.total += p.bcount[((size_t)it.b * sh.Hm + hm) * sh.nKt + it.kt];
+  }
+  return it;
+}
+
 template <int D>
 struct __align__(1024) DkdvSmem {
   uint8_t k[kTile * D * 2];
@@ -63,7 +88,7 @@ struct __align__(1024) DkdvSmem {
   uint8_t dout[kvb::kDoStages][kTile * D * 2];
   float lse2[kvb::kLStages][kTile];
   float dsum[kvb::kLStages][kTile];
-  int ring_item[kvb::kRing];
+  KvItem ring[kvb::kRing];
   uint64_t ring_full[kvb::kRing], ring_empty[kvb::kRing];
   uint64_t k_full, k_empty, v_full, v_empty;
   uint64_t q_full[kvb::kQStages], q_empty[kvb::kQStages];
@@ -79,26 +104,6 @@ struct __align__(1024) DkdvSmem {
 
 static_assert(sizeof(DkdvSmem<128>) <= 232448, "key-side shared memory exceeds the per-CTA limit");
 static_assert(sizeof(DkdvSmem<64>) <= 232448, "key-side shared memory exceeds the per-CTA limit");
-
-struct KvItem {
-  int b, hkv, kt, total;  // total = q-tiles over all q-heads of the group
-};
-
-__device__ __forceinline__ KvItem decode_kv_item(const BwdParams& p, int item) {
-  const Shape& sh = p.s;
-  KvItem it;
-  const ItemCoord c = decode_kv_item_coord(sh, p.order[item]);
-  it.b = c.b;
-  it.hkv = c.hkv;
-  it.kt = c.t;
-  it.total = 0;
-  for (int gi = 0; gi < sh.G; ++gi) {
-    const int h = it.hkv * sh.G + gi;
-    const int hm = (sh.Hm == 1) ? 0 : h;
-    it.total += p.bcount[((size_t)it.b * sh.Hm + hm) * sh.nKt + it.kt];
-  }
-  return it;
-}
 
 // Calls f(j, h, hm, qt, cls) for the item's q-tiles in the order every role walks them.
 template <typename F>
@@ -223,10 +228,10 @@ __global__ void __launch_bounds__(kvb::kThreads, 1)
         const int slot = k % kRing;
         if (!(ok = mbar_wait(&s.ring_empty[slot], ((k / kRing) & 1) ^ 1, w))) break;
         const int item = s.abort_flag ? INT_MAX : atomicAdd(p.counter, 1);
-        s.ring_item[slot] = item;
+        const KvItem it = decode_kv_item(p, item);
+        s.ring[slot] = it;
         mbar_arrive(&s.ring_full[slot]);
         if (item >= p.n_items) break;
-        const KvItem it = decode_kv_item(p, item);
         if (it.total == 0) continue;
         if (!(ok = mbar_wait(&s.k_empty, (act & 1) ^ 1, w))) break;  // last S^T of the previous item done
         mbar_arrive_expect_tx(&s.k_full, kTileBytes);
@@ -259,10 +264,9 @@ __global__ void __launch_bounds__(kvb::kThreads, 1)
       for (uint32_t k = 0; ok; ++k) {
         const int slot = k % kRing;
         if (!(ok = mbar_wait(&s.ring_full[slot], (k / kRing) & 1, w))) break;
-        const int item = s.ring_item[slot];
+        const KvItem it = s.ring[slot];
         mbar_arrive(&s.ring_empty[slot]);
-        if (item >= p.n_items) break;
-        const KvItem it = decode_kv_item(p, item);
+        if (it.item >= p.n_items) break;
         if (it.total == 0) continue;
         if (!(ok = mbar_wait(&s.v_empty, (act & 1) ^ 1, w))) break;  // last dP^T of the previous item done
         mbar_arrive_expect_tx(&s.v_full, kTileBytes);
@@ -301,10 +305,9 @@ __global__ void __launch_bounds__(kvb::kThreads, 1)
       for (uint32_t k = 0; ok; ++k) {
         const int slot = k % kRing;
         if (!(ok = mbar_wait(&s.ring_full[slot], (k / kRing) & 1, w))) break;
-        const int item = s.ring_item[slot];
+        const KvItem it = s.ring[slot];
         mbar_arrive(&s.ring_empty[slot]);
-        if (item >= p.n_items) break;
-        const KvItem it = decode_kv_item(p, item);
+        if (it.item >= p.n_items) break;
         const int n = it.total;
         if (n == 0) continue;
         // first q-tile: S^T and dP^T
@@ -368,11 +371,10 @@ __global__ void __launch_bounds__(kvb::kThreads, 1)
     for (uint32_t k = 0; ok; ++k) {
       const int slot = k % kRing;
       if (!(ok = __all_sync(0xffffffffu, mbar_wait(&s.ring_full[slot], (k / kRing) & 1, w)))) break;
-      const int item = s.ring_item[slot];
+      const KvItem it = s.ring[slot];
       __syncwarp();
       if (lane == 0) mbar_arrive(&s.ring_empty[slot]);
-      if (item >= p.n_items) break;
-      const KvItem it = decode_kv_item(p, item);
+      if (it.item >= p.n_items) break;
       const int key = it.kt * kTile + jl;
       if (it.total > 0) {
         int cur_hm = -1;

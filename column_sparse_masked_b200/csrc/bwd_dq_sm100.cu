@@ -58,13 +58,57 @@ constexpr int kVStages = 2;  // V tiles: last read by dP(t), freed earlier
 constexpr uint32_t kColS = 0, kColDP = 256, kColDQ = 384;
 }  // namespace qb
 
+// A decoded work item (batch, q-head, q-tile).  The producer decodes each item
+// once and publishes it in the shared-memory ring; the other roles read it
+// there.  item >= n_items2 ends the work.
+struct __align__(16) QItem {
+  int item, b, h, hm, qt, g;
+  int cnt;  // entries of the q-tile's block list (for both q-tiles of the block)
+  int n;    // entries not skipped for this q-tile
+  // forward work list of the q-tile's block
+  __device__ __forceinline__ const int* list(const BwdParams& p) const {
+    const Shape& sh = p.s;
+    return p.flist + (((size_t)b * sh.Hm + hm) * sh.nQB + (qt >> 1)) * sh.nKt;
+  }
+};
+
+__device__ __forceinline__ QItem decode_q_item(const BwdParams& p, int item) {
+  const Shape& sh = p.s;
+  QItem it{};
+  it.item = item;
+  if (item >= p.n_items2) return it;
+  const ItemCoord c = decode_q_item_coord(sh, p.forder[item]);
+  it.b = c.b;
+  it.h = c.hkv * sh.G + c.hg;
+  it.hm = (sh.Hm == 1) ? 0 : it.h;
+  it.qt = c.t;
+  it.g = c.t & 1;
+  const size_t lrow = ((size_t)it.b * sh.Hm + it.hm) * sh.nQB + (c.t >> 1);
+  it.cnt = (it.qt < sh.nQt) ? p.fcount[lrow] : 0;
+  it.n = (it.qt < sh.nQt) ? p.qcount[lrow * 2 + it.g] : 0;  // per-q-tile count of the lists
+  return it;
+}
+
+// Calls f(kt, cls) for the q-tile's non-skipped k-tiles in increasing order.
+template <typename F>
+__device__ __forceinline__ bool for_each_ktile(const BwdParams& p, const QItem& it, F&& f) {
+  const int* list = it.list(p);
+  for (int t = 0; t < it.cnt; ++t) {
+    const int e = list[t];
+    const int cls = (e >> (2 * it.g)) & 3;
+    if (cls == kClsSkip) continue;
+    if (!f(e >> 8, cls)) return false;
+  }
+  return true;
+}
+
 template <int D>
 struct __align__(1024) DqSmem {
   uint8_t q[kTile * D * 2];
   uint8_t dout[kTile * D * 2];
   uint8_t k[qb::kKStages][kTile * D * 2];
   uint8_t v[qb::kVStages][kTile * D * 2];
-  int ring_item[qb::kRing];
+  QItem ring[qb::kRing];
   uint64_t ring_full[qb::kRing], ring_empty[qb::kRing];
   uint64_t q_full, q_empty;
   uint64_t k_full[qb::kKStages], k_empty[qb::kKStages];
@@ -79,43 +123,6 @@ struct __align__(1024) DqSmem {
 
 static_assert(sizeof(DqSmem<128>) <= 232448, "query-side shared memory exceeds the per-CTA limit");
 static_assert(sizeof(DqSmem<64>) <= 232448, "query-side shared memory exceeds the per-CTA limit");
-
-struct QItem {
-  int b, h, hm, qt, g;
-  const int* list;  // forward work list of the q-tile's block (entries for both q-tiles of the block)
-  int cnt;          // entries in that list
-  int n;            // entries not skipped for this q-tile
-};
-
-__device__ __forceinline__ QItem decode_q_item(const BwdParams& p, int item) {
-  const Shape& sh = p.s;
-  QItem it;
-  const ItemCoord c = decode_q_item_coord(sh, p.forder[item]);
-  it.b = c.b;
-  it.h = c.hkv * sh.G + c.hg;
-  it.hm = (sh.Hm == 1) ? 0 : it.h;
-  it.qt = c.t;
-  it.g = c.t & 1;
-  const int qbk = c.t >> 1;
-  const size_t lrow = ((size_t)it.b * sh.Hm + it.hm) * sh.nQB + qbk;
-  it.list = p.flist + lrow * sh.nKt;
-  it.cnt = (it.qt < sh.nQt) ? p.fcount[lrow] : 0;
-  it.n = 0;
-  for (int t = 0; t < it.cnt; ++t) it.n += (((it.list[t] >> (2 * it.g)) & 3) != kClsSkip) ? 1 : 0;
-  return it;
-}
-
-// Calls f(kt, cls) for the q-tile's non-skipped k-tiles in increasing order.
-template <typename F>
-__device__ __forceinline__ bool for_each_ktile(const QItem& it, F&& f) {
-  for (int t = 0; t < it.cnt; ++t) {
-    const int e = it.list[t];
-    const int cls = (e >> (2 * it.g)) & 3;
-    if (cls == kClsSkip) continue;
-    if (!f(e >> 8, cls)) return false;
-  }
-  return true;
-}
 
 // S (or dP) = A B^T over the head dimension, both K-major SW128 (128 x 128).
 template <int D>
@@ -211,10 +218,10 @@ __global__ void __launch_bounds__(qb::kThreads, 1)
         const int slot = k % kRing;
         if (!(ok = mbar_wait(&s.ring_empty[slot], ((k / kRing) & 1) ^ 1, w))) break;
         const int item = s.abort_flag ? INT_MAX : atomicAdd(p.counter2, 1);
-        s.ring_item[slot] = item;
+        const QItem it = decode_q_item(p, item);
+        s.ring[slot] = it;
         mbar_arrive(&s.ring_full[slot]);
         if (item >= p.n_items2) break;
-        const QItem it = decode_q_item(p, item);
         if (it.n == 0) continue;
         if (!(ok = mbar_wait(&s.q_empty, (act & 1) ^ 1, w))) break;
         mbar_arrive_expect_tx(&s.q_full, 2 * kTileBytes);
@@ -226,7 +233,7 @@ __global__ void __launch_bounds__(qb::kThreads, 1)
           tma_load_4d(s.dout + bx * 16384, &tdo, &s.q_full, bx * 64, it.h, it.qt * kTile, it.b);
         }
         ++act;
-        ok = for_each_ktile(it, [&](int kt, int) {
+        ok = for_each_ktile(p, it, [&](int kt, int) {
           const int sk = kv_iter % kKStages;
           const uint32_t pk = (kv_iter / kKStages) & 1;
           const int hkv = it.h / sh.G;
@@ -250,12 +257,11 @@ __global__ void __launch_bounds__(qb::kThreads, 1)
       for (uint32_t k = 0; ok; ++k) {
         const int slot = k % kRing;
         if (!(ok = mbar_wait(&s.ring_full[slot], (k / kRing) & 1, w))) break;
-        const int item = s.ring_item[slot];
+        const QItem it = s.ring[slot];
         mbar_arrive(&s.ring_empty[slot]);
-        if (item >= p.n_items2) break;
-        const QItem it = decode_q_item(p, item);
+        if (it.item >= p.n_items2) break;
         if (it.n == 0) continue;
-        ok = for_each_ktile(it, [&](int kt, int) {
+        ok = for_each_ktile(p, it, [&](int kt, int) {
           const int sv = kv_iter % kVStages;
           const uint32_t pv = (kv_iter / kVStages) & 1;
           if (!mbar_wait(&s.v_empty[sv], pv ^ 1, w)) return false;
@@ -277,10 +283,9 @@ __global__ void __launch_bounds__(qb::kThreads, 1)
       for (uint32_t k = 0; ok; ++k) {
         const int slot = k % kRing;
         if (!(ok = mbar_wait(&s.ring_full[slot], (k / kRing) & 1, w))) break;
-        const int item = s.ring_item[slot];
+        const QItem it = s.ring[slot];
         mbar_arrive(&s.ring_empty[slot]);
-        if (item >= p.n_items2) break;
-        const QItem it = decode_q_item(p, item);
+        if (it.item >= p.n_items2) break;
         const int n = it.n;
         if (n == 0) continue;
         if (!(ok = mbar_wait(&s.q_full, act & 1, w))) break;
@@ -343,11 +348,10 @@ __global__ void __launch_bounds__(qb::kThreads, 1)
     for (uint32_t k = 0; ok; ++k) {
       const int slot = k % kRing;
       if (!(ok = __all_sync(0xffffffffu, mbar_wait(&s.ring_full[slot], (k / kRing) & 1, w)))) break;
-      const int item = s.ring_item[slot];
+      const QItem it = s.ring[slot];
       __syncwarp();
       if (lane == 0) mbar_arrive(&s.ring_empty[slot]);
-      if (item >= p.n_items2) break;
-      const QItem it = decode_q_item(p, item);
+      if (it.item >= p.n_items2) break;
       if (it.qt >= sh.nQt) continue;
       const int row = it.qt * kTile + rl;
       const bool valid = row < sh.Nq;
@@ -365,7 +369,7 @@ __global__ void __launch_bounds__(qb::kThreads, 1)
       const float drow = p.dsum[roff];
       const int4* recs = p.rec + ((size_t)it.b * sh.Hm + it.hm) * sh.nKt * kTile;
       const int rbase = it.qt * kTile + wq * 32;  // first row of this warp
-      ok = for_each_ktile(it, [&](int kt, int cls) {
+      ok = for_each_ktile(p, it, [&](int kt, int cls) {
         const int bf = tc & 1;
         const bool need = cls == kClsPartial;
         // this lane's two key columns of the warpgroup's half (read early; L2-resident)

@@ -191,6 +191,7 @@ struct BwdParams {
   // query side (dQ): per (b, hm, q-block) k-tile lists, units (b, hm, q-block)
   const int* flist;
   const int* fcount;
+  const int* qcount;    // [B, Hm, nQB*2]: non-skipped k-tiles per q-tile
   const int* forder;
   int* counter2;
   int n_items2;

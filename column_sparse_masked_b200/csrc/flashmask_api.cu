@@ -458,6 +458,7 @@ int flashmask_bwd(const void* q, const void* k, const void* v, const void* o, co
   kp.n_items = (int)s.n_kv_items;
   kp.flist = pp.flist;
   kp.fcount = pp.fcount;
+  kp.qcount = pp.qcount;
   kp.forder = sf.order;
   kp.counter2 = sf.counter;
   kp.n_items2 = (int)s.n_q_items;
