@@ -212,16 +212,33 @@ __global__ void __launch_bounds__(qb::kThreads, 1)
 
   if (warp == kProducerWarp) {
     if (lane == 0) {
-      uint32_t kv_iter = 0, act = 0;
+      uint32_t kv_iter = 0, act = 0, k = 0;
       bool ok = true;
-      for (uint32_t k = 0; ok; ++k) {
+      // Items are taken one ahead: while one item's tiles stream, the next
+      // item's Q and dO are prefetched into L2, so their load (which may only
+      // start once the current item's last S and dP have been issued) hits L2.
+      auto take = [&](QItem& out) -> bool {
         const int slot = k % kRing;
-        if (!(ok = mbar_wait(&s.ring_empty[slot], ((k / kRing) & 1) ^ 1, w))) break;
+        if (!mbar_wait(&s.ring_empty[slot], ((k / kRing) & 1) ^ 1, w)) return false;
         const int item = s.abort_flag ? INT_MAX : atomicAdd(p.counter2, 1);
-        const QItem it = decode_q_item(p, item);
-        s.ring[slot] = it;
+        out = decode_q_item(p, item);
+        s.ring[slot] = out;
         mbar_arrive(&s.ring_full[slot]);
-        if (item >= p.n_items2) break;
+        ++k;
+        if (out.item < p.n_items2 && out.n > 0) {
+#pragma unroll
+          for (int bx = 0; bx < kBoxes; ++bx) {
+            tma_prefetch_l2_4d(&tq, bx * 64, out.h, out.qt * kTile, out.b);
+            tma_prefetch_l2_4d(&tdo, bx * 64, out.h, out.qt * kTile, out.b);
+          }
+        }
+        return true;
+      };
+      QItem nxt{};
+      ok = take(nxt);
+      while (ok && nxt.item < p.n_items2) {
+        const QItem it = nxt;
+        if (!(ok = take(nxt))) break;
         if (it.n == 0) continue;
         if (!(ok = mbar_wait(&s.q_empty, (act & 1) ^ 1, w))) break;
         mbar_arrive_expect_tx(&s.q_full, 2 * kTileBytes);

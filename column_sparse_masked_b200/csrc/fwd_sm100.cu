@@ -183,16 +183,33 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
 
   if (warp == Cfg::kProducerWarp) {
     if (lane == 0) {
-      uint32_t pos = 0, act = 0;  // ring position of the next K/V tile
+      uint32_t pos = 0, act = 0, k = 0;  // pos: ring position of the next K/V tile
       bool ok = true;
-      for (uint32_t k = 0; ok; ++k) {
+      // Items are taken one ahead: while one item's tiles stream, the next
+      // item's Q is prefetched into L2, so its load (which may only start
+      // once the current item's last QK^T has been issued) hits L2.
+      auto take = [&](FwdItem& out) -> bool {
         const int slot = k % kRing;
-        if (!(ok = mbar_wait(&s.ring_empty[slot], ((k / kRing) & 1) ^ 1, w))) break;
+        if (!mbar_wait(&s.ring_empty[slot], ((k / kRing) & 1) ^ 1, w)) return false;
         const int item = s.abort_flag ? INT_MAX : atomicAdd(p.counter, 1);
-        const FwdItem it = decode_fwd(p, item);
-        s.ring[slot] = it;
+        out = decode_fwd(p, item);
+        s.ring[slot] = out;
         mbar_arrive(&s.ring_full[slot]);
-        if (item >= p.n_items) break;
+        ++k;
+        if (out.item < p.n_items && out.n > 0) {
+#pragma unroll
+          for (int g = 0; g < 2; ++g)
+#pragma unroll
+            for (int bx = 0; bx < Cfg::kBoxes; ++bx)
+              tma_prefetch_l2_4d(&tq, bx * 64, out.h, out.qb * 256 + g * kTile, out.b);
+        }
+        return true;
+      };
+      FwdItem nxt{};
+      ok = take(nxt);
+      while (ok && nxt.item < p.n_items) {
+        const FwdItem it = nxt;
+        if (!(ok = take(nxt))) break;
         if (it.n == 0) continue;
         const int* list = it.list(p);
         if (!(ok = mbar_wait(&s.q_empty, (act & 1) ^ 1, w))) break;
