@@ -162,17 +162,20 @@ def recorded_traffic(kernel_file: str, workload: str):
 # ----------------------------------------------------------------------------
 # CPU oracle leg (bounded sample) -- the only place bench.py executes oracle/
 # ----------------------------------------------------------------------------
-def oracle_sample(w: wl.Workload, rows: int, inp=None):
-    """(b=0, q-head 0) restricted to its first `rows` queries and keys (mask localised onto [0, rows))."""
+def oracle_sample(w: wl.Workload, rows: int, inp=None, head: int = 0):
+    """(b=0, q-head `head` with its KV head) restricted to its first `rows` queries and keys
+    (mask localised onto [0, rows))."""
     import oracle
 
     full = wl.make_inputs(w, with_grad=True) if inp is None else inp
     n = min(rows, w.N)
-    q = full["q"][:1, :n, :1].contiguous()
-    k = full["k"][:1, :n, :1].contiguous()
-    v = full["v"][:1, :n, :1].contiguous()
-    do = full["do"][:1, :n, :1].contiguous()
-    vecs = [oracle.localize(full[m][:1, :1, :n].numpy(), 0, n) for m in ("lts", "lte", "uts", "ute")]
+    hk = head // (w.Hq // w.Hkv)
+    hm = 0 if full["lts"].shape[1] == 1 else head
+    q = full["q"][:1, :n, head:head + 1].contiguous()
+    k = full["k"][:1, :n, hk:hk + 1].contiguous()
+    v = full["v"][:1, :n, hk:hk + 1].contiguous()
+    do = full["do"][:1, :n, head:head + 1].contiguous()
+    vecs = [oracle.localize(full[m][:1, hm:hm + 1, :n].numpy(), 0, n) for m in ("lts", "lte", "uts", "ute")]
     pairs = oracle.count_unmasked(*vecs, n, n, 1)
     return q, k, v, do, vecs, pairs, n
 
@@ -187,17 +190,26 @@ def run_oracle_step(sample):
     return time.perf_counter() - t0
 
 
+CPU_TARGET_SECONDS = 10.0  # the CPU leg runs whole heads until about this much oracle time
+
+
 def cpu_baseline(w: wl.Workload, rows: int = CPU_SAMPLE_ROWS, inp=None):
+    """The oracle as it stands on the host cores: fp64 fwd+bwd of (batch 0, q-head h) restricted to
+    the first `rows` queries and keys, for h = 0, 1, ... until about CPU_TARGET_SECONDS of work."""
     import oracle
 
-    sample = oracle_sample(w, rows, inp)
-    dt = run_oracle_step(sample)
-    pairs, n = sample[5], sample[6]
+    full = wl.make_inputs(w, with_grad=True) if inp is None else inp
+    dt, pairs, heads, n = 0.0, 0, 0, min(rows, w.N)
+    while heads < w.Hq and dt < CPU_TARGET_SECONDS:
+        sample = oracle_sample(w, rows, full, head=heads)
+        dt += run_oracle_step(sample)
+        pairs += sample[5]
+        heads += 1
     ff, fb = effective_flops(pairs, w.d)
     return {"value": (ff + fb) / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
             "seconds": dt,
-            "sample": f"{w.name}: batch 0, q-head 0 with its KV head, first {n} queries x {n} keys "
-                      f"(mask localised onto [0,{n})), fp64 fwd+bwd, {pairs} unmasked pairs"}
+            "sample": f"{w.name}: batch 0, q-heads 0..{heads - 1} each with its KV head, first {n} queries x "
+                      f"{n} keys (mask localised onto [0,{n})), fp64 fwd+bwd, {pairs} unmasked pairs"}
 
 
 # ----------------------------------------------------------------------------
