@@ -89,6 +89,11 @@ def test_mask_pair_must_be_complete(lib):
     assert rc == -1
 
 
+def test_timeout_info_rejects_null(lib):
+    # checked on the host before any device access
+    assert lib.flashmask_get_timeout_info(None) == -1
+
+
 def test_localize_argument_checks(lib):
     assert lib.flashmask_localize(None, None, ctypes.c_int64(-1), 0, 1, None) == -1
     assert lib.flashmask_localize(None, None, ctypes.c_int64(10), 5, 2, None) == -1
