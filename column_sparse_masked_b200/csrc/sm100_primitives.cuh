@@ -96,7 +96,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
 }
 
 // ----------------------------------------------------------------------------
-// TMA (bulk tensor and bulk linear copies, global -> shared, no multicast)
+// TMA (bulk tensor and bulk linear copies, global -> this CTA's shared memory only)
 // ----------------------------------------------------------------------------
 __device__ __forceinline__ void tma_prefetch_map(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
