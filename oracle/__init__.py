@@ -21,6 +21,7 @@ forms, finite differences, brute force); nothing here is unpinned.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 import subprocess
@@ -39,23 +40,60 @@ _I64 = ctypes.POINTER(ctypes.c_int64)
 _U8 = ctypes.POINTER(ctypes.c_uint8)
 
 
+def _compile(src: str, out: str) -> None:
+    cmd = ["gcc", "-O2", "-march=x86-64-v3", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-o", out, src, "-lm"]
+    subprocess.run(cmd, check=True)
+
+
 def build_oracle(force: bool = False) -> str:
     """Compiles the C oracle with gcc (OpenMP, portable x86-64-v3 code)."""
     if not force and os.path.exists(_LIB_PATH) and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC):
         return _LIB_PATH
     os.makedirs(os.path.dirname(_LIB_PATH), exist_ok=True)
     tmp = _LIB_PATH + f".tmp{os.getpid()}"
-    cmd = ["gcc", "-O2", "-march=x86-64-v3", "-fopenmp", "-fPIC", "-shared", "-std=c11", "-o", tmp, _SRC, "-lm"]
-    subprocess.run(cmd, check=True)
+    _compile(_SRC, tmp)
     os.replace(tmp, _LIB_PATH)
     return _LIB_PATH
+
+
+def source() -> str:
+    """The C source of the oracle."""
+    with open(_SRC) as f:
+        return f.read()
+
+
+def build_variant(c_source: str, out_dir: str) -> str:
+    """Compiles another version of the oracle's C source (the tests plant mistakes in a copy to
+    show that the pins catch them); returns the path of the shared library."""
+    src = os.path.join(out_dir, "oracle_variant.c")
+    with open(src, "w") as f:
+        f.write(c_source)
+    out = os.path.join(out_dir, "liboracle_variant.so")
+    _compile(src, out)
+    return out
+
+
+@contextlib.contextmanager
+def use_library(path: str):
+    """Routes every oracle function through the library at `path` inside the block."""
+    global _lib
+    saved = _lib
+    _lib = _bind(ctypes.CDLL(path))
+    try:
+        yield
+    finally:
+        _lib = saved
 
 
 def _load():
     global _lib
     if _lib is not None:
         return _lib
-    lib = ctypes.CDLL(build_oracle())
+    _lib = _bind(ctypes.CDLL(build_oracle()))
+    return _lib
+
+
+def _bind(lib):
     lib.oracle_fwd_head.argtypes = [_D, _I64, ctypes.c_int64, _D, _D, ctypes.c_int64, ctypes.c_int64,
                                     _I32, _I32, _I32, _I32, ctypes.c_double, _D, _D]
     lib.oracle_dq_head.argtypes = [_D, _D, _I64, ctypes.c_int64, _D, _D, ctypes.c_int64, ctypes.c_int64,
@@ -70,7 +108,6 @@ def _load():
     lib.oracle_count_unmasked.restype = ctypes.c_int64
     lib.oracle_mask_row.argtypes = [_I32, _I32, _I32, _I32, ctypes.c_int64, ctypes.c_int64, _U8]
     lib.oracle_num_threads.restype = ctypes.c_int
-    _lib = lib
     return lib
 
 

@@ -1,0 +1,81 @@
+"""The oracle's pins catch plausible mistakes (CPU only).
+
+Each case copies the oracle's C source, plants one mistake in the copy (an
+off-by-one in the mask predicate, a dropped term, a wrong sign, a transposed
+operand, a wrong index), compiles it, routes the oracle through the mutant and
+checks that at least one pin of ``test_oracle_pins.py`` now fails.  A control
+case compiles the unchanged source the same way and checks that the same pins
+pass.  Every planted mistake keeps all memory accesses in bounds.
+"""
+import pytest
+
+import oracle
+import test_oracle_pins as pins
+
+FWD = [
+    lambda o: pins.test_unmasked_equals_sdpa(o, 33, 50, 16),
+    lambda o: pins.test_causal_encoding_equals_sdpa_causal(o, 40, 32),
+    lambda o: pins.test_random_mask_equals_sdpa_boolean_mask(o),
+    lambda o: pins.test_zero_query_closed_form_random_masks(o, 0),
+    lambda o: pins.test_golden_hand_example(o),
+]
+BWD = [
+    lambda o: pins.test_backward_finite_differences(o, 2, 4, 2),
+    lambda o: pins.test_backward_equals_torch_autograd_sdpa(o),
+]
+CLASSIFY = [lambda o, s=s: pins.test_classify_sound_random(o, s) for s in range(6)] + [
+    lambda o: pins.test_classify_causal_closed_form(o),
+]
+LOCALIZE = [lambda o, s=s: pins.test_localize_reproduces_dense_rows(o, s) for s in range(3)]
+LOCALIZE_MULTI = [lambda o, s=s: pins.test_localize_multi_reproduces_dense_rows(o, s) for s in range(3)]
+COUNT = [lambda o: pins.test_count_unmasked(o)]
+
+# (name, text in the source, planted replacement, pins expected to catch it)
+MUTATIONS = [
+    ("predicate_lts_strict", "(lts[j] <= i && i < lte[j])", "(lts[j] < i && i < lte[j])", FWD),
+    ("predicate_ute_inclusive", "(uts[j] <= i && i < ute[j])", "(uts[j] <= i && i <= ute[j])", FWD),
+    ("scale_dropped", "s_buf[j] = scale * dot(qi, k + j * d, d);", "s_buf[j] = dot(qi, k + j * d, d);", FWD),
+    ("lse_without_max", "      lse[r] = m + log(l);\n", "      lse[r] = log(l);\n", FWD),
+    ("softmax_unnormalised", "const double p = exp(s[j] - m) / l;", "const double p = exp(s[j] - m);", FWD),
+    ("ds_sign", "const double ds = s[j] * (dp[j] - D);", "const double ds = s[j] * (dp[j] + D);", BWD),
+    ("dq_wrong_operand", "g[c] += scale * ds * k[j * d + c];", "g[c] += scale * ds * v[j * d + c];", BWD),
+    ("dk_scale_dropped", "gk[c] += scale * ds * q[i * d + c];", "gk[c] += ds * q[i * d + c];", BWD),
+    ("dv_wrong_operand", "gv[c] += p * dout[i * d + c];", "gv[c] += p * q[i * d + c];", BWD),
+    ("row_sum_D_wrong_operand", "D += exp(s[j] - lse[i]) * dot(dout + i * d, v + j * d, d);",
+     "D += exp(s[j] - lse[i]) * dot(dout + i * d, k + j * d, d);", BWD),
+    ("classify_skip_uses_min", "if ((mx[0] <= r0 && mn[1] >= r1)", "if ((mn[0] <= r0 && mn[1] >= r1)", CLASSIFY),
+    ("classify_full_uses_max", "else if ((mn[0] >= r1 ||", "else if ((mx[0] >= r1 ||", CLASSIFY),
+    ("localize_shift_off_by_one", "x = x - a;", "x = x - a - 1;", LOCALIZE),
+    ("localize_multi_first_offset", "acc += x - a[t];", "acc += x - a[0];", LOCALIZE_MULTI),
+    ("count_negated", "cnt += !is_masked(", "cnt += is_masked(", COUNT),
+]
+
+
+def _fails(check) -> bool:
+    try:
+        check(oracle)
+    except AssertionError:
+        return True
+    return False
+
+
+@pytest.fixture(scope="module")
+def source():
+    oracle.build_oracle()
+    return oracle.source()
+
+
+def test_control_unchanged_source_passes_every_pin(source, tmp_path):
+    lib = oracle.build_variant(source, str(tmp_path))
+    with oracle.use_library(lib):
+        for check in FWD + BWD + CLASSIFY + LOCALIZE + LOCALIZE_MULTI + COUNT:
+            assert not _fails(check)
+
+
+@pytest.mark.parametrize("name,old,new,checks", MUTATIONS, ids=[m[0] for m in MUTATIONS])
+def test_planted_mistake_is_caught(source, tmp_path, name, old, new, checks):
+    assert source.count(old) == 1, f"{name}: the text to mutate must occur exactly once"
+    lib = oracle.build_variant(source.replace(old, new), str(tmp_path))
+    with oracle.use_library(lib):
+        caught = [i for i, check in enumerate(checks) if _fails(check)]
+    assert caught, f"{name}: no pin caught the planted mistake"
