@@ -5,7 +5,7 @@
 //
 // Method: "FlashMask-3 targets masked distributed attention on Hopper GPUs",
 // In-depth insight -- the column-wise mask (four query-axis boundary vectors
-// per key column), tiles decided from O(n) data, and the zero-communication
+// per key column), tiles decided from O(n) data, and the exchange-free
 // clip-shift-max localisation of a query chunk.
 #include <cuda_runtime.h>
 #include <climits>

@@ -122,18 +122,20 @@ int flashmask_fwd_noalloc(const void* q, const void* k, const void* v, const int
 size_t flashmask_bwd_workspace_size(const flashmask_dims* dims);
 
 /*
- * Backward of the forward above for the loss sum(O * dO) (same page:
- * "forward+backward"): dQ, dK, dV.  dK and dV sum the contributions of the
+ * Backward of the forward above for the loss sum(O * dO) (same page and
+ * section: the mask-aware kernels cover both passes): dQ, dK, dV.  dK and dV sum the contributions of the
  * Hq/Hkv q-heads that share a KV head.  `o` and `lse` must be the forward's
  * outputs for the same inputs.  Key columns that no row sees get dK = dV = 0;
  * fully masked rows get dQ = 0.  Outputs are written in full, each element by
  * exactly one CTA (no atomics): results are deterministic.
- * The dK/dV kernel runs on `stream`; the dQ kernel runs alongside it on a
- * stream the library owns (one per device, created on first use), ordered
- * after the call's earlier work on `stream` by an event and joined back to
- * `stream` by another: everything the call writes is complete in `stream`
- * order when the call's last operation there completes.  Concurrent calls
- * from several host threads share that stream and are serialised on it.
+ * The mask summary, lists, orders and the dK/dV kernel run on `stream`; the
+ * preprocess (each row's D = rowsum(dO*O) and LSE in log2 units) and the dQ
+ * kernel run on a stream the library owns (one per device, created on first
+ * use), ordered after the call's earlier work on `stream` by an event and
+ * joined back to `stream` by another: everything the call writes is complete
+ * in `stream` order when the call's last operation there completes.
+ * Concurrent calls from several host threads share that stream and are
+ * serialised on it.
  */
 int flashmask_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
                   const int32_t* lts, const int32_t* lte, const int32_t* uts, const int32_t* ute, float scale,
@@ -156,8 +158,9 @@ int flashmask_classify(const int32_t* lts, const int32_t* lte, const int32_t* ut
                        void* stream);
 
 /*
- * Clip-shift-max localisation (same page: the "provably zero-communication"
- * per-chunk mask localisation): for the contiguous query chunk [a, b),
+ * Clip-shift-max localisation (same page and section: each query chunk's
+ * mask is derived locally from the global vectors, with no data exchanged
+ * between chunks): for the contiguous query chunk [a, b),
  * out[t] = max(min(in[t], b) - a, 0) for t < n.  Applied to each of the four
  * vectors, the result encodes exactly rows [a, b) of the full mask.  in and
  * out are device int32 arrays of n elements (may alias).  0 <= a <= b.
@@ -166,8 +169,8 @@ int flashmask_localize(const int32_t* in, int32_t* out, int64_t n, int32_t a, in
 
 /*
  * Localisation onto several increasing, disjoint chunks [starts[c], ends[c])
- * concatenated in order into one local query sequence ("any multi-chunk
- * context-parallel assignment"): out[t] = sum_c (clamp(in[t], starts[c],
+ * concatenated in order into one local query sequence (a rank that holds
+ * several chunks of the sequence): out[t] = sum_c (clamp(in[t], starts[c],
  * ends[c]) - starts[c]).  starts/ends are HOST arrays of nchunks (<= 64)
  * values.
  */
@@ -223,7 +226,7 @@ int flashmask_profiler_enable(int on);
 int flashmask_profiler_read(double* ms, int64_t* launches);
 
 /* Number of kernels this library has launched since the process started
- * (every kind: summary, lists, ordering, attention, preprocess, finalise). */
+ * (every kind: summary, lists, ordering, preprocess, attention, helpers). */
 int64_t flashmask_launch_count(void);
 
 /* Human-readable text of an error code (static storage). */
