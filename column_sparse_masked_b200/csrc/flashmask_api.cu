@@ -413,7 +413,10 @@ int flashmask_bwd(const void* q, const void* k, const void* v, const void* o, co
   pp.blist = reinterpret_cast<int*>(ws + L.blist);
   pp.fcount = reinterpret_cast<int*>(ws + L.fcount);
   pp.flist = reinterpret_cast<int*>(ws + L.flist);
-  FM_CUDA(launch_plan_bwd(pp, st));
+  pp.qcount = reinterpret_cast<int*>(ws + L.qcount);
+  // key-side lists (per k-tile q-tile lists) and query-side lists (the
+  // forward's per q-block k-tile lists, per q-tile counts) in one launch
+  FM_CUDA(launch_plan_both(pp, st));
   int* counters = reinterpret_cast<int*>(ws + L.counters);
   SortParams sb{};
   sb.s = s;
@@ -425,9 +428,6 @@ int flashmask_bwd(const void* q, const void* k, const void* v, const void* o, co
   sb.items_per_group = s.nKt;
   sb.wave = wave_groups((size_t)s.G * s.Nq * s.d * 2 * 2, s.B * s.Hkv, s.n_kv_items, di.sm_count);
   finish_sort_params(sb);
-  // query side: per q-block k-tile lists (the forward's), per q-tile counts
-  pp.qcount = reinterpret_cast<int*>(ws + L.qcount);
-  FM_CUDA(launch_plan_fwd(pp, st));
   SortParams sf{};
   sf.s = s;
   sf.mode = 2;

@@ -10,6 +10,8 @@ namespace fm {
 cudaError_t launch_mask_prep(const MaskPrepParams& p, cudaStream_t st);
 cudaError_t launch_plan_fwd(const PlanParams& p, cudaStream_t st);
 cudaError_t launch_plan_bwd(const PlanParams& p, cudaStream_t st);
+// Key-side and query-side lists of the backward in one launch.
+cudaError_t launch_plan_both(const PlanParams& p, cudaStream_t st);
 cudaError_t launch_classify_export(const PlanParams& p, cudaStream_t st);
 // Sorts the work items of count (1 or 2) independent orders, one block each.
 cudaError_t launch_sort_units(const SortParams* ps, int count, cudaStream_t st);

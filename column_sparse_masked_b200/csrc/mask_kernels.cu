@@ -82,11 +82,9 @@ __device__ __forceinline__ int block_compact128(bool flag, int* warp_tot, int* t
 // 2a. forward work lists: per (b, hm, block of two q-tiles) the k-tiles that
 //     are not skipped for at least one of the two q-tiles, in increasing order
 // ----------------------------------------------------------------------------
-__global__ void __launch_bounds__(128) plan_fwd_kernel(PlanParams p) {
-  griddep_wait();
-  griddep_launch_dependents();
+__device__ void plan_fwd_body(const PlanParams& p, int qb) {
   const Shape& s = p.s;
-  const int qb = blockIdx.x, hm = blockIdx.y, b = blockIdx.z;
+  const int hm = blockIdx.y, b = blockIdx.z;
   const size_t row = (size_t)b * s.Hm + hm;
   const int qt0 = 2 * qb, qt1 = 2 * qb + 1;
   const int r00 = qt0 * kTile, r01 = min(r00 + kTile, s.Nq);
@@ -97,6 +95,7 @@ __global__ void __launch_bounds__(128) plan_fwd_kernel(PlanParams p) {
   __shared__ int total;
   __shared__ int qc[2];
   if (threadIdx.x < 2) qc[threadIdx.x] = 0;
+  __syncthreads();  // the per-q-tile counts are zeroed before any warp adds to them
   int count = 0;
   for (int base = 0; base < s.nKt; base += kTile) {
     const int kt = base + threadIdx.x;
@@ -128,11 +127,9 @@ __global__ void __launch_bounds__(128) plan_fwd_kernel(PlanParams p) {
 // ----------------------------------------------------------------------------
 // 2b. backward work lists: per (b, hm, k-tile) the q-tiles that are not skipped
 // ----------------------------------------------------------------------------
-__global__ void __launch_bounds__(128) plan_bwd_kernel(PlanParams p) {
-  griddep_wait();
-  griddep_launch_dependents();
+__device__ void plan_bwd_body(const PlanParams& p, int kt) {
   const Shape& s = p.s;
-  const int kt = blockIdx.x, hm = blockIdx.y, b = blockIdx.z;
+  const int hm = blockIdx.y, b = blockIdx.z;
   const size_t row = (size_t)b * s.Hm + hm;
   int sm[8];
   const int* src = p.ksum + (row * s.nKt + kt) * 8;
@@ -153,6 +150,30 @@ __global__ void __launch_bounds__(128) plan_bwd_kernel(PlanParams p) {
     __syncthreads();
   }
   if (threadIdx.x == 0) p.bcount[row * s.nKt + kt] = count;
+}
+
+__global__ void __launch_bounds__(128) plan_fwd_kernel(PlanParams p) {
+  griddep_wait();
+  griddep_launch_dependents();
+  plan_fwd_body(p, blockIdx.x);
+}
+
+__global__ void __launch_bounds__(128) plan_bwd_kernel(PlanParams p) {
+  griddep_wait();
+  griddep_launch_dependents();
+  plan_bwd_body(p, blockIdx.x);
+}
+
+// Both list sets of the backward in one launch: blocks [0, nKt) build the
+// key-side lists, blocks [nKt, nKt + nQB) the query-side (forward) lists.
+__global__ void __launch_bounds__(128) plan_both_kernel(PlanParams p) {
+  griddep_wait();
+  griddep_launch_dependents();
+  const int x = blockIdx.x;
+  if (x < p.s.nKt)
+    plan_bwd_body(p, x);
+  else
+    plan_fwd_body(p, x - p.s.nKt);
 }
 
 // ----------------------------------------------------------------------------
@@ -407,6 +428,11 @@ cudaError_t launch_mask_prep(const MaskPrepParams& p, cudaStream_t st) {
 cudaError_t launch_plan_fwd(const PlanParams& p, cudaStream_t st) {
   if (p.s.B == 0 || p.s.nQB == 0) return cudaSuccess;
   return launch_after(plan_fwd_kernel, dim3(p.s.nQB, p.s.Hm, p.s.B), dim3(128), 0, st, p);
+}
+
+cudaError_t launch_plan_both(const PlanParams& p, cudaStream_t st) {
+  if (p.s.B == 0 || p.s.nKt + p.s.nQB == 0) return cudaSuccess;
+  return launch_after(plan_both_kernel, dim3(p.s.nKt + p.s.nQB, p.s.Hm, p.s.B), dim3(128), 0, st, p);
 }
 
 cudaError_t launch_plan_bwd(const PlanParams& p, cudaStream_t st) {
