@@ -109,6 +109,57 @@ def _masks(lts, lte, uts, ute):
     return vecs, Hm
 
 
+def _shaped(name: str, t, shape, dtype):
+    """Checks type, dtype and shape of an argument (any device); the kernels trust these sizes."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _qkv_shapes(q, k, v):
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        if not isinstance(t, torch.Tensor) or t.dim() != 4:
+            raise ValueError(f"{n} must be a 4-D tensor [B, N, H, d]")
+    B, Nq, Hq, d = q.shape
+    Nk, Hkv = k.shape[1], k.shape[2]
+    _shaped("q", q, (B, Nq, Hq, d), torch.bfloat16)
+    _shaped("k", k, (B, Nk, Hkv, d), torch.bfloat16)
+    _shaped("v", v, (B, Nk, Hkv, d), torch.bfloat16)
+    return B, Nq, Hq, d, Nk, Hkv
+
+
+def _mask_shapes(lts, lte, uts, ute, B: int, Nk: int) -> int:
+    vecs = [lts, lte, uts, ute]
+    ref = next((x for x in vecs if x is not None), None)
+    if ref is not None and (not isinstance(ref, torch.Tensor) or ref.dim() != 3):
+        raise ValueError("mask vectors must be 3-D tensors [B, Hm, Nk]")
+    Hm = ref.shape[1] if ref is not None else 1
+    for n, x in zip(("lts", "lte", "uts", "ute"), vecs):
+        if x is not None:
+            _shaped(n, x, (B, Hm, Nk), torch.int32)
+    return Hm
+
+
+def _on_device(dev, named):
+    """Every tensor on the CUDA device `dev` and contiguous."""
+    for n, t in named:
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise TypeError(f"{n} must be a CUDA tensor")
+        if t.device != dev:
+            raise ValueError(f"{n} is on {t.device}, expected {dev}")
+        if not t.is_contiguous():
+            raise ValueError(f"{n} must be contiguous")
+
+
+def _ws_bytes(ws: torch.Tensor) -> int:
+    return ws.numel() * ws.element_size()
+
+
 def workspace_size(kind: str, B, Hq, Hkv, Hm, Nq, Nk, d) -> int:
     lib = load_library()
     dm = _dims(B, Hq, Hkv, Hm, Nq, Nk, d)
@@ -125,21 +176,23 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, lts=None, lte=None, u
         workspace: Optional[torch.Tensor] = None):
     """Masked attention forward -> (o [B,Nq,Hq,d] bf16, lse [B,Hq,Nq] fp32)."""
     lib = load_library()
-    for n, t in (("q", q), ("k", k), ("v", v)):
-        _need_cuda(n, t, torch.bfloat16)
-    B, Nq, Hq, d = q.shape
-    Nk, Hkv = k.shape[1], k.shape[2]
-    vecs, Hm = _masks(lts, lte, uts, ute)
-    dm = _dims(B, Hq, Hkv, Hm, Nq, Nk, d)
+    B, Nq, Hq, d, Nk, Hkv = _qkv_shapes(q, k, v)
+    Hm = _mask_shapes(lts, lte, uts, ute, B, Nk)
+    vecs = [lts, lte, uts, ute]
+    if out is not None:
+        o, lse = out
+        _shaped("o", o, (B, Nq, Hq, d), torch.bfloat16)
+        _shaped("lse", lse, (B, Hq, Nq), torch.float32)
+    _on_device(q.device, [("q", q), ("k", k), ("v", v)] + list(zip(("lts", "lte", "uts", "ute"), vecs)))
     if out is None:
         o = torch.empty_like(q)
         lse = torch.empty(B, Hq, Nq, dtype=torch.float32, device=q.device)
-    else:
-        o, lse = out
+    dm = _dims(B, Hq, Hkv, Hm, Nq, Nk, d)
     need = int(lib.flashmask_fwd_workspace_size(ctypes.byref(dm)))
     ws = workspace if workspace is not None else _workspace(need, q.device)
+    _on_device(q.device, [("o", o), ("lse", lse), ("workspace", ws)])
     rc = lib.flashmask_fwd(_ptr(q), _ptr(k), _ptr(v), *[_ptr(x) for x in vecs], ctypes.c_float(scale or 0.0),
-                           ctypes.byref(dm), _ptr(o), _ptr(lse), _ptr(ws), ctypes.c_size_t(ws.numel()),
+                           ctypes.byref(dm), _ptr(o), _ptr(lse), _ptr(ws), ctypes.c_size_t(_ws_bytes(ws)),
                            _stream(q.device))
     _check(rc, "flashmask_fwd")
     return o, lse
@@ -150,22 +203,28 @@ def bwd(q, k, v, o, lse, dout, lts=None, lte=None, uts=None, ute=None, scale: Op
         workspace: Optional[torch.Tensor] = None):
     """Masked attention backward of sum(O * dO) -> (dq, dk, dv), bf16."""
     lib = load_library()
-    for n, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout)):
-        _need_cuda(n, t, torch.bfloat16)
-    _need_cuda("lse", lse, torch.float32)
-    B, Nq, Hq, d = q.shape
-    Nk, Hkv = k.shape[1], k.shape[2]
-    vecs, Hm = _masks(lts, lte, uts, ute)
-    dm = _dims(B, Hq, Hkv, Hm, Nq, Nk, d)
+    B, Nq, Hq, d, Nk, Hkv = _qkv_shapes(q, k, v)
+    _shaped("o", o, (B, Nq, Hq, d), torch.bfloat16)
+    _shaped("dout", dout, (B, Nq, Hq, d), torch.bfloat16)
+    _shaped("lse", lse, (B, Hq, Nq), torch.float32)
+    Hm = _mask_shapes(lts, lte, uts, ute, B, Nk)
+    vecs = [lts, lte, uts, ute]
+    if out is not None:
+        dq, dk, dv = out
+        _shaped("dq", dq, (B, Nq, Hq, d), torch.bfloat16)
+        _shaped("dk", dk, (B, Nk, Hkv, d), torch.bfloat16)
+        _shaped("dv", dv, (B, Nk, Hkv, d), torch.bfloat16)
+    _on_device(q.device, [("q", q), ("k", k), ("v", v), ("o", o), ("lse", lse), ("dout", dout)]
+               + list(zip(("lts", "lte", "uts", "ute"), vecs)))
     if out is None:
         dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    else:
-        dq, dk, dv = out
+    dm = _dims(B, Hq, Hkv, Hm, Nq, Nk, d)
     need = int(lib.flashmask_bwd_workspace_size(ctypes.byref(dm)))
     ws = workspace if workspace is not None else _workspace(need, q.device)
+    _on_device(q.device, [("dq", dq), ("dk", dk), ("dv", dv), ("workspace", ws)])
     rc = lib.flashmask_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout), *[_ptr(x) for x in vecs],
                            ctypes.c_float(scale or 0.0), ctypes.byref(dm), _ptr(dq), _ptr(dk), _ptr(dv), _ptr(ws),
-                           ctypes.c_size_t(ws.numel()), _stream(q.device))
+                           ctypes.c_size_t(_ws_bytes(ws)), _stream(q.device))
     _check(rc, "flashmask_bwd")
     return dq, dk, dv
 
