@@ -74,6 +74,21 @@ struct AuxStream {
   cudaEvent_t fork = nullptr, pre = nullptr, plan = nullptr, join = nullptr;
   std::mutex mu;
 };
+// Joins the second stream back to the caller's stream if a call returns early
+// (an error after the fork), so that none of the call's work stays unordered
+// with respect to the caller's later work on its stream.
+struct JoinOnExit {
+  AuxStream* ax = nullptr;
+  cudaStream_t st = nullptr;
+  bool armed = false;
+  ~JoinOnExit() {
+    if (armed) {
+      cudaEventRecord(ax->join, ax->stream);
+      cudaStreamWaitEvent(st, ax->join, 0);
+    }
+  }
+};
+
 AuxStream* aux_stream() {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
@@ -385,6 +400,9 @@ int flashmask_bwd(const void* q, const void* k, const void* v, const void* o, co
   AuxStream* ax = aux_stream();
   std::unique_lock<std::mutex> ax_lock;
   if (ax) ax_lock = std::unique_lock<std::mutex>(ax->mu);
+  JoinOnExit join_guard;  // destroyed before the lock is released
+  join_guard.ax = ax;
+  join_guard.st = st;
   BwdPreParams bp{};
   bp.s = s;
   bp.o = static_cast<const __nv_bfloat16*>(o);
@@ -396,6 +414,7 @@ int flashmask_bwd(const void* q, const void* k, const void* v, const void* o, co
   if (ax) {
     FM_CUDA(cudaEventRecord(ax->fork, st));
     FM_CUDA(cudaStreamWaitEvent(ax->stream, ax->fork, 0));
+    join_guard.armed = true;
     if (has_q) FM_CUDA(launch_bwd_pre(bp, pre_blocks, ax->stream));
     FM_CUDA(cudaEventRecord(ax->pre, ax->stream));
   } else if (has_q) {
@@ -484,6 +503,7 @@ int flashmask_bwd(const void* q, const void* k, const void* v, const void* o, co
     if (grid_q > 0) FM_CUDA(launch_bwd_dq(kp, tq, tk, tv, tdo, grid_q, ax->stream));
     FM_CUDA(cudaEventRecord(ax->join, ax->stream));
     FM_CUDA(cudaStreamWaitEvent(st, ax->join, 0));
+    join_guard.armed = false;
     profile_end(prof, st);
   } else {
     const int prof = profile_begin(3, st);
