@@ -6,7 +6,12 @@ operand, a wrong index), compiles it, routes the oracle through the mutant and
 checks that at least one pin of ``test_oracle_pins.py`` now fails.  A control
 case compiles the unchanged source the same way and checks that the same pins
 pass.  Every planted mistake keeps all memory accesses in bounds.
+
+The head and batch mapping lives in the oracle's Python layer; those mistakes
+are planted in a copy of the module's source, executed as a separate module.
 """
+import types
+
 import pytest
 
 import oracle
@@ -29,6 +34,11 @@ CLASSIFY = [lambda o, s=s: pins.test_classify_sound_random(o, s) for s in range(
 LOCALIZE = [lambda o, s=s: pins.test_localize_reproduces_dense_rows(o, s) for s in range(3)]
 LOCALIZE_MULTI = [lambda o, s=s: pins.test_localize_multi_reproduces_dense_rows(o, s) for s in range(3)]
 COUNT = [lambda o: pins.test_count_unmasked(o)]
+GQA = [
+    lambda o: pins.test_gqa_and_batches_equal_sdpa_with_repeated_kv(o),
+    lambda o: pins.test_gqa_backward_equals_torch_autograd_repeated_kv(o),
+]
+PER_HEAD = [lambda o: pins.test_per_head_masks_equal_sdpa_per_head(o)]
 
 # (name, text in the source, planted replacement, pins expected to catch it)
 MUTATIONS = [
@@ -49,6 +59,41 @@ MUTATIONS = [
     ("localize_multi_first_offset", "acc += x - a[t];", "acc += x - a[0];", LOCALIZE_MULTI),
     ("count_negated", "cnt += !is_masked(", "cnt += is_masked(", COUNT),
 ]
+
+# (name, text in oracle/__init__.py, planted replacement, pins expected to catch it)
+PY_MUTATIONS = [
+    ("kv_head_interleaved", "return (lambda h: h // G), (lambda h: 0 if Hm == 1 else h)",
+     "return (lambda h: h % Hkv), (lambda h: 0 if Hm == 1 else h)", GQA),
+    ("mask_head_always_first", "(lambda h: 0 if Hm == 1 else h)", "(lambda h: 0)", PER_HEAD),
+    ("dkdv_group_interleaved", "for h in range(hk * G, (hk + 1) * G):", "for h in range(hk, Hq, Hkv):", GQA),
+    ("forward_mask_of_first_batch",
+     "vecs = [np.ascontiguousarray(x[b, hm]) for x in m4]\n        if sel is None:\n            qb = _f64(",
+     "vecs = [np.ascontiguousarray(x[0, hm]) for x in m4]\n        if sel is None:\n            qb = _f64(", GQA),
+    ("dq_mask_of_first_batch",
+     "vecs = [np.ascontiguousarray(x[b, hm]) for x in m4]\n        if sel is None:\n            qb, gb,",
+     "vecs = [np.ascontiguousarray(x[0, hm]) for x in m4]\n        if sel is None:\n            qb, gb,", GQA),
+]
+
+
+def _python_source() -> str:
+    with open(oracle.__file__) as f:
+        return f.read()
+
+
+def _python_variant(text: str):
+    """Executes a version of the oracle's Python layer as a module of its own (same C library)."""
+    mod = types.ModuleType("oracle_python_variant")
+    mod.__file__ = oracle.__file__
+    exec(compile(text, oracle.__file__, "exec"), mod.__dict__)
+    return mod
+
+
+def _fails_with(mod, check) -> bool:
+    try:
+        check(mod)
+    except AssertionError:
+        return True
+    return False
 
 
 def _fails(check) -> bool:
@@ -78,4 +123,21 @@ def test_planted_mistake_is_caught(source, tmp_path, name, old, new, checks):
     lib = oracle.build_variant(source.replace(old, new), str(tmp_path))
     with oracle.use_library(lib):
         caught = [i for i, check in enumerate(checks) if _fails(check)]
+    assert caught, f"{name}: no pin caught the planted mistake"
+
+
+def test_control_unchanged_python_layer_passes_its_pins():
+    oracle.build_oracle()
+    mod = _python_variant(_python_source())
+    for check in GQA + PER_HEAD + FWD[:1] + BWD[:1]:
+        assert not _fails_with(mod, check)
+
+
+@pytest.mark.parametrize("name,old,new,checks", PY_MUTATIONS, ids=[m[0] for m in PY_MUTATIONS])
+def test_planted_mapping_mistake_is_caught(name, old, new, checks):
+    oracle.build_oracle()
+    text = _python_source()
+    assert text.count(old) == 1, f"{name}: the text to mutate must occur exactly once"
+    mod = _python_variant(text.replace(old, new))
+    caught = [i for i, check in enumerate(checks) if _fails_with(mod, check)]
     assert caught, f"{name}: no pin caught the planted mistake"

@@ -163,6 +163,49 @@ def test_golden_hand_example(oracle_mod):
     assert np.abs(lse[0, 0] - np.log(np.array(g["visible_count"], np.float64))).max() < 1e-12
 
 
+def test_gqa_and_batches_equal_sdpa_with_repeated_kv(oracle_mod):
+    """Grouped KV heads and batches: torch SDPA per batch on K, V repeated over each group.
+
+    q-head h reads KV head h // (Hq / Hkv) (consecutive q-heads share a KV
+    head); batch b uses its own mask vectors.  The reference expands K and V
+    with np.repeat along the head axis and builds each batch's dense mask here.
+    """
+    rng = np.random.default_rng(9)
+    B, nq, nk, hq, hkv, d = 2, 29, 23, 6, 2, 8
+    per_batch = [wl.random_interval_vectors(rng, nq, nk) for _ in range(B)]
+    vecs = [np.stack([pb[t] for pb in per_batch])[:, None, :] for t in range(4)]
+    q, k, v = rand64(rng, B, nq, hq, d), rand64(rng, B, nk, hkv, d), rand64(rng, B, nk, hkv, d)
+    o, lse = oracle_mod.attention_forward(q, k, v, *vecs, scale=0.4)
+    G = hq // hkv
+    for b in range(B):
+        dense = dense_mask_np(*per_batch[b], nq)
+        ok_rows = ~dense.all(1)
+        assert ok_rows.sum() > nq // 2
+        ref = sdpa64(q[b], np.repeat(k[b], G, axis=1), np.repeat(v[b], G, axis=1), allowed=~dense, scale=0.4)
+        assert np.abs(o[b][ok_rows] - ref[ok_rows]).max() < 1e-12
+        assert np.all(o[b][~ok_rows] == 0.0)
+        assert np.all(np.isneginf(lse[b][:, ~ok_rows]))
+
+
+def test_per_head_masks_equal_sdpa_per_head(oracle_mod):
+    """One mask per q-head (Hm = Hq): head h follows its own vectors, checked head by head."""
+    rng = np.random.default_rng(10)
+    nq, nk, h, d = 31, 27, 3, 8
+    per_head = [wl.random_interval_vectors(rng, nq, nk, p_empty=0.1) for _ in range(h)]
+    vecs = [np.stack([ph[t] for ph in per_head])[None] for t in range(4)]
+    q, k, v = rand64(rng, 1, nq, h, d), rand64(rng, 1, nk, h, d), rand64(rng, 1, nk, h, d)
+    o, lse = oracle_mod.attention_forward(q, k, v, *vecs)
+    distinct = 0
+    for hh in range(h):
+        dense = dense_mask_np(*per_head[hh], nq)
+        distinct += int(not np.array_equal(dense, dense_mask_np(*per_head[0], nq)))
+        ok_rows = ~dense.all(1)
+        ref = sdpa64(q[0][:, hh:hh + 1], k[0][:, hh:hh + 1], v[0][:, hh:hh + 1], allowed=~dense)
+        assert np.abs(o[0][ok_rows, hh] - ref[ok_rows, 0]).max() < 1e-12
+        assert np.all(o[0][~ok_rows, hh] == 0.0) and np.all(np.isneginf(lse[0, hh][~ok_rows]))
+    assert distinct == h - 1  # the heads' masks really differ
+
+
 # ----------------------------------------------------------------------------
 # backward
 # ----------------------------------------------------------------------------
@@ -214,6 +257,29 @@ def test_backward_equals_torch_autograd_sdpa(oracle_mod):
     for a, b in ((dq, q.grad), (dk, k.grad), (dv, v.grad)):
         assert np.abs(a - b.numpy()).max() < 1e-12
     del sdpa_t
+
+
+def test_gqa_backward_equals_torch_autograd_repeated_kv(oracle_mod):
+    """Grouped KV heads and batches in the backward: autograd of float64 SDPA on K, V repeated
+    over each group (repeat_interleave sums the group's gradients into each KV head), with each
+    batch's own causal-document mask as a dense boolean mask."""
+    rng = np.random.default_rng(11)
+    B, n, hq, hkv, d = 2, 26, 4, 2, 8
+    G = hq // hkv
+    docs = [[9, 17], [5, 12, 9]]
+    per_batch = [wl.causal_document_vectors(L) for L in docs]
+    vecs = [np.stack([pb[t] for pb in per_batch])[:, None, :] for t in range(4)]
+    allowed = torch.as_tensor(np.stack([~dense_mask_np(*pb, n) for pb in per_batch]))[:, None]
+    q, k, v = (torch.tensor(rand64(rng, B, n, h, d), requires_grad=True) for h in (hq, hkv, hkv))
+    g = torch.tensor(rand64(rng, B, n, hq, d))
+    kr, vr = (x.repeat_interleave(G, dim=2) for x in (k, v))
+    o = torch.nn.functional.scaled_dot_product_attention(
+        q.permute(0, 2, 1, 3), kr.permute(0, 2, 1, 3), vr.permute(0, 2, 1, 3), attn_mask=allowed,
+        scale=0.5).permute(0, 2, 1, 3)
+    (o * g).sum().backward()
+    dq, dk, dv = oracle_mod.attention_backward(q.detach(), k.detach(), v.detach(), g, *vecs, scale=0.5)
+    for a, b in ((dq, q.grad), (dk, k.grad), (dv, v.grad)):
+        assert np.abs(a - b.numpy()).max() < 1e-12
 
 
 def test_backward_half_squared_norm(oracle_mod):
