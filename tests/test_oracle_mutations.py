@@ -34,6 +34,7 @@ CLASSIFY = [lambda o, s=s: pins.test_classify_sound_random(o, s) for s in range(
 LOCALIZE = [lambda o, s=s: pins.test_localize_reproduces_dense_rows(o, s) for s in range(3)]
 LOCALIZE_MULTI = [lambda o, s=s: pins.test_localize_multi_reproduces_dense_rows(o, s) for s in range(3)]
 COUNT = [lambda o: pins.test_count_unmasked(o)]
+COUNT_HEADS = [lambda o: pins.test_count_unmasked_batches_and_per_head_masks(o)]
 GQA = [
     lambda o: pins.test_gqa_and_batches_equal_sdpa_with_repeated_kv(o),
     lambda o: pins.test_gqa_backward_equals_torch_autograd_repeated_kv(o),
@@ -72,6 +73,10 @@ PY_MUTATIONS = [
     ("dq_mask_of_first_batch",
      "vecs = [np.ascontiguousarray(x[b, hm]) for x in m4]\n        if sel is None:\n            qb, gb,",
      "vecs = [np.ascontiguousarray(x[0, hm]) for x in m4]\n        if sel is None:\n            qb, gb,", GQA),
+    ("count_per_head_masks_broadcast", "total += per_head[0] * Hq if Hm == 1 else sum(per_head)",
+     "total += per_head[0] * Hq", COUNT_HEADS),
+    ("count_last_batch_only", "        total += per_head[0] * Hq if Hm == 1 else sum(per_head)\n",
+     "        total = per_head[0] * Hq if Hm == 1 else sum(per_head)\n", COUNT_HEADS),
 ]
 
 
@@ -129,7 +134,7 @@ def test_planted_mistake_is_caught(source, tmp_path, name, old, new, checks):
 def test_control_unchanged_python_layer_passes_its_pins():
     oracle.build_oracle()
     mod = _python_variant(_python_source())
-    for check in GQA + PER_HEAD + FWD[:1] + BWD[:1]:
+    for check in GQA + PER_HEAD + COUNT_HEADS + FWD[:1] + BWD[:1]:
         assert not _fails_with(mod, check)
 
 

@@ -428,3 +428,17 @@ def test_count_unmasked(oracle_mod):
     lengths = [100, 300, 377]
     got = oracle_mod.count_unmasked(*[x[None, None] for x in wl.causal_document_vectors(lengths)], n, n, 2)
     assert got == 2 * sum(L * (L + 1) // 2 for L in lengths)
+
+
+def test_count_unmasked_batches_and_per_head_masks(oracle_mod):
+    """B = 2 batches with one mask per q-head (Hm = Hq): the count is the sum of every
+    (batch, head) dense count; with Hm = 1 each batch's count is taken Hq times."""
+    rng = np.random.default_rng(12)
+    B, nq, nk, hq = 2, 41, 37, 3
+    per = [[wl.random_interval_vectors(rng, nq, nk) for _ in range(hq)] for _ in range(B)]
+    vecs = [np.stack([np.stack([per[b][h][t] for h in range(hq)]) for b in range(B)]) for t in range(4)]
+    want = sum(int((~dense_mask_np(*per[b][h], nq)).sum()) for b in range(B) for h in range(hq))
+    assert oracle_mod.count_unmasked(*vecs, nq, nk, hq) == want
+    first = [x[:, :1].copy() for x in vecs]
+    want1 = hq * sum(int((~dense_mask_np(*per[b][0], nq)).sum()) for b in range(B))
+    assert oracle_mod.count_unmasked(*first, nq, nk, hq) == want1
