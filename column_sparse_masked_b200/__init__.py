@@ -19,6 +19,7 @@ from __future__ import annotations
 
 from ._binding import (  # noqa: F401
     FlashMaskError,
+    balance_chunks,
     classify,
     count_unmasked,
     flashmask_attention,

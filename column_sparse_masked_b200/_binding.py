@@ -3,7 +3,7 @@ from __future__ import annotations
 
 import ctypes
 import os
-from typing import Optional, Sequence, Tuple
+from typing import List, Optional, Sequence, Tuple
 
 import torch
 
@@ -25,6 +25,7 @@ _SIGS = {
     "flashmask_localize": (ctypes.c_int, [_P, _P, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, _P]),
     "flashmask_localize_multi": (ctypes.c_int, [_P, _P, ctypes.c_int64, _P, _P, ctypes.c_int32, _P]),
     "flashmask_count_unmasked": (ctypes.c_int, [_P, _P, _P, _P, _DIMS, _P, _P]),
+    "flashmask_balance_chunks": (ctypes.c_int, [_P, ctypes.c_int32, ctypes.c_int32, _P, _P]),
     "flashmask_get_timeout_info": (ctypes.c_int, [_P]),
     "flashmask_get_status": (ctypes.c_int, []),
     "flashmask_set_wait_limit_ns": (None, [ctypes.c_int64]),
@@ -280,6 +281,22 @@ def count_unmasked(lts, lte, uts, ute, Nq: int, Hq: int) -> int:
     rc = lib.flashmask_count_unmasked(*[_ptr(x) for x in vecs], ctypes.byref(dm), _ptr(out), _stream(ref.device))
     _check(rc, "flashmask_count_unmasked")
     return int(out.item())
+
+
+def balance_chunks(costs: Sequence[int], parts: int) -> Tuple[List[int], int]:
+    """Splits q-tiles into ``parts`` contiguous chunks with the smallest possible largest cost.
+
+    ``costs`` holds the work of each q-tile (its unmasked pairs); returns ``(bounds, max_cost)``
+    with chunk p = tiles ``[bounds[p], bounds[p + 1])``.  Host computation in the library
+    (``flashmask_balance_chunks``).
+    """
+    lib = load_library()
+    c = (ctypes.c_int64 * max(1, len(costs)))(*[int(x) for x in costs])
+    bounds = (ctypes.c_int32 * (max(0, int(parts)) + 1))()
+    best = ctypes.c_int64(0)
+    rc = lib.flashmask_balance_chunks(c, len(costs), int(parts), bounds, ctypes.byref(best))
+    _check(rc, "flashmask_balance_chunks")
+    return [int(x) for x in bounds], int(best.value)
 
 
 def get_status() -> int:

@@ -186,6 +186,24 @@ int flashmask_localize_multi(const int32_t* in, int32_t* out, int64_t n, const i
 int flashmask_count_unmasked(const int32_t* lts, const int32_t* lte, const int32_t* uts, const int32_t* ute,
                              const flashmask_dims* dims, int64_t* pairs, void* stream);
 
+/*
+ * Sparsity-aware split of a query sequence into `parts` contiguous chunks of
+ * whole q-tiles, one per context-parallel rank.  The same page and section
+ * name a sparsity-aware load balancer (HCC-IPO) without its rule; read here as
+ * making the ranks' unmasked-pair counts as even as possible.  A rank's mask
+ * then follows from the global vectors by flashmask_localize on its chunk.
+ * costs: HOST array of n >= 0 int64 values >= 0, the work of each q-tile (its
+ * unmasked (row, key) pairs over heads and batches).  bounds: HOST array of
+ * parts + 1 int32, filled with 0 = bounds[0] <= ... <= bounds[parts] = n;
+ * chunk p is q-tiles [bounds[p], bounds[p+1]).  The largest chunk cost is the
+ * smallest possible; every chunk is non-empty when n >= parts (otherwise the
+ * first n chunks hold one tile each).  *max_cost (may be NULL) receives that
+ * largest cost.  Pure host computation: no device, no stream.  Returns
+ * FLASHMASK_ERR_INVALID_ARG for parts <= 0, n < 0, NULL arrays, a negative
+ * cost or a total above INT64_MAX / 4.
+ */
+int flashmask_balance_chunks(const int64_t* costs, int32_t n, int32_t parts, int32_t* bounds, int64_t* max_cost);
+
 /* Synchronises the current device, returns its status word (0 or a negative
  * FLASHMASK_ERR_* code written by a kernel) and resets it to 0. */
 int flashmask_get_status(void);

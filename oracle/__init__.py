@@ -25,7 +25,7 @@ import contextlib
 import ctypes
 import os
 import subprocess
-from typing import Optional, Sequence, Tuple
+from typing import List, Optional, Sequence, Tuple
 
 import numpy as np
 
@@ -107,6 +107,8 @@ def _bind(lib):
     lib.oracle_count_unmasked.argtypes = [_I32, _I32, _I32, _I32, ctypes.c_int64, ctypes.c_int64]
     lib.oracle_count_unmasked.restype = ctypes.c_int64
     lib.oracle_mask_row.argtypes = [_I32, _I32, _I32, _I32, ctypes.c_int64, ctypes.c_int64, _U8]
+    lib.oracle_tile_costs.argtypes = [_I32, _I32, _I32, _I32, ctypes.c_int64, ctypes.c_int64, ctypes.c_int64,
+                                      ctypes.POINTER(ctypes.c_int64)]
     lib.oracle_num_threads.restype = ctypes.c_int
     return lib
 
@@ -384,6 +386,52 @@ def count_unmasked(lts, lte, uts, ute, Nq: int, Nk: int, Hq: int) -> int:
             per_head.append(int(lib.oracle_count_unmasked(*[_p(x, _I32) for x in vecs], Nq, Nk)))
         total += per_head[0] * Hq if Hm == 1 else sum(per_head)
     return total
+
+
+def tile_costs(lts, lte, uts, ute, Nq: int, Nk: int, Hq: int, bm: int = 128) -> np.ndarray:
+    """Unmasked (row, key) pairs of each ``bm``-row query tile, summed over batches and all Hq
+    query heads (brute force over the mask predicate): ``int64 [ceil(Nq / bm)]``.
+
+    This is the per-tile work that the load balancer of "FlashMask-3 targets masked distributed
+    attention on Hopper GPUs", section "In-depth insight" (named there, HCC-IPO) evens out
+    across ranks.
+    """
+    lib = _load()
+    B = _i32(lts if lts is not None else uts).shape[0]
+    m4 = _mask_arrays(lts, lte, uts, ute, B, Nk)
+    Hm = m4[0].shape[1]
+    nt = -(-Nq // bm)
+    total = np.zeros(nt, np.int64)
+    one = np.zeros(nt, np.int64)
+    for b in range(B):
+        for hm in range(Hm):
+            vecs = [np.ascontiguousarray(x[b, hm]) for x in m4]
+            lib.oracle_tile_costs(*[_p(x, _I32) for x in vecs], Nq, Nk, bm, one.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)))
+            total += one * (Hq if Hm == 1 else 1)
+    return total
+
+
+def balance_minimax(costs: Sequence[int], parts: int) -> Tuple[int, List[int]]:
+    """Splits tiles 0..n-1 into ``parts`` contiguous (possibly empty) chunks so that the largest
+    chunk cost is as small as possible, by trying every split (small inputs only).
+
+    Returns ``(best, bounds)``: the optimal largest cost and the first optimal split found in
+    lexicographic order of the boundaries (``bounds[0] = 0``, ``bounds[parts] = n``).
+    """
+    import itertools
+
+    c = [int(x) for x in costs]
+    n = len(c)
+    prefix = [0]
+    for x in c:
+        prefix.append(prefix[-1] + x)
+    best, arg = None, None
+    for cuts in itertools.combinations_with_replacement(range(n + 1), parts - 1):
+        bounds = [0, *cuts, n]
+        worst = max(prefix[bounds[p + 1]] - prefix[bounds[p]] for p in range(parts))
+        if best is None or worst < best:
+            best, arg = worst, bounds
+    return best, arg
 
 
 def mask_dense(lts, lte, uts, ute, Nq: int) -> np.ndarray:

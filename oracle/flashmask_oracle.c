@@ -298,6 +298,21 @@ int64_t oracle_count_unmasked(const int32_t* lts, const int32_t* lte, const int3
   return total;
 }
 
+/* Unmasked (i, j) pairs of each bm-row query tile of one (batch, mask head),
+ * by brute force: out[t] counts the pairs of rows [t*bm, min((t+1)*bm, nq)). */
+void oracle_tile_costs(const int32_t* lts, const int32_t* lte, const int32_t* uts, const int32_t* ute, int64_t nq,
+                       int64_t nk, int64_t bm, int64_t* out) {
+  const int64_t nt = (nq + bm - 1) / bm;
+#pragma omp parallel for schedule(static)
+  for (int64_t t = 0; t < nt; ++t) {
+    int64_t cnt = 0;
+    const int64_t r1 = (t + 1) * bm < nq ? (t + 1) * bm : nq;
+    for (int64_t i = t * bm; i < r1; ++i)
+      for (int64_t j = 0; j < nk; ++j) cnt += !is_masked(lts, lte, uts, ute, j, i);
+    out[t] = cnt;
+  }
+}
+
 int oracle_num_threads(void) {
   int n = 1;
 #pragma omp parallel

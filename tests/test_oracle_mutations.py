@@ -15,6 +15,7 @@ import types
 import pytest
 
 import oracle
+import test_balance
 import test_oracle_pins as pins
 
 FWD = [
@@ -34,6 +35,8 @@ CLASSIFY = [lambda o, s=s: pins.test_classify_sound_random(o, s) for s in range(
 LOCALIZE = [lambda o, s=s: pins.test_localize_reproduces_dense_rows(o, s) for s in range(3)]
 LOCALIZE_MULTI = [lambda o, s=s: pins.test_localize_multi_reproduces_dense_rows(o, s) for s in range(3)]
 COUNT = [lambda o: pins.test_count_unmasked(o)]
+TILE_COSTS = [lambda o: test_balance.test_tile_costs_sum_to_pair_count(o),
+              lambda o: test_balance.test_tile_costs_causal_closed_form(o)]
 COUNT_HEADS = [lambda o: pins.test_count_unmasked_batches_and_per_head_masks(o)]
 GQA = [
     lambda o: pins.test_gqa_and_batches_equal_sdpa_with_repeated_kv(o),
@@ -58,7 +61,10 @@ MUTATIONS = [
     ("classify_full_uses_max", "else if ((mn[0] >= r1 ||", "else if ((mx[0] >= r1 ||", CLASSIFY),
     ("localize_shift_off_by_one", "x = x - a;", "x = x - a - 1;", LOCALIZE),
     ("localize_multi_first_offset", "acc += x - a[t];", "acc += x - a[0];", LOCALIZE_MULTI),
-    ("count_negated", "cnt += !is_masked(", "cnt += is_masked(", COUNT),
+    ("count_negated", "cnt += !is_masked(lts, lte, uts, ute, j, i);\n    total += cnt;",
+     "cnt += is_masked(lts, lte, uts, ute, j, i);\n    total += cnt;", COUNT),
+    ("tile_costs_row_past_tile", "for (int64_t i = t * bm; i < r1; ++i)", "for (int64_t i = t * bm; i <= r1; ++i)",
+     TILE_COSTS),
 ]
 
 # (name, text in oracle/__init__.py, planted replacement, pins expected to catch it)
@@ -118,7 +124,7 @@ def source():
 def test_control_unchanged_source_passes_every_pin(source, tmp_path):
     lib = oracle.build_variant(source, str(tmp_path))
     with oracle.use_library(lib):
-        for check in FWD + BWD + CLASSIFY + LOCALIZE + LOCALIZE_MULTI + COUNT:
+        for check in FWD + BWD + CLASSIFY + LOCALIZE + LOCALIZE_MULTI + COUNT + TILE_COSTS:
             assert not _fails(check)
 
 
