@@ -41,7 +41,7 @@ from ._binding import (  # noqa: F401
 )
 
 __all__ = [
-    "FlashMaskError", "classify", "count_unmasked", "flashmask_attention", "fwd", "bwd", "get_status", "get_timeout_info",
+    "FlashMaskError", "balance_chunks", "classify", "count_unmasked", "flashmask_attention", "fwd", "bwd", "get_status", "get_timeout_info",
     "launch_count", "lib_path", "load_library", "localize", "localize_multi", "profiler_enable", "profiler_read", "set_wait_limit_ns", "test_wait_timeout",
     "version", "workspace_size",
 ]
