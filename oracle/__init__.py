@@ -17,7 +17,8 @@ mask vectors ``[B, Hm, Nk]`` int32 with Hm in {1, Hq}; q-head h uses KV head
 ``h // (Hq // Hkv)`` and mask head ``0 if Hm == 1 else h``.
 
 Parity pins: see ``tests/test_oracle_pins.py`` (library special cases, closed
-forms, finite differences, brute force); nothing here is unpinned.
+forms, finite differences, brute force) and, for the per-tile costs and the
+exhaustive chunk split, ``tests/test_balance.py``; nothing here is unpinned.
 """
 from __future__ import annotations
 
