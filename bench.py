@@ -4,19 +4,26 @@
 One step = one forward (``flashmask_fwd``) and one backward (``flashmask_bwd``)
 over one batch of the workload, through the library's C ABI.  Effective FLOPs
 count only unmasked (i, j) pairs: 4*d*pairs forward, 10*d*pairs backward
-(pairs from the library's closed-form count).  The default workload is the
-8K causal-document mask with 32 query / 8 KV heads, head_dim 128.
+(pairs from the library's closed-form count).  The default (headline)
+workload is the largest single-GPU one: the 131072-token causal-document mask
+with 30% of its 128-key tiles dropped, 32 query / 8 KV heads, head_dim 128.
+The 8K document and 32K share-question workloads are timed in the same run
+and reported under "secondary".
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--config NAME]
 
-N > 1 runs under torchrun as independent replicas (one per GPU, no data-path
+N > 1 runs as independent replicas (one process per GPU, no data-path
 collective; the path has no exchange step): value = all ranks' FLOPs / max
-over ranks of the device time.  Rank 0 prints one JSON line.
+over ranks of the device time.  Started without torchrun's environment,
+``--gpus N`` re-launches itself under ``torch.distributed.run`` with N
+processes.  Rank 0 prints one JSON line.
 """
 from __future__ import annotations
 
 import argparse
 import hashlib
+import platform
+import socket
 import json
 import os
 import statistics
@@ -35,21 +42,50 @@ from column_sparse_masked_b200 import workloads as wl  # noqa: E402
 METRIC = "FlashMask fwd+bwd effective TFLOP/s (unmasked FLOPs only), % of B200 bf16 peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 CPU_SAMPLE_ROWS = 8192  # bounded oracle sample: first rows/keys of (batch 0, q-head 0)
+DEFAULT_CONFIG = "docblocksparse128k"
+SECONDARY = ("doc8k", "sharequestion32k")
+SECONDARY_STEPS = 30
 
 
-def parse_args():
+def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=40)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", default="doc8k", choices=wl.CONFIG_ORDER)
+    ap.add_argument("--config", default=DEFAULT_CONFIG, choices=wl.CONFIG_ORDER)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    return ap.parse_args()
+    ap.add_argument("--no-secondary", action="store_true", help="time only the headline workload")
+    return ap.parse_args(argv)
 
 
 def dist_env():
     return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def free_port() -> int:
+    sk = socket.socket()
+    sk.bind(("127.0.0.1", 0))
+    port = sk.getsockname()[1]
+    sk.close()
+    return port
+
+
+def relaunch_command(argv, gpus: int, port: int):
+    """torch.distributed.run command that starts this script once per GPU (replicas)."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={gpus}",
+            "--master-addr", "127.0.0.1", f"--master-port={port}", os.path.abspath(__file__), *argv]
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return platform.processor() or "unknown"
 
 
 def load_peaks():
@@ -207,7 +243,7 @@ def cpu_baseline(w: wl.Workload, rows: int = CPU_SAMPLE_ROWS, inp=None):
         heads += 1
     ff, fb = effective_flops(pairs, w.d)
     return {"value": (ff + fb) / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
-            "seconds": dt,
+            "cpu_model": cpu_model(), "seconds": dt,
             "sample": f"{w.name}: batch 0, q-heads 0..{heads - 1} each with its KV head, first {n} queries x "
                       f"{n} keys (mask localised onto [0,{n})), fp64 fwd+bwd, {pairs} unmasked pairs"}
 
@@ -215,94 +251,134 @@ def cpu_baseline(w: wl.Workload, rows: int = CPU_SAMPLE_ROWS, inp=None):
 # ----------------------------------------------------------------------------
 # our arm
 # ----------------------------------------------------------------------------
-def run_ours(args, rank, world, local_rank):
-    import column_sparse_masked_b200 as fm
+MASK_NAMES = ("lts", "lte", "uts", "ute")
+INPUT_NAMES = ("q", "k", "v", "do") + MASK_NAMES
 
-    dev = torch.device("cuda", local_rank)
-    torch.cuda.set_device(dev)
-    w = wl.CONFIGS[args.config]
+
+def class_histogram(fm, masks, w) -> dict:
+    """Skip / partial / full counts of the (batch, mask head, q-tile, k-tile) tiles."""
+    cls = fm.classify(*masks, Nq=w.N)
+    c = torch.bincount(cls.flatten().long(), minlength=3).tolist()
+    return {"skip": c[0], "partial": c[1], "full": c[2], "tiles": sum(c),
+            "unit": "128x128 (batch, mask head, q-tile, k-tile) tiles"}
+
+
+def setup_problem(fm, w, dev) -> dict:
+    """Pinned host inputs, their device copies, outputs and workspace of one workload."""
     inp = wl.make_inputs(w, with_grad=True)
-    names = ("q", "k", "v", "do", "lts", "lte", "uts", "ute")
-    host = {n: inp[n].pin_memory() for n in names}
-    d_in = {n: host[n].to(dev) for n in names}
-    masks = [d_in[n] for n in ("lts", "lte", "uts", "ute")]
-    pairs = fm.count_unmasked(*masks, Nq=w.N, Hq=w.Hq)
-    f_fwd, f_bwd = effective_flops(pairs, w.d)
-    o = torch.empty_like(d_in["q"])
-    lse = torch.empty(w.B, w.Hq, w.N, dtype=torch.float32, device=dev)
-    dq, dk, dv = torch.empty_like(d_in["q"]), torch.empty_like(d_in["k"]), torch.empty_like(d_in["v"])
-    ws = torch.empty(fm.workspace_size("bwd", w.B, w.Hq, w.Hkv, 1, w.N, w.N, w.d), dtype=torch.uint8, device=dev)
-    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+    host = {n: inp[n].pin_memory() for n in INPUT_NAMES}
+    d_in = {n: host[n].to(dev) for n in INPUT_NAMES}
+    pb = {"w": w, "inp": inp, "host": host, "d_in": d_in,
+          "o": torch.empty_like(d_in["q"]),
+          "lse": torch.empty(w.B, w.Hq, w.N, dtype=torch.float32, device=dev),
+          "dq": torch.empty_like(d_in["q"]), "dk": torch.empty_like(d_in["k"]), "dv": torch.empty_like(d_in["v"]),
+          "ws": torch.empty(fm.workspace_size("bwd", w.B, w.Hq, w.Hkv, 1, w.N, w.N, w.d), dtype=torch.uint8,
+                            device=dev)}
+    pb["pairs"] = fm.count_unmasked(*[d_in[n] for n in MASK_NAMES], Nq=w.N, Hq=w.Hq)
+    return pb
 
-    def step(src):
-        fm.fwd(src["q"], src["k"], src["v"], *[src[n] for n in ("lts", "lte", "uts", "ute")], out=(o, lse),
-               workspace=ws)
-        fm.bwd(src["q"], src["k"], src["v"], o, lse, src["do"], *[src[n] for n in ("lts", "lte", "uts", "ute")],
-               out=(dq, dk, dv), workspace=ws)
 
-    for _ in range(args.warmup):
+def run_step(fm, pb, src):
+    """One step of the hot path: forward then backward, through the library's C ABI."""
+    m = [src[n] for n in MASK_NAMES]
+    fm.fwd(src["q"], src["k"], src["v"], *m, out=(pb["o"], pb["lse"]), workspace=pb["ws"])
+    fm.bwd(src["q"], src["k"], src["v"], pb["o"], pb["lse"], src["do"], *m,
+           out=(pb["dq"], pb["dk"], pb["dv"]), workspace=pb["ws"])
+
+
+def time_device(fm, pb, steps, warmup, flush, world, clocks=None):
+    """Device time of `steps` steps (CUDA events per step, L2 flushed before each step outside the
+    events), with the library's per-kernel profiler on.  Returns (per-step ms, profiler, launches, clocks)."""
+    for _ in range(warmup):
         flush.fill_(1)
-        step(d_in)
+        run_step(fm, pb, pb["d_in"])
     torch.cuda.synchronize()
     assert fm.get_status() == 0, "device status word set during warm-up"
-
-    # ---- device-resident timing ----
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-    vis = [x for x in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if x.strip()]
-    clocks = ClockSampler(vis[local_rank] if local_rank < len(vis) else str(local_rank))
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     barrier(world)
     torch.cuda.synchronize()
     launches0 = fm.launch_count()
     fm.profiler_read()
     fm.profiler_enable(True)
-    clocks.start()
-    for i in range(args.steps):
+    if clocks is not None:
+        clocks.start()
+    for i in range(steps):
         flush.fill_(i & 0xFF)
         evs[i][0].record()
-        step(d_in)
+        run_step(fm, pb, pb["d_in"])
         evs[i][1].record()
     torch.cuda.synchronize()
     barrier(world)
-    clk = clocks.stop()
+    clk = clocks.stop() if clocks is not None else None
     fm.profiler_enable(False)
     prof = fm.profiler_read()
     launches = fm.launch_count() - launches0
-    step_ms = [a.elapsed_time(b) for a, b in evs]
+    assert fm.get_status() == 0, "device status word set during the timed steps"
+    return [a.elapsed_time(b) for a, b in evs], prof, launches, clk
+
+
+def unit_rates(prof, pairs, d, peak):
+    """Effective TFLOP/s and fraction of peak of the forward unit and the backward pair."""
+    out = {}
+    for k, fl in (("fwd", 4.0 * d * pairs), ("bwd_pair", 10.0 * d * pairs)):
+        ms, nl = prof[f"{k}_ms"], prof[f"{k}_launches"]
+        tf = fl / (ms / nl / 1e3) / 1e12 if nl else None
+        out[k] = {"ms_per_launch": ms / nl if nl else None, "tflops": tf, "frac": tf / peak if tf else None}
+    return out
+
+
+def run_ours(args, rank, world, local_rank):
+    import column_sparse_masked_b200 as fm
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    peaks, peak_src = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    w = wl.CONFIGS[args.config]
+    pb = setup_problem(fm, w, dev)
+    pairs = pb["pairs"]
+    f_fwd, f_bwd = effective_flops(pairs, w.d)
+    hist = class_histogram(fm, [pb["d_in"][n] for n in MASK_NAMES], w)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(2 * l2, dtype=torch.uint8, device=dev)
+
+    # ---- device-resident timing ----
+    vis = [x for x in os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",") if x.strip()]
+    clocks = ClockSampler(vis[local_rank] if local_rank < len(vis) else str(local_rank))
+    step_ms, prof, launches, clk = time_device(fm, pb, args.steps, args.warmup, flush, world, clocks)
     local_ms = sum(step_ms)
     value, total_ms = aggregate(local_ms, f_fwd + f_bwd, args.steps, world, dev)
-    assert fm.get_status() == 0, "device status word set during the timed steps"
 
     # ---- end to end: host buffers, copies inside the timed region ----
-    h_out = {"o": torch.empty_like(o, device="cpu").pin_memory(),
-             "lse": torch.empty_like(lse, device="cpu").pin_memory(),
-             "dq": torch.empty_like(dq, device="cpu").pin_memory(),
-             "dk": torch.empty_like(dk, device="cpu").pin_memory(),
-             "dv": torch.empty_like(dv, device="cpu").pin_memory()}
-    d_e2e = {n: torch.empty_like(d_in[n]) for n in names}
+    host = pb["host"]
+    outs = {n: pb[n] for n in ("o", "lse", "dq", "dk", "dv")}
+    h_out = {n: torch.empty_like(t, device="cpu").pin_memory() for n, t in outs.items()}
+    d_e2e = {n: torch.empty_like(pb["d_in"][n]) for n in INPUT_NAMES}
 
     def e2e_step():
-        for n in names:
+        for n in INPUT_NAMES:
             d_e2e[n].copy_(host[n], non_blocking=True)
-        step(d_e2e)
-        for n, t in (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv)):
+        run_step(fm, pb, d_e2e)
+        for n, t in outs.items():
             h_out[n].copy_(t, non_blocking=True)
 
     e2e_step()
     torch.cuda.synchronize()
-    e_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    e2e_steps = min(args.steps, 20)
+    e_evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(e2e_steps)]
     barrier(world)
     torch.cuda.synchronize()
-    for i in range(args.steps):
+    for i in range(e2e_steps):
         flush.fill_(i & 0xFF)
         e_evs[i][0].record()
         e2e_step()
         e_evs[i][1].record()
     torch.cuda.synchronize()
     barrier(world)
-    e2e_value, e2e_ms = aggregate(sum(a.elapsed_time(b) for a, b in e_evs), f_fwd + f_bwd, args.steps, world, dev)
-    h2d = sum(host[n].numel() * host[n].element_size() for n in names)
+    e2e_value, e2e_ms = aggregate(sum(a.elapsed_time(b) for a, b in e_evs), f_fwd + f_bwd, e2e_steps, world, dev)
+    h2d = sum(host[n].numel() * host[n].element_size() for n in INPUT_NAMES)
     d2h = sum(t.numel() * t.element_size() for t in h_out.values())
+    del d_e2e, h_out
 
     # ---- roofline of the dominant unit ----
     # Units: the forward kernel, and the backward's two attention kernels,
@@ -313,7 +389,6 @@ def run_ours(args, rank, world, local_rank):
     # 10*d*pairs.  Executed work per kernel (reported beside it) adds the
     # query side's recomputed S and dP: key side 8*d*pairs, query side
     # 6*d*pairs.
-    peaks, peak_src = load_peaks()
     d = w.d
     units = {"fwd": (("fwd_sm100.cu",), f"fm_fwd_kernel<{d}>", 4.0 * d * pairs),
              "bwd_pair": (("bwd_dkdv_sm100.cu", "bwd_dq_sm100.cu"),
@@ -327,6 +402,7 @@ def run_ours(args, rank, world, local_rank):
         tr = [recorded_traffic(sf, w.name) for sf in srcs]
         per_unit[k] = {"kernel": kname, "ms_per_launch": ms / nl if nl else None, "launches": nl,
                        "tflops": fl / (ms / nl / 1e3) / 1e12 if nl else None, "flops": fl,
+                       "frac": fl / (ms / nl / 1e3) / 1e12 / peak if nl else None,
                        "traffic": (sum(tr) if all(t is not None for t in tr) else None)}
     per_kernel = {}
     for k, (kname, fl) in executed.items():
@@ -336,7 +412,6 @@ def run_ours(args, rank, world, local_rank):
                          "note": "runs concurrently with the other backward kernel" if k != "fwd" else ""}
     dom = max(per_unit, key=lambda k: prof[f"{k}_ms"])
     pk = per_unit[dom]
-    peak = float(peaks["bf16_tflops"])
     roof = {"bound": "tensor", "achieved": pk["tflops"], "peak": peak, "unit": "TFLOP/s",
             "frac": (pk["tflops"] / peak) if pk["tflops"] else None,
             "traffic": pk["traffic"], "kernel": pk["kernel"],
@@ -352,17 +427,37 @@ def run_ours(args, rank, world, local_rank):
         "pct_of_bf16_peak": 100.0 * value / world / peak,
         "config": {"workload": w.name, "description": w.description, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv,
                    "seqlen": w.N, "head_dim": w.d, "unmasked_pairs": pairs,
-                   "flops_per_step": {"fwd": f_fwd, "bwd": f_bwd},
+                   "flops_per_step": {"fwd": f_fwd, "bwd": f_bwd}, "tile_classes": hist,
                    "l2": "flushed before every step (2x L2 bytes written, outside the step's events)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
-        "e2e": {"value": e2e_value, "unit": "TFLOP/s",
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.steps},
+        "e2e": {"value": e2e_value, "unit": "TFLOP/s", "steps": e2e_steps,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / e2e_steps},
         "roofline": roof,
         "gpu_launches": launches,
         "clocks": clk,
     }
+    cpu_inp = pb["inp"]
+    del pb
+
+    # ---- the other document / share-question workloads, same run (not the headline) ----
+    if not args.no_secondary:
+        sec = {}
+        for name in SECONDARY:
+            if name == w.name:
+                continue
+            ws_ = wl.CONFIGS[name]
+            sp = setup_problem(fm, ws_, dev)
+            sms, sprof, _, _ = time_device(fm, sp, SECONDARY_STEPS, args.warmup, flush, world)
+            sff, sfb = effective_flops(sp["pairs"], ws_.d)
+            sec[name] = {"value": (sff + sfb) / (sum(sms) / len(sms) / 1e3) / 1e12, "unit": "TFLOP/s",
+                         "steps": SECONDARY_STEPS, "unmasked_pairs": sp["pairs"],
+                         "tile_classes": class_histogram(fm, [sp["d_in"][n] for n in MASK_NAMES], ws_),
+                         "units": unit_rates(sprof, sp["pairs"], ws_.d, peak)}
+            del sp
+            torch.cuda.empty_cache()
+        line["secondary"] = sec
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, inp=inp)
+        line["cpu_baseline"] = cpu_baseline(w, inp=cpu_inp)
     return line
 
 
@@ -389,13 +484,18 @@ def run_reference(args, rank, world):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": w.name, "sample_rows": n, "unmasked_pairs_per_step": pairs},
         "cpu_baseline": {"value": v, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
-                         "sample": desc},
+                         "cpu_model": cpu_model(), "sample": desc},
         "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
 
 def main():
     args = parse_args()
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # one process per GPU: start the replicas under torch.distributed.run
+        cmd = relaunch_command(sys.argv[1:], args.gpus, free_port())
+        sys.stdout.flush()
+        os.execv(cmd[0], cmd)
     rank, world, local_rank = dist_env()
     if world > 1 and args.impl == "ours":
         from datetime import timedelta

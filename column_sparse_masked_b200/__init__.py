@@ -34,14 +34,16 @@ from ._binding import (  # noqa: F401
     localize_multi,
     profiler_enable,
     profiler_read,
+    set_max_ctas,
     set_wait_limit_ns,
     test_wait_timeout,
+    tile_costs,
     version,
     workspace_size,
 )
 
 __all__ = [
     "FlashMaskError", "balance_chunks", "classify", "count_unmasked", "flashmask_attention", "fwd", "bwd", "get_status", "get_timeout_info",
-    "launch_count", "lib_path", "load_library", "localize", "localize_multi", "profiler_enable", "profiler_read", "set_wait_limit_ns", "test_wait_timeout",
+    "launch_count", "lib_path", "load_library", "localize", "localize_multi", "profiler_enable", "profiler_read", "set_max_ctas", "set_wait_limit_ns", "test_wait_timeout", "tile_costs",
     "version", "workspace_size",
 ]

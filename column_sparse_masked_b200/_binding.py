@@ -25,7 +25,9 @@ _SIGS = {
     "flashmask_localize": (ctypes.c_int, [_P, _P, ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, _P]),
     "flashmask_localize_multi": (ctypes.c_int, [_P, _P, ctypes.c_int64, _P, _P, ctypes.c_int32, _P]),
     "flashmask_count_unmasked": (ctypes.c_int, [_P, _P, _P, _P, _DIMS, _P, _P]),
+    "flashmask_tile_costs": (ctypes.c_int, [_P, _P, _P, _P, _DIMS, _P, _P]),
     "flashmask_balance_chunks": (ctypes.c_int, [_P, ctypes.c_int32, ctypes.c_int32, _P, _P]),
+    "flashmask_set_max_ctas": (ctypes.c_int, [ctypes.c_int32]),
     "flashmask_get_timeout_info": (ctypes.c_int, [_P]),
     "flashmask_get_status": (ctypes.c_int, []),
     "flashmask_set_wait_limit_ns": (None, [ctypes.c_int64]),
@@ -281,6 +283,24 @@ def count_unmasked(lts, lte, uts, ute, Nq: int, Hq: int) -> int:
     rc = lib.flashmask_count_unmasked(*[_ptr(x) for x in vecs], ctypes.byref(dm), _ptr(out), _stream(ref.device))
     _check(rc, "flashmask_count_unmasked")
     return int(out.item())
+
+
+def tile_costs(lts, lte, uts, ute, Nq: int, Hq: int) -> torch.Tensor:
+    """Unmasked pairs of each 128-row q-tile over batches and Hq query heads (int64 CUDA tensor)."""
+    lib = load_library()
+    vecs, Hm = _masks(lts, lte, uts, ute)
+    ref = next(x for x in vecs if x is not None)
+    B, Nk = ref.shape[0], ref.shape[2]
+    dm = _dims(B, Hq, 1, Hm, Nq, Nk, 128)
+    out = torch.zeros(max(1, -(-int(Nq) // 128)), dtype=torch.int64, device=ref.device)
+    rc = lib.flashmask_tile_costs(*[_ptr(x) for x in vecs], ctypes.byref(dm), _ptr(out), _stream(ref.device))
+    _check(rc, "flashmask_tile_costs")
+    return out[: -(-int(Nq) // 128)]
+
+
+def set_max_ctas(n: int) -> None:
+    """Caps the attention kernels' persistent grid at n CTAs (0 = one per SM); for tests."""
+    _check(load_library().flashmask_set_max_ctas(int(n)), "flashmask_set_max_ctas")
 
 
 def balance_chunks(costs: Sequence[int], parts: int) -> Tuple[List[int], int]:

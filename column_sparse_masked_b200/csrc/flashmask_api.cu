@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <atomic>
 #include <climits>
@@ -30,6 +31,23 @@ __device__ int g_status_word[8];
 namespace {
 
 std::atomic<int64_t> g_wait_limit_ns{2000000000LL};
+std::atomic<int> g_max_ctas{0};  // 0: one persistent CTA per SM
+
+// Persistent grid of an attention kernel: one CTA per SM, at most one per
+// work item, at most the process-wide cap when one is set.
+int persistent_grid(int64_t n_items, int sm_count) {
+  int64_t g = n_items < sm_count ? n_items : sm_count;
+  const int cap = g_max_ctas.load(std::memory_order_relaxed);
+  if (cap > 0 && g > cap) g = cap;
+  return (int)g;
+}
+
+// NVTX range around an entry point (visible in a profiler's timeline; a no-op
+// when no tool is attached).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+};
 thread_local char g_last_cuda_error[256] = "";
 std::mutex g_mu;
 
@@ -292,6 +310,7 @@ size_t flashmask_bwd_workspace_size(const flashmask_dims* d) {
 int flashmask_fwd(const void* q, const void* k, const void* v, const int32_t* lts, const int32_t* lte,
                   const int32_t* uts, const int32_t* ute, float scale, const flashmask_dims* dims, void* o,
                   float* lse, void* workspace, size_t workspace_bytes, void* stream) {
+  NvtxRange nvtx("flashmask_fwd");
   FM_TRY(check_dims(dims));
   FM_TRY(check_masks(lts, lte, uts, ute));
   const flashmask_dims& d = *dims;
@@ -352,7 +371,7 @@ int flashmask_fwd(const void* q, const void* k, const void* v, const int32_t* lt
   fp.lse = lse;
   fp.status = di.status;
   fp.wait_limit_ns = (uint64_t)g_wait_limit_ns.load();
-  const int grid = fp.n_items < di.sm_count ? fp.n_items : di.sm_count;
+  const int grid = persistent_grid(fp.n_items, di.sm_count);
   if (grid > 0) FM_CUDA(launch_fwd(fp, tq, tk, tv, grid, st));
   return FLASHMASK_OK;
 }
@@ -361,6 +380,7 @@ int flashmask_bwd(const void* q, const void* k, const void* v, const void* o, co
                   const int32_t* lts, const int32_t* lte, const int32_t* uts, const int32_t* ute, float scale,
                   const flashmask_dims* dims, void* dq, void* dk, void* dv, void* workspace,
                   size_t workspace_bytes, void* stream) {
+  NvtxRange nvtx("flashmask_bwd");
   FM_TRY(check_dims(dims));
   FM_TRY(check_masks(lts, lte, uts, ute));
   const flashmask_dims& d = *dims;
@@ -488,8 +508,8 @@ int flashmask_bwd(const void* q, const void* k, const void* v, const void* o, co
   kp.dv = static_cast<__nv_bfloat16*>(dv);
   kp.status = di.status;
   kp.wait_limit_ns = (uint64_t)g_wait_limit_ns.load();
-  const int grid_kv = kp.n_items < di.sm_count ? kp.n_items : di.sm_count;
-  const int grid_q = (has_q && kp.n_items2 > 0) ? (kp.n_items2 < di.sm_count ? kp.n_items2 : di.sm_count) : 0;
+  const int grid_kv = persistent_grid(kp.n_items, di.sm_count);
+  const int grid_q = (has_q && kp.n_items2 > 0) ? persistent_grid(kp.n_items2, di.sm_count) : 0;
   // The key-side and query-side kernels are independent (same inputs,
   // disjoint outputs).  The query side runs on the library's second stream
   // and is joined back to the caller's stream, so its CTAs take the SMs that
@@ -517,6 +537,7 @@ int flashmask_bwd(const void* q, const void* k, const void* v, const void* o, co
 int flashmask_classify(const int32_t* lts, const int32_t* lte, const int32_t* uts, const int32_t* ute,
                        const flashmask_dims* dims, uint8_t* cls, void* workspace, size_t workspace_bytes,
                        void* stream) {
+  NvtxRange nvtx("flashmask_classify");
   FM_TRY(check_dims(dims));
   FM_TRY(check_masks(lts, lte, uts, ute));
   const flashmask_dims& d = *dims;
@@ -540,6 +561,7 @@ int flashmask_classify(const int32_t* lts, const int32_t* lte, const int32_t* ut
 }
 
 int flashmask_localize(const int32_t* in, int32_t* out, int64_t n, int32_t a, int32_t b, void* stream) {
+  NvtxRange nvtx("flashmask_localize");
   if (n < 0 || a < 0 || b < a) return FLASHMASK_ERR_INVALID_ARG;
   if (n == 0) return FLASHMASK_OK;
   if (!in || !out) return FLASHMASK_ERR_INVALID_ARG;
@@ -551,6 +573,7 @@ int flashmask_localize(const int32_t* in, int32_t* out, int64_t n, int32_t a, in
 
 int flashmask_localize_multi(const int32_t* in, int32_t* out, int64_t n, const int32_t* starts,
                              const int32_t* ends, int32_t nchunks, void* stream) {
+  NvtxRange nvtx("flashmask_localize_multi");
   if (n < 0 || nchunks < 0 || nchunks > 64) return FLASHMASK_ERR_INVALID_ARG;
   if (nchunks > 0 && (!starts || !ends)) return FLASHMASK_ERR_INVALID_ARG;
   for (int c = 0; c < nchunks; ++c) {
@@ -567,6 +590,7 @@ int flashmask_localize_multi(const int32_t* in, int32_t* out, int64_t n, const i
 
 int flashmask_count_unmasked(const int32_t* lts, const int32_t* lte, const int32_t* uts, const int32_t* ute,
                              const flashmask_dims* dims, int64_t* pairs, void* stream) {
+  NvtxRange nvtx("flashmask_count_unmasked");
   FM_TRY(check_dims(dims));
   FM_TRY(check_masks(lts, lte, uts, ute));
   if (!pairs) return FLASHMASK_ERR_INVALID_ARG;
@@ -577,6 +601,30 @@ int flashmask_count_unmasked(const int32_t* lts, const int32_t* lte, const int32
   mp.lts = lts; mp.lte = lte; mp.uts = uts; mp.ute = ute;
   mp.B = d.B; mp.Hm = d.Hm; mp.Nk = d.Nk;
   FM_CUDA(launch_count_unmasked(mp, d.Hq, d.Nq, pairs, static_cast<cudaStream_t>(stream)));
+  return FLASHMASK_OK;
+}
+
+int flashmask_tile_costs(const int32_t* lts, const int32_t* lte, const int32_t* uts, const int32_t* ute,
+                         const flashmask_dims* dims, int64_t* costs, void* stream) {
+  NvtxRange nvtx("flashmask_tile_costs");
+  FM_TRY(check_dims(dims));
+  FM_TRY(check_masks(lts, lte, uts, ute));
+  const flashmask_dims& d = *dims;
+  if (d.Nq == 0) return FLASHMASK_OK;
+  if (!costs) return FLASHMASK_ERR_INVALID_ARG;
+  if (!aligned16(costs)) return FLASHMASK_ERR_ALIGN;
+  DeviceInfo di;
+  FM_TRY(current_device(&di));
+  MaskPrepParams mp{};
+  mp.lts = lts; mp.lte = lte; mp.uts = uts; mp.ute = ute;
+  mp.B = d.B; mp.Hm = d.Hm; mp.Nk = d.Nk;
+  FM_CUDA(launch_tile_costs(mp, d.Hq, d.Nq, costs, static_cast<cudaStream_t>(stream)));
+  return FLASHMASK_OK;
+}
+
+int flashmask_set_max_ctas(int32_t n) {
+  if (n < 0) return FLASHMASK_ERR_INVALID_ARG;
+  g_max_ctas.store(n);
   return FLASHMASK_OK;
 }
 

@@ -21,6 +21,8 @@ cudaError_t launch_localize(const int32_t* in, int32_t* out, int64_t n, int32_t 
 cudaError_t launch_localize_multi(const int32_t* in, int32_t* out, int64_t n, const int32_t* starts,
                                   const int32_t* ends, int nchunks, cudaStream_t st);
 cudaError_t launch_count_unmasked(const MaskPrepParams& p, int Hq, int Nq, int64_t* out, cudaStream_t st);
+// Unmasked pairs of each 128-row q-tile over batches and Hq q-heads: out[ceil(Nq/128)].
+cudaError_t launch_tile_costs(const MaskPrepParams& p, int Hq, int Nq, int64_t* out, cudaStream_t st);
 cudaError_t launch_wait_timeout(int* status, uint64_t limit_ns, cudaStream_t st);
 
 // Forward / backward attention kernels.  `grid` is the persistent CTA count.

@@ -397,6 +397,36 @@ __global__ void __launch_bounds__(1024) count_unmasked_kernel(MaskPrepParams p, 
 }
 
 // ----------------------------------------------------------------------------
+// 5b. unmasked pairs of each 128-row q-tile (the work a sparsity-aware chunk
+//     split evens out), one CTA per q-tile, same closed form restricted to the
+//     tile's rows [r0, r1):  unmasked_j = (r1 - r0) - |L n R| - |U n R| + |L n U n R|
+// ----------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) tile_costs_kernel(MaskPrepParams p, int Hq, int Nq, int64_t* out) {
+  const int qt = blockIdx.x;
+  const int64_t r0 = (int64_t)qt * kTile, r1 = min(r0 + kTile, (int64_t)Nq);
+  const int64_t total = (int64_t)p.B * p.Hm * p.Nk;
+  const int64_t weight = (p.Hm == 1) ? Hq : 1;
+  unsigned long long acc = 0;
+  for (int64_t t = threadIdx.x; t < total; t += blockDim.x) {
+    const int64_t lts = p.lts ? p.lts[t] : 0, lte = p.lte ? p.lte[t] : 0;
+    const int64_t uts = p.uts ? p.uts[t] : 0, ute = p.ute ? p.ute[t] : 0;
+    const int64_t mL = overlap_len(lts, lte, r0, r1);
+    const int64_t mU = overlap_len(uts, ute, r0, r1);
+    const int64_t mLU = overlap_len(max(lts, uts), min(lte, ute), r0, r1);
+    acc += (unsigned long long)((r1 - r0 - (mL + mU - mLU)) * weight);
+  }
+  __shared__ unsigned long long red[8];
+  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = acc;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    unsigned long long s = 0;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) s += red[w];
+    out[qt] = (int64_t)s;
+  }
+}
+
+// ----------------------------------------------------------------------------
 // 6. bounded-wait self test: waits on a barrier that nothing arrives on
 // ----------------------------------------------------------------------------
 __global__ void wait_timeout_kernel(int* status, uint64_t limit_ns) {
@@ -512,6 +542,14 @@ cudaError_t launch_localize_multi(const int32_t* in, int32_t* out, int64_t n, co
 
 cudaError_t launch_count_unmasked(const MaskPrepParams& p, int Hq, int Nq, int64_t* out, cudaStream_t st) {
   { note_launch(); count_unmasked_kernel<<<1, 1024, 0, st>>>(p, Hq, Nq, out);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_tile_costs(const MaskPrepParams& p, int Hq, int Nq, int64_t* out, cudaStream_t st) {
+  const int nqt = (Nq + kTile - 1) / kTile;
+  if (nqt == 0) return cudaSuccess;
+  { note_launch(); tile_costs_kernel<<<nqt, 256, 0, st>>>(p, Hq, Nq, out);
   }
   return cudaGetLastError();
 }

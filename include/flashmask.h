@@ -187,6 +187,19 @@ int flashmask_count_unmasked(const int32_t* lts, const int32_t* lte, const int32
                              const flashmask_dims* dims, int64_t* pairs, void* stream);
 
 /*
+ * Work of each 128-row query tile: costs[t] (device int64, ceil(Nq/128)
+ * entries, 16-byte aligned) receives the number of unmasked (i, j) pairs with
+ * row i in [128 t, min(128 t + 128, Nq)), over all batches, all Hq query heads
+ * and all Nk key columns (closed form per key column restricted to the tile's
+ * rows, one CTA per q-tile).  These are the per-tile loads that
+ * flashmask_balance_chunks evens out across context-parallel ranks (same page
+ * and section: the sparsity-aware load balancer).  Uses dims->B, Hq, Hm, Nq,
+ * Nk (Hkv and d are only checked).  Errors as flashmask_count_unmasked.
+ */
+int flashmask_tile_costs(const int32_t* lts, const int32_t* lte, const int32_t* uts, const int32_t* ute,
+                         const flashmask_dims* dims, int64_t* costs, void* stream);
+
+/*
  * Sparsity-aware split of a query sequence into `parts` contiguous chunks of
  * whole q-tiles, one per context-parallel rank.  The same page and section
  * name a sparsity-aware load balancer (HCC-IPO) without its rule; read here as
@@ -221,6 +234,15 @@ int flashmask_get_timeout_info(int32_t* info);
 /* Sets the limit of every bounded device-side wait, in nanoseconds (default
  * 2e9).  Values <= 0 restore the default.  Host-side setting, process-wide. */
 void flashmask_set_wait_limit_ns(int64_t ns);
+
+/* Caps the persistent grid of the attention kernels at n CTAs (0, the
+ * default, restores one CTA per SM).  With a small cap one CTA walks many
+ * work items in a row, so tests can drive every item-to-item hand-over of the
+ * persistent kernels (ring wrap-round, buffer hand-over, phase flips) on
+ * problems small enough to check element by element.  Results do not depend
+ * on the cap.  Host-side setting, process-wide; FLASHMASK_ERR_INVALID_ARG
+ * for n < 0. */
+int flashmask_set_max_ctas(int32_t n);
 
 /* Launches one CTA whose only job is a bounded wait on a barrier that nothing
  * arrives on; the wait gives up after `limit_ns` and records

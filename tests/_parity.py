@@ -2,7 +2,15 @@
 
 Tolerances: max |err| <= 2e-2 for O, dQ, dK, dV and <= 1e-3 for LSE (natural
 log units); -inf LSE (row with no visible key) must match -inf exactly.
+
+Every comparison also records its plain max |err| (and the max over the
+elements with |ref| <= 5, where the plain 2e-2 bound is asserted as stated);
+when FLASHMASK_PARITY_RECORD names a file, the records of the session are
+written there as JSON lines.
 """
+import json
+import os
+
 import numpy as np
 import torch
 
@@ -53,13 +61,14 @@ def max_err(gpu: torch.Tensor, ref: np.ndarray) -> float:
     return float(np.abs(g - ref).max()) if g.size else 0.0
 
 
-def check_lse(gpu: torch.Tensor, ref: np.ndarray, tol=TOL_LSE):
+def check_lse(gpu: torch.Tensor, ref: np.ndarray, tol=TOL_LSE, case=""):
     g = gpu.detach().cpu().numpy().astype(np.float64)
     ninf_g, ninf_r = np.isneginf(g), np.isneginf(ref)
     assert np.array_equal(ninf_g, ninf_r), f"-inf pattern differs at {np.argwhere(ninf_g != ninf_r)[:5]}"
     fin = ~ninf_r
     err = float(np.abs(g[fin] - ref[fin]).max()) if fin.any() else 0.0
     assert err <= tol, f"LSE max err {err}"
+    record({"case": case, "name": "LSE", "max_err": err, "n": int(g.size)})
     return err
 
 
@@ -68,8 +77,21 @@ def check_lse(gpu: torch.Tensor, ref: np.ndarray, tol=TOL_LSE):
 BF16_HALF_ULP_REL = 2.0 ** -8
 
 
-def check_out(name, gpu, ref, tol=TOL_OUT):
-    """Elementwise |gpu - ref| <= tol + 2^-8 |ref|; returns the plain max |err|."""
+# Below this magnitude bf16 output rounding (half an ulp <= 2^-6) leaves room
+# for the plain bound; there the stated 2e-2 is asserted as it stands.
+PLAIN_REF_MAX = 5.0
+
+
+def record(entry: dict):
+    path = os.environ.get("FLASHMASK_PARITY_RECORD")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps(entry) + "\n")
+
+
+def check_out(name, gpu, ref, tol=TOL_OUT, case=""):
+    """Elementwise |gpu - ref| <= tol + 2^-8 |ref|, and the plain |gpu - ref| <= tol wherever
+    |ref| <= 5; returns the plain max |err|."""
     g = gpu.detach().float().cpu().numpy().astype(np.float64)
     assert np.isfinite(g).all(), f"{name} has non-finite values"
     err = np.abs(g - ref)
@@ -77,4 +99,10 @@ def check_out(name, gpu, ref, tol=TOL_OUT):
     worst = np.unravel_index(np.argmax(err - bound), err.shape) if err.size else None
     assert err.size == 0 or (err <= bound).all(), \
         f"{name} err {err[worst]:.4g} > bound {bound[worst]:.4g} at {worst} (ref {ref[worst]:.4g}); max err {err.max():.4g}"
-    return float(err.max()) if err.size else 0.0
+    small = np.abs(ref) <= PLAIN_REF_MAX
+    plain = float(err[small].max()) if small.any() else 0.0
+    assert plain <= tol, f"{name}: plain max |err| {plain:.4g} > {tol} among elements with |ref| <= {PLAIN_REF_MAX}"
+    mx = float(err.max()) if err.size else 0.0
+    record({"case": case, "name": name, "max_err": mx, "max_err_ref_le_5": plain, "n": int(err.size),
+            "max_abs_ref": float(np.abs(ref).max()) if err.size else 0.0})
+    return mx

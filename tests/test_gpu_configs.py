@@ -60,17 +60,30 @@ def rows_with_visible_key(vecs, nq):
     return (nk - np.cumsum(hidden)[:nq]) > 0
 
 
-def pick_columns(vecs, nq, hkv_count, seed, n_cheap=4, n_rand=4, max_rows=2048):
+def pick_columns(vecs, nq, hkv_count, seed, n_cheap=3, n_rand=3, max_rows=2048, extra=()):
+    """Key columns for the sampled dK/dV check, spread over the whole range of visible-row counts:
+    the column the most rows see (the first key of the longest document, the last prefix key),
+    columns at 3/4, 1/2 and 1/4 of that count which the same rows see (the heaviest column's
+    neighbours to its right), the cheapest columns, random columns seen by <= max_rows rows,
+    `extra` columns, and a column no row sees (dK = dV = 0)."""
     cnt = visible_counts(vecs, nq)
     rng = np.random.default_rng(seed)
+    heavy = int(np.argmax(cnt))
+    cols = {heavy}
+    for frac in (0.75, 0.5, 0.25):  # long-range accumulation over many q-tiles, same rows as `heavy`
+        right = np.nonzero((np.arange(cnt.size) > heavy) & (cnt > 0) & (cnt <= frac * cnt[heavy]))[0]
+        if right.size:
+            cols.add(int(right[0]))
     ok = np.nonzero((cnt > 0) & (cnt <= max_rows))[0]
-    cheap = ok[np.argsort(cnt[ok], kind="stable")[:n_cheap]]
-    rand = rng.choice(ok, size=min(n_rand, ok.size), replace=False) if ok.size else []
-    cols = sorted(set(int(x) for x in cheap) | set(int(x) for x in rand))
+    cols |= set(int(x) for x in ok[np.argsort(cnt[ok], kind="stable")[:n_cheap]])
+    if ok.size:
+        cols |= set(int(x) for x in rng.choice(ok, size=min(n_rand, ok.size), replace=False))
+    cols |= set(int(j) for j in extra)
+    cols = sorted(cols)
     none = np.nonzero(cnt == 0)[0]
     if none.size:
         cols.append(int(none[0]))  # a column no row sees: dK = dV = 0
-    return [(0, int(rng.integers(0, hkv_count)), j) for j in cols]
+    return [(0, int(rng.integers(0, hkv_count)), j) for j in cols], cnt
 
 
 def run_full(w, inp):
@@ -89,12 +102,12 @@ def test_tiny_doc_all_outputs(oracle_mod):
     dev, m, o, lse, dq, dk, dv = run_full(w, inp)
     masks = [inp[n] for n in ("lts", "lte", "uts", "ute")]
     ro, rl = oracle_mod.attention_forward(inp["q"], inp["k"], inp["v"], *masks)
-    check_out("O", o, ro)
-    check_lse(lse, rl)
+    check_out("O", o, ro, case="tiny_doc")
+    check_lse(lse, rl, case="tiny_doc")
     rdq, rdk, rdv = oracle_mod.attention_backward(inp["q"], inp["k"], inp["v"], inp["do"], *masks)
-    check_out("dQ", dq, rdq)
-    check_out("dK", dk, rdk)
-    check_out("dV", dv, rdv)
+    check_out("dQ", dq, rdq, case="tiny_doc")
+    check_out("dK", dk, rdk, case="tiny_doc")
+    check_out("dV", dv, rdv, case="tiny_doc")
 
 
 def _identity_checks(w, inp, dk, dv):
@@ -125,16 +138,18 @@ def test_config_sampled_parity(oracle_mod, name):
     go = torch.stack([o[b, i, h] for b, h, i in rows])
     gl = torch.stack([lse[b, h, i] for b, h, i in rows])
     gdq = torch.stack([dq[b, i, h] for b, h, i in rows])
-    check_out("O(sampled)", go, ro)
-    check_lse(gl, rl)
-    check_out("dQ(sampled)", gdq, rdq)
+    check_out("O(sampled)", go, ro, case=name)
+    check_lse(gl, rl, case=name)
+    check_out("dQ(sampled)", gdq, rdq, case=name)
     vecs0 = [x[0, 0].numpy() for x in masks]
-    cols = pick_columns(vecs0, w.N, w.Hkv, seed=w.seed + 20)
+    extra = (0,) if name == "prefixwindow64k" else ()  # first prefix key: seen by the first 4096 rows
+    cols, cnt = pick_columns(vecs0, w.N, w.Hkv, seed=w.seed + 20, extra=extra)
+    assert max(cnt[j] for _, _, j in cols) == cnt.max()
     rdk, rdv = oracle_mod.attention_backward_dkdv(inp["q"], inp["k"], inp["v"], inp["do"], *masks, samples=cols)
     gdk = torch.stack([dk[b, j, hk] for b, hk, j in cols])
     gdv = torch.stack([dv[b, j, hk] for b, hk, j in cols])
-    check_out("dK(sampled)", gdk, rdk)
-    check_out("dV(sampled)", gdv, rdv)
+    check_out("dK(sampled)", gdk, rdk, case=name)
+    check_out("dV(sampled)", gdv, rdv, case=name)
     _identity_checks(w, inp, dk, dv)
 
     if w.chunks:
@@ -159,3 +174,42 @@ def test_config_sampled_parity(oracle_mod, name):
             err = (s - full.float()).abs()
             bound = 2e-2 + 4 * BF16_HALF_ULP_REL * full.float().abs()
             assert (err <= bound).all(), f"sum over chunks of {nm} vs full run: max err {err.max().item()}"
+
+
+@pytest.mark.parametrize("name", ["doc8k", "docblocksparse128k"])
+def test_zigzag_multichunk_equals_full_run(name):
+    """Multi-chunk localisation ("FlashMask-3 targets masked distributed attention on Hopper GPUs",
+    In-depth insight: exchange-free localisation under any multi-chunk context-parallel assignment).
+    A 4-rank zigzag assignment: rank r holds query chunks [r N/8, (r+1) N/8) and
+    [(7-r) N/8, (8-r) N/8), concatenated in order, with the boundary vectors localised onto the
+    pair.  Against all keys, each rank's O and LSE equal the full run's rows bit for bit (chunk
+    ends are multiples of 256 rows); its dQ rows match within tolerance; the ranks' dK, dV sum to
+    the full run's within tolerance."""
+    w = wl.CONFIGS[name]
+    inp = wl.make_inputs(w)
+    dev, m, o, lse, dq, dk, dv = run_full(w, inp)
+    n8 = w.N // 8
+    assert n8 % 256 == 0
+    dk_sum = torch.zeros_like(dk, dtype=torch.float32)
+    dv_sum = torch.zeros_like(dv, dtype=torch.float32)
+    for r in range(4):
+        chunks = [(r * n8, (r + 1) * n8), ((7 - r) * n8, (8 - r) * n8)]
+        loc = [fm.localize_multi(x, chunks) for x in m]
+        rows = torch.cat([torch.arange(a, b, device="cuda") for a, b in chunks])
+        qc = dev["q"][:, rows].contiguous()
+        doc = dev["do"][:, rows].contiguous()
+        oc, lc = fm.fwd(qc, dev["k"], dev["v"], *loc)
+        assert torch.equal(oc, o[:, rows]), f"rank {r}: O differs from the full run's rows"
+        assert torch.equal(lc, lse[:, :, rows].contiguous()), f"rank {r}: LSE differs"
+        dqc, dkc, dvc = fm.bwd(qc, dev["k"], dev["v"], oc, lc, doc, *loc)
+        ref = dq[:, rows].float()
+        err = (dqc.float() - ref).abs()
+        assert (err <= 2e-2 + BF16_HALF_ULP_REL * ref.abs()).all(), f"rank {r}: dQ max err {err.max().item()}"
+        dk_sum += dkc.float()
+        dv_sum += dvc.float()
+    torch.cuda.synchronize()
+    assert fm.get_status() == 0
+    for nm, s_, full in (("dK", dk_sum, dk), ("dV", dv_sum, dv)):
+        err = (s_ - full.float()).abs()
+        bound = 2e-2 + 4 * BF16_HALF_ULP_REL * full.float().abs()
+        assert (err <= bound).all(), f"sum over zigzag ranks of {nm} vs full run: max err {err.max().item()}"

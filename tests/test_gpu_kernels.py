@@ -51,12 +51,82 @@ def test_forward_backward_parity(oracle_mod, case):
     torch.cuda.synchronize()
     assert fm.get_status() == 0
     ro, rl = oracle_mod.attention_forward(q, k, v, *masks)
-    check_out("O", o, ro)
-    check_lse(lse, rl)
+    cid = _ids(case)
+    check_out("O", o, ro, case=cid)
+    check_lse(lse, rl, case=cid)
     rdq, rdk, rdv = oracle_mod.attention_backward(q, k, v, do, *masks)
-    check_out("dQ", dq, rdq)
-    check_out("dK", dk, rdk)
-    check_out("dV", dv, rdv)
+    check_out("dQ", dq, rdq, case=cid)
+    check_out("dK", dk, rdk, case=cid)
+    check_out("dV", dv, rdv, case=cid)
+
+
+# Cases whose work items outnumber a capped persistent grid many times over:
+# with 1-3 CTAs each CTA walks 5-32 items, so every item-to-item path of the
+# three persistent kernels runs and is compared element by element: the
+# 4-deep item ring wrapping round, the Q/O (Q/dO, K/V) buffer hand-over
+# between items, the accumulator phase flips, zero-work items between real
+# ones and the next item's L2 prefetch.
+CAP_CASES = [
+    (1, 1000, 1000, 4, 2, 1, 128, "doc", 16),      # 16 fwd / 16 key-side / 32 query-side items
+    (1, 2048, 2048, 2, 1, 1, 64, "random", 91),    # d = 64: 16 / 16 / 32 items
+    (2, 517, 389, 4, 2, 1, 128, "random", 14),     # ragged tails, two batches
+    (1, 1100, 1100, 2, 1, 1, 128, "blocksparse", 18),  # zero-work key tiles between real ones
+]
+
+
+@pytest.mark.parametrize("cap", [1, 2, 3])
+@pytest.mark.parametrize("case", CAP_CASES, ids=_ids)
+def test_persistent_walk_parity(oracle_mod, case, cap):
+    q, k, v, do, masks = make_case(*case)
+    qg, kg, vg, dog = cuda(q, k, v, do)
+    mg = cuda(*masks)
+    fm.set_max_ctas(cap)
+    try:
+        o, lse = fm.fwd(qg, kg, vg, *mg)
+        dq, dk, dv = fm.bwd(qg, kg, vg, o, lse, dog, *mg)
+        torch.cuda.synchronize()
+    finally:
+        fm.set_max_ctas(0)
+    assert fm.get_status() == 0
+    cid = f"{_ids(case)}_cap{cap}"
+    ro, rl = oracle_mod.attention_forward(q, k, v, *masks)
+    check_out("O", o, ro, case=cid)
+    check_lse(lse, rl, case=cid)
+    rdq, rdk, rdv = oracle_mod.attention_backward(q, k, v, do, *masks)
+    check_out("dQ", dq, rdq, case=cid)
+    check_out("dK", dk, rdk, case=cid)
+    check_out("dV", dv, rdv, case=cid)
+    # the full grid computes the same bits (results do not depend on the grid)
+    o2, lse2 = fm.fwd(qg, kg, vg, *mg)
+    dq2, dk2, dv2 = fm.bwd(qg, kg, vg, o2, lse2, dog, *mg)
+    assert torch.equal(o, o2) and torch.equal(lse, lse2)
+    assert torch.equal(dq, dq2) and torch.equal(dk, dk2) and torch.equal(dv, dv2)
+
+
+@pytest.mark.parametrize("name", wl.CONFIG_ORDER)
+def test_tile_costs_bit_exact_configs(oracle_mod, name):
+    w = wl.CONFIGS[name]
+    vecs = [torch.from_numpy(x) for x in wl.mask_vectors(w)]
+    got = fm.tile_costs(*cuda(*vecs), Nq=w.N, Hq=w.Hq).cpu().numpy()
+    ref = oracle_mod.tile_costs(*vecs, w.N, w.N, w.Hq)
+    assert got.dtype == np.int64 and np.array_equal(got, ref)
+    assert int(got.sum()) == fm.count_unmasked(*cuda(*vecs), Nq=w.N, Hq=w.Hq)
+
+
+@pytest.mark.parametrize("seed", range(3))
+def test_tile_costs_bit_exact_random(oracle_mod, seed):
+    rng = np.random.default_rng(800 + seed)
+    B, Hq = 2, 3
+    nq, nk = int(rng.integers(1, 1200)), int(rng.integers(1, 900))
+    per = [[wl.random_interval_vectors(rng, nq, nk, p_empty=0.3) for _ in range(Hq)] for _ in range(B)]
+    vecs = [torch.from_numpy(np.ascontiguousarray(np.array([[per[b][h][t] for h in range(Hq)] for b in range(B)],
+                                                           np.int32))) for t in range(4)]
+    got = fm.tile_costs(*cuda(*vecs), Nq=nq, Hq=Hq).cpu().numpy()
+    assert np.array_equal(got, oracle_mod.tile_costs(*vecs, nq, nk, Hq))
+    # the chunk split fed from the library itself
+    bounds, worst = fm.balance_chunks(got.tolist(), 4)
+    best, _ = oracle_mod.balance_minimax(got.tolist(), 4) if got.size <= 12 else (worst, None)
+    assert worst == best
 
 
 def test_forward_is_deterministic():
@@ -106,6 +176,15 @@ def test_classify_bit_exact(oracle_mod, seed):
     got = fm.classify(*cuda(*vecs), Nq=nq).cpu().numpy()
     ref = oracle_mod.classify(*vecs, nq, nk)
     assert np.array_equal(got, ref)
+
+
+def test_classify_golden_clauses_on_gpu():
+    """The hand-derived golden of the tile rule (tests/golden/classify_clauses.json), on the GPU."""
+    from test_oracle_pins import classify_golden
+
+    vecs, nq, expect = classify_golden()
+    got = fm.classify(*cuda(*[torch.from_numpy(x[None, None].copy()) for x in vecs]), Nq=nq).cpu().numpy()
+    assert np.array_equal(got[0, 0], expect), np.argwhere(got[0, 0] != expect)
 
 
 @pytest.mark.parametrize("name", wl.CONFIG_ORDER)

@@ -32,6 +32,7 @@ BWD = [
 CLASSIFY = [lambda o, s=s: pins.test_classify_sound_random(o, s) for s in range(6)] + [
     lambda o: pins.test_classify_causal_closed_form(o),
 ]
+CLASSIFY_GOLDEN = [lambda o: pins.test_classify_golden_clauses(o)]
 LOCALIZE = [lambda o, s=s: pins.test_localize_reproduces_dense_rows(o, s) for s in range(3)]
 LOCALIZE_MULTI = [lambda o, s=s: pins.test_localize_multi_reproduces_dense_rows(o, s) for s in range(3)]
 COUNT = [lambda o: pins.test_count_unmasked(o)]
@@ -59,6 +60,19 @@ MUTATIONS = [
      "D += exp(s[j] - lse[i]) * dot(dout + i * d, k + j * d, d);", BWD),
     ("classify_skip_uses_min", "if ((mx[0] <= r0 && mn[1] >= r1)", "if ((mn[0] <= r0 && mn[1] >= r1)", CLASSIFY),
     ("classify_full_uses_max", "else if ((mn[0] >= r1 ||", "else if ((mx[0] >= r1 ||", CLASSIFY),
+    # conservative slips (sound, so the soundness pins pass them): the golden catches each
+    ("classify_drop_empty_lt", "(mn[0] >= r1 || mx[1] <= r0 || mn[0] >= mx[1])", "(mn[0] >= r1 || mx[1] <= r0)",
+     CLASSIFY_GOLDEN),
+    ("classify_drop_empty_ut", "(mn[2] >= r1 || mx[3] <= r0 || mn[2] >= mx[3])", "(mn[2] >= r1 || mx[3] <= r0)",
+     CLASSIFY_GOLDEN),
+    ("classify_lt_ends_strict", "mx[1] <= r0", "mx[1] < r0", CLASSIFY_GOLDEN),
+    ("classify_ut_ends_strict", "mx[3] <= r0", "mx[3] < r0", CLASSIFY_GOLDEN),
+    ("classify_lt_starts_strict", "(mn[0] >= r1 ||", "(mn[0] > r1 ||", CLASSIFY_GOLDEN),
+    ("classify_ut_starts_strict", "(mn[2] >= r1 ||", "(mn[2] > r1 ||", CLASSIFY_GOLDEN),
+    ("classify_skip_lt_covers_strict", "mx[0] <= r0 && mn[1] >= r1", "mx[0] <= r0 && mn[1] > r1", CLASSIFY_GOLDEN),
+    ("classify_skip_ut_starts_strict", "mx[2] <= r0 && mn[3] >= r1", "mx[2] < r0 && mn[3] >= r1", CLASSIFY_GOLDEN),
+    ("classify_skip_ut_covers_strict", "mx[2] <= r0 && mn[3] >= r1", "mx[2] <= r0 && mn[3] > r1", CLASSIFY_GOLDEN),
+    ("classify_skip_lt_starts_strict", "mx[0] <= r0 && mn[1] >= r1", "mx[0] < r0 && mn[1] >= r1", CLASSIFY_GOLDEN),
     ("localize_shift_off_by_one", "x = x - a;", "x = x - a - 1;", LOCALIZE),
     ("localize_multi_first_offset", "acc += x - a[t];", "acc += x - a[0];", LOCALIZE_MULTI),
     ("count_negated", "cnt += !is_masked(lts, lte, uts, ute, j, i);\n    total += cnt;",
@@ -124,7 +138,7 @@ def source():
 def test_control_unchanged_source_passes_every_pin(source, tmp_path):
     lib = oracle.build_variant(source, str(tmp_path))
     with oracle.use_library(lib):
-        for check in FWD + BWD + CLASSIFY + LOCALIZE + LOCALIZE_MULTI + COUNT + TILE_COSTS:
+        for check in FWD + BWD + CLASSIFY + CLASSIFY_GOLDEN + LOCALIZE + LOCALIZE_MULTI + COUNT + TILE_COSTS:
             assert not _fails(check)
 
 

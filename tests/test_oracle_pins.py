@@ -374,6 +374,31 @@ def test_classify_causal_closed_form(oracle_mod):
     assert np.array_equal(cls, expect)
 
 
+def classify_golden():
+    """Vectors, Nq and expected classes of tests/golden/classify_clauses.json (hand-derived)."""
+    with open(os.path.join(GOLDEN, "classify_clauses.json")) as f:
+        d = json.load(f)
+    vec = {n: [] for n in ("lts", "lte", "uts", "ute")}
+    for t in d["ktiles"]:
+        for n in vec:
+            x = t[n]
+            vec[n] += list(x) if isinstance(x, list) else [x] * t["n"]
+            assert len(vec[n]) == len(vec["lts"]) or n == "lts"
+    vecs = [np.array(vec[n], np.int32) for n in ("lts", "lte", "uts", "ute")]
+    return vecs, int(d["Nq"]), np.array(d["expected"], np.uint8)
+
+
+def test_classify_golden_clauses(oracle_mod):
+    """Every clause of the tile rule, at its boundary, is the only one deciding some tile of the
+    hand-derived golden: a dropped clause or a strict/non-strict slip changes a class."""
+    vecs, nq, expect = classify_golden()
+    nk = vecs[0].size
+    cls = oracle_mod.classify(*[x[None, None] for x in vecs], nq, nk)[0, 0]
+    assert cls.shape == expect.shape
+    assert np.array_equal(cls, expect), np.argwhere(cls != expect)
+    _check_sound(expect, dense_mask_np(*vecs, nq), 128, 128)  # the golden itself is sound
+
+
 def test_classify_tile_aligned_documents(oracle_mod):
     lengths = [256, 128, 384, 256]
     vecs = wl.causal_document_vectors(lengths)
