@@ -56,6 +56,8 @@ def parse_args(argv=None):
     ap.add_argument("--config", default=DEFAULT_CONFIG, choices=wl.CONFIG_ORDER)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-secondary", action="store_true", help="time only the headline workload")
+    ap.add_argument("--bwd-mode", choices=["fused", "split"], default="fused",
+                    help="backward: one key-stationary pass (default) or the deterministic two-kernel split")
     return ap.parse_args(argv)
 
 
@@ -320,7 +322,7 @@ def time_device(fm, pb, steps, warmup, flush, world, clocks=None):
 def unit_rates(prof, pairs, d, peak):
     """Effective TFLOP/s and fraction of peak of the forward unit and the backward pair."""
     out = {}
-    for k, fl in (("fwd", 4.0 * d * pairs), ("bwd_pair", 10.0 * d * pairs)):
+    for k, fl in (("fwd", 4.0 * d * pairs), ("bwd", 10.0 * d * pairs)):
         ms, nl = prof[f"{k}_ms"], prof[f"{k}_launches"]
         tf = fl / (ms / nl / 1e3) / 1e12 if nl else None
         out[k] = {"ms_per_launch": ms / nl if nl else None, "tflops": tf, "frac": tf / peak if tf else None}
@@ -332,6 +334,7 @@ def run_ours(args, rank, world, local_rank):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
+    fm.set_bwd_mode(args.bwd_mode)
     peaks, peak_src = load_peaks()
     peak = float(peaks["bf16_tflops"])
     w = wl.CONFIGS[args.config]
@@ -381,21 +384,31 @@ def run_ours(args, rank, world, local_rank):
     del d_e2e, h_out
 
     # ---- roofline of the dominant unit ----
-    # Units: the forward kernel, and the backward's two attention kernels,
-    # which run concurrently (key side on the caller's stream, query side on
-    # the library's second stream) and are timed together from fork to join.
+    # Units: the forward kernel, and the backward's attention unit.  Fused
+    # mode: the key-stationary kernel that computes all five matmuls of each
+    # pair plus the dQ finalize (an HBM-bound conversion), timed together.
+    # Split mode: the key-side and query-side kernels, which run concurrently
+    # (key side on the caller's stream, query side on the library's second
+    # stream), timed together from fork to join.
     # Algorithmic work = the matmuls the method needs over unmasked pairs:
     # forward 2 (QK^T, PV) = 4*d*pairs; backward 5 (S, dP, dV, dK, dQ) =
-    # 10*d*pairs.  Executed work per kernel (reported beside it) adds the
-    # query side's recomputed S and dP: key side 8*d*pairs, query side
-    # 6*d*pairs.
+    # 10*d*pairs.  Executed work per kernel is reported beside it (split mode
+    # adds the query side's recomputed S and dP: key side 8*d*pairs, query
+    # side 6*d*pairs).
     d = w.d
-    units = {"fwd": (("fwd_sm100.cu",), f"fm_fwd_kernel<{d}>", 4.0 * d * pairs),
-             "bwd_pair": (("bwd_dkdv_sm100.cu", "bwd_dq_sm100.cu"),
-                          f"fm_bwd_dkdv_kernel<{d}> + fm_bwd_dq_kernel<{d}> (concurrent)", 10.0 * d * pairs)}
-    executed = {"fwd": (f"fm_fwd_kernel<{d}>", 4.0 * d * pairs),
-                "bwd_kv": (f"fm_bwd_dkdv_kernel<{d}>", 8.0 * d * pairs),
-                "bwd_q": (f"fm_bwd_dq_kernel<{d}>", 6.0 * d * pairs)}
+    if args.bwd_mode == "fused":
+        bwd_unit = (("bwd_fused_sm100.cu",), f"fm_bwd_fused_kernel<{d}> + fm_dq_finalize_kernel<{d}>",
+                    10.0 * d * pairs)
+        executed = {"fwd": (f"fm_fwd_kernel<{d}>", 4.0 * d * pairs),
+                    "bwd_fused": (f"fm_bwd_fused_kernel<{d}>", 10.0 * d * pairs),
+                    "dq_finalize": (f"fm_dq_finalize_kernel<{d}>", 0.0)}
+    else:
+        bwd_unit = (("bwd_dkdv_sm100.cu", "bwd_dq_sm100.cu"),
+                    f"fm_bwd_dkdv_kernel<{d}> + fm_bwd_dq_kernel<{d}> (concurrent)", 10.0 * d * pairs)
+        executed = {"fwd": (f"fm_fwd_kernel<{d}>", 4.0 * d * pairs),
+                    "bwd_kv": (f"fm_bwd_dkdv_kernel<{d}>", 8.0 * d * pairs),
+                    "bwd_q": (f"fm_bwd_dq_kernel<{d}>", 6.0 * d * pairs)}
+    units = {"fwd": (("fwd_sm100.cu",), f"fm_fwd_kernel<{d}>", 4.0 * d * pairs), "bwd": bwd_unit}
     per_unit = {}
     for k, (srcs, kname, fl) in units.items():
         ms, nl = prof[f"{k}_ms"], prof[f"{k}_launches"]
@@ -408,8 +421,9 @@ def run_ours(args, rank, world, local_rank):
     for k, (kname, fl) in executed.items():
         ms, nl = prof[f"{k}_ms"], prof[f"{k}_launches"]
         per_kernel[k] = {"kernel": kname, "ms_per_launch": ms / nl if nl else None, "launches": nl,
-                         "executed_tflops": fl / (ms / nl / 1e3) / 1e12 if nl else None, "executed_flops": fl,
-                         "note": "runs concurrently with the other backward kernel" if k != "fwd" else ""}
+                         "executed_tflops": fl / (ms / nl / 1e3) / 1e12 if nl and fl else None,
+                         "executed_flops": fl,
+                         "note": "runs concurrently with the other backward kernel" if k in ("bwd_kv", "bwd_q") else ""}
     dom = max(per_unit, key=lambda k: prof[f"{k}_ms"])
     pk = per_unit[dom]
     roof = {"bound": "tensor", "achieved": pk["tflops"], "peak": peak, "unit": "TFLOP/s",
@@ -428,6 +442,7 @@ def run_ours(args, rank, world, local_rank):
         "config": {"workload": w.name, "description": w.description, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv,
                    "seqlen": w.N, "head_dim": w.d, "unmasked_pairs": pairs,
                    "flops_per_step": {"fwd": f_fwd, "bwd": f_bwd}, "tile_classes": hist,
+                   "bwd_mode": args.bwd_mode,
                    "l2": "flushed before every step (2x L2 bytes written, outside the step's events)",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "e2e": {"value": e2e_value, "unit": "TFLOP/s", "steps": e2e_steps,

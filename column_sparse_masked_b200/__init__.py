@@ -34,6 +34,8 @@ from ._binding import (  # noqa: F401
     localize_multi,
     profiler_enable,
     profiler_read,
+    get_bwd_mode,
+    set_bwd_mode,
     set_max_ctas,
     set_wait_limit_ns,
     test_wait_timeout,
@@ -44,6 +46,6 @@ from ._binding import (  # noqa: F401
 
 __all__ = [
     "FlashMaskError", "balance_chunks", "classify", "count_unmasked", "flashmask_attention", "fwd", "bwd", "get_status", "get_timeout_info",
-    "launch_count", "lib_path", "load_library", "localize", "localize_multi", "profiler_enable", "profiler_read", "set_max_ctas", "set_wait_limit_ns", "test_wait_timeout", "tile_costs",
+    "launch_count", "lib_path", "load_library", "localize", "localize_multi", "profiler_enable", "profiler_read", "get_bwd_mode", "set_bwd_mode", "set_max_ctas", "set_wait_limit_ns", "test_wait_timeout", "tile_costs",
     "version", "workspace_size",
 ]

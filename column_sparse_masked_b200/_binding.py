@@ -28,6 +28,8 @@ _SIGS = {
     "flashmask_tile_costs": (ctypes.c_int, [_P, _P, _P, _P, _DIMS, _P, _P]),
     "flashmask_balance_chunks": (ctypes.c_int, [_P, ctypes.c_int32, ctypes.c_int32, _P, _P]),
     "flashmask_set_max_ctas": (ctypes.c_int, [ctypes.c_int32]),
+    "flashmask_set_bwd_mode": (ctypes.c_int, [ctypes.c_int32]),
+    "flashmask_get_bwd_mode": (ctypes.c_int, []),
     "flashmask_get_timeout_info": (ctypes.c_int, [_P]),
     "flashmask_get_status": (ctypes.c_int, []),
     "flashmask_set_wait_limit_ns": (None, [ctypes.c_int64]),
@@ -303,6 +305,22 @@ def set_max_ctas(n: int) -> None:
     _check(load_library().flashmask_set_max_ctas(int(n)), "flashmask_set_max_ctas")
 
 
+BWD_FUSED, BWD_SPLIT = 0, 1
+_BWD_MODES = {"fused": BWD_FUSED, "split": BWD_SPLIT}
+
+
+def set_bwd_mode(mode) -> None:
+    """Backward mode of later ``bwd`` calls: "fused" (default; one key-stationary pass, dQ by fp32
+    reductions) or "split" (separate dK/dV and dQ kernels, bit-reproducible)."""
+    m = _BWD_MODES.get(mode, mode)
+    _check(load_library().flashmask_set_bwd_mode(int(m)), "flashmask_set_bwd_mode")
+
+
+def get_bwd_mode() -> str:
+    m = int(load_library().flashmask_get_bwd_mode())
+    return {v: k for k, v in _BWD_MODES.items()}[m]
+
+
 def balance_chunks(costs: Sequence[int], parts: int) -> Tuple[List[int], int]:
     """Splits q-tiles into ``parts`` contiguous chunks with the smallest possible largest cost.
 
@@ -324,7 +342,7 @@ def get_status() -> int:
     return int(load_library().flashmask_get_status())
 
 
-_TIMEOUT_KERNELS = ("forward", "backward key side", "backward query side", "wait self-test")
+_TIMEOUT_KERNELS = ("forward", "backward key side", "backward query side", "wait self-test", "fused backward")
 
 
 def get_timeout_info() -> dict:
@@ -352,14 +370,19 @@ def profiler_enable(on: bool = True) -> None:
     _check(load_library().flashmask_profiler_enable(1 if on else 0), "flashmask_profiler_enable")
 
 
+PROFILER_KINDS = ("fwd", "bwd_kv", "bwd_q", "bwd", "bwd_fused", "dq_finalize")
+
+
 def profiler_read():
-    """{'<kind>_ms', '<kind>_launches'} since the last read, kinds fwd, bwd_kv, bwd_q and bwd_pair
-    (the two backward kernels run concurrently; bwd_pair is their joint duration)."""
-    ms = (ctypes.c_double * 4)()
-    cnt = (ctypes.c_int64 * 4)()
+    """{'<kind>_ms', '<kind>_launches'} since the last read.  Kinds: fwd; bwd_kv and bwd_q (split
+    backward's two kernels, concurrent); bwd (the backward's attention unit: split, the two kernels
+    from fork to join; fused, the fused kernel and the dQ finalize); bwd_fused; dq_finalize."""
+    n = len(PROFILER_KINDS)
+    ms = (ctypes.c_double * n)()
+    cnt = (ctypes.c_int64 * n)()
     _check(load_library().flashmask_profiler_read(ms, cnt), "flashmask_profiler_read")
     out = {}
-    for i, k in enumerate(("fwd", "bwd_kv", "bwd_q", "bwd_pair")):
+    for i, k in enumerate(PROFILER_KINDS):
         out[f"{k}_ms"] = ms[i]
         out[f"{k}_launches"] = cnt[i]
     return out

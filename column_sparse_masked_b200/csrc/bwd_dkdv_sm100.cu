@@ -39,6 +39,7 @@
 #include <climits>
 #include <cmath>
 
+#include "bwd_items.cuh"
 #include "common.cuh"
 #include "launchers.h"
 #include "sm100_primitives.cuh"
@@ -54,31 +55,6 @@ constexpr int kDoStages = 2;  // dO tiles: last read by dV(t), freed earlier
 constexpr int kLStages = 2;   // LSE2 / D rows: last read by the compute warps
 constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256;
 }  // namespace kvb
-
-// A decoded work item (batch, KV head, k-tile).  The first producer decodes
-// each item once and publishes it in the shared-memory ring; the other roles
-// read it there.  item >= n_items ends the work.
-struct __align__(16) KvItem {
-  int item, b, hkv, kt, total;  // total = q-tiles over all q-heads of the group
-};
-
-__device__ __forceinline__ KvItem decode_kv_item(const BwdParams& p, int item) {
-  const Shape& sh = p.s;
-  KvItem it{};
-  it.item = item;
-  if (item >= p.n_items) return it;
-  const ItemCoord c = decode_kv_item_coord(sh, p.order[item]);
-  it.b = c.b;
-  it.hkv = c.hkv;
-  it.kt = c.t;
-  it.total = 0;
-  for (int gi = 0; gi < sh.G; ++gi) {
-    const int h = it.hkv * sh.G + gi;
-    const int hm = (sh.Hm == 1) ? 0 : h;
-    it.total += p.bcount[((size_t)it.b * sh.Hm + hm) * sh.nKt + it.kt];
-  }
-  return it;
-}
 
 template <int D>
 struct __align__(1024) DkdvSmem {
@@ -104,25 +80,6 @@ struct __align__(1024) DkdvSmem {
 
 static_assert(sizeof(DkdvSmem<128>) <= 232448, "key-side shared memory exceeds the per-CTA limit");
 static_assert(sizeof(DkdvSmem<64>) <= 232448, "key-side shared memory exceeds the per-CTA limit");
-
-// Calls f(j, h, hm, qt, cls) for the item's q-tiles in the order every role walks them.
-template <typename F>
-__device__ __forceinline__ bool for_each_qtile(const BwdParams& p, const KvItem& it, F&& f) {
-  const Shape& sh = p.s;
-  int j = 0;
-  for (int gi = 0; gi < sh.G; ++gi) {
-    const int h = it.hkv * sh.G + gi;
-    const int hm = (sh.Hm == 1) ? 0 : h;
-    const size_t lrow = ((size_t)it.b * sh.Hm + hm) * sh.nKt + it.kt;
-    const int* list = p.blist + lrow * sh.nQt;
-    const int cnt = p.bcount[lrow];
-    for (int t = 0; t < cnt; ++t, ++j) {
-      const int e = list[t];
-      if (!f(j, h, hm, e >> 2, e & 3)) return false;
-    }
-  }
-  return true;
-}
 
 // D[tmem] = A B^T, both K-major SW128 over the head dimension (128 x 128 tile).
 template <int D>

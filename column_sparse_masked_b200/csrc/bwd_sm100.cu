@@ -15,7 +15,8 @@
 namespace fm {
 
 // ----------------------------------------------------------------------------
-// preprocess: D = rowsum(dO * O) and LSE in log2 units, per padded row.
+// preprocess: D = rowsum(dO * O) and LSE in log2 units, per padded row (and,
+// for the fused backward, zeroing of its fp32 dQ accumulator).
 // Half a warp per (b, row, h) of the padded row range, h fastest (coalesced):
 // each lane loads 16 bytes of O and of dO, a warp covers two rows per step.
 // The kernel is bound by reading O and dO once from HBM.
@@ -31,6 +32,12 @@ __global__ void __launch_bounds__(256) fm_bwd_pre_kernel(BwdPreParams p) {
   const int sub = lane / kLanes, sl = lane % kLanes;
   const int64_t warp0 = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  if (p.dqacc) {  // fused backward: zero the fp32 dQ accumulator (16-byte stores, grid-stride)
+    const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < p.dqacc_vec4;
+         t += (int64_t)gridDim.x * blockDim.x)
+      p.dqacc[t] = z;
+  }
   for (int64_t r0 = warp0 * kRowsPerWarp; r0 < rows; r0 += nwarps * kRowsPerWarp) {
     const int64_t r = r0 + sub;
     const bool in = r < rows;

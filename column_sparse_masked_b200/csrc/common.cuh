@@ -66,10 +66,18 @@ inline Shape make_shape(int B, int Hq, int Hkv, int Hm, int Nq, int Nk, int d) {
 struct WsLayout {
   size_t rec, ksum, fcount, flist, qcount, forder, counters;  // forward part
   size_t bcount, blist, border, qorder, lse2, dsum;        // backward part
+  size_t dqacc;                                            // fused backward: fp32 dQ accumulator
   size_t fwd_bytes, bwd_bytes;
 };
 
 inline size_t ws_align(size_t x) { return (x + 255) & ~size_t(255); }
+
+// fp32 dQ accumulator of the fused backward, one 128-row tile per
+// (batch, q-head, q-tile), laid out [B, Hq, nQt, d/4, 128, 4]: four
+// consecutive columns of one row are 16 contiguous bytes, and the 128 rows of
+// one 4-column chunk are contiguous, so one warp-wide 16-byte reduction of 32
+// consecutive rows covers 512 contiguous bytes.
+inline size_t dqacc_bytes(const Shape& s) { return (size_t)s.B * s.Hq * s.nQt * kTile * s.d * 4; }
 
 inline WsLayout make_layout(const Shape& s) {
   WsLayout L{};
@@ -90,6 +98,7 @@ inline WsLayout make_layout(const Shape& s) {
   L.qorder = take((size_t)s.n_q_items * 4);
   L.lse2 = take((size_t)s.B * s.Hq * s.nQt * kTile * 4);
   L.dsum = take((size_t)s.B * s.Hq * s.nQt * kTile * 4);
+  L.dqacc = take(dqacc_bytes(s));
   L.bwd_bytes = off;
   return L;
 }
@@ -175,6 +184,8 @@ struct BwdPreParams {
   const float* lse;
   float* lse2;     // [B, Hq, nQt*128]: LSE * log2(e); +inf for empty and padded rows
   float* dsum;     // [B, Hq, nQt*128]: rowsum(dO * O); 0 for padded rows
+  float4* dqacc;   // fused backward: accumulator zeroed here (null: none)
+  int64_t dqacc_vec4;
 };
 
 struct BwdParams {
@@ -200,6 +211,7 @@ struct BwdParams {
   __nv_bfloat16* dq;
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
+  float* dqacc;         // fused backward: [B, Hq, nQt, d/4, 128, 4] fp32, zeroed before the kernel
   int* status;
   uint64_t wait_limit_ns;
 };

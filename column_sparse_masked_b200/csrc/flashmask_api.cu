@@ -32,6 +32,7 @@ namespace {
 
 std::atomic<int64_t> g_wait_limit_ns{2000000000LL};
 std::atomic<int> g_max_ctas{0};  // 0: one persistent CTA per SM
+std::atomic<int> g_bwd_mode{FLASHMASK_BWD_FUSED};
 
 // Persistent grid of an attention kernel: one CTA per SM, at most one per
 // work item, at most the process-wide cap when one is set.
@@ -246,7 +247,7 @@ int wave_groups(size_t group_bytes, int n_groups, int64_t n_items, int sm_count)
 void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 // A begin/end pair is recorded only while profiling is on.
-constexpr int kProfKinds = 4;
+constexpr int kProfKinds = 6;
 
 int profile_begin(int kind, cudaStream_t st) {
   if (!g_profiling.load(std::memory_order_relaxed)) return -1;
@@ -423,6 +424,7 @@ int flashmask_bwd(const void* q, const void* k, const void* v, const void* o, co
   JoinOnExit join_guard;  // destroyed before the lock is released
   join_guard.ax = ax;
   join_guard.st = st;
+  const bool fused = g_bwd_mode.load(std::memory_order_relaxed) == FLASHMASK_BWD_FUSED;
   BwdPreParams bp{};
   bp.s = s;
   bp.o = static_cast<const __nv_bfloat16*>(o);
@@ -430,6 +432,10 @@ int flashmask_bwd(const void* q, const void* k, const void* v, const void* o, co
   bp.lse = lse;
   bp.lse2 = reinterpret_cast<float*>(ws + L.lse2);
   bp.dsum = reinterpret_cast<float*>(ws + L.dsum);
+  if (fused) {  // the preprocess also zeroes the fp32 dQ accumulator
+    bp.dqacc = reinterpret_cast<float4*>(ws + L.dqacc);
+    bp.dqacc_vec4 = (int64_t)(dqacc_bytes(s) / 16);
+  }
   const int pre_blocks = 64 * di.sm_count;
   if (ax) {
     FM_CUDA(cudaEventRecord(ax->fork, st));
@@ -444,7 +450,56 @@ int flashmask_bwd(const void* q, const void* k, const void* v, const void* o, co
   const MaskPrepParams mp = prep_params(s, L, ws, lts, lte, uts, ute);
   FM_CUDA(launch_mask_prep(mp, st));
 
-  // key side: per k-tile q-tile lists, longest-first units
+  if (fused) {
+    // one key-stationary pass: key-side lists and order only
+    PlanParams pp{};
+    pp.s = s;
+    pp.ksum = mp.ksum;
+    pp.bcount = reinterpret_cast<int*>(ws + L.bcount);
+    pp.blist = reinterpret_cast<int*>(ws + L.blist);
+    FM_CUDA(launch_plan_bwd(pp, st));
+    SortParams sb{};
+    sb.s = s;
+    sb.mode = 1;
+    sb.count = pp.bcount;
+    sb.order = reinterpret_cast<int*>(ws + L.border);
+    sb.counter = reinterpret_cast<int*>(ws + L.counters) + 1;
+    sb.n_items = (int)s.n_kv_items;
+    sb.items_per_group = s.nKt;
+    sb.wave = wave_groups((size_t)s.G * s.Nq * s.d * 2 * 2, s.B * s.Hkv, s.n_kv_items, di.sm_count);
+    finish_sort_params(sb);
+    if (sb.n_items > 0) FM_CUDA(launch_sort_units(&sb, 1, st));
+    BwdParams kp{};
+    kp.s = s;
+    kp.scale = sc;
+    kp.scale_log2 = sc * 1.4426950408889634f;
+    kp.rec = mp.rec;
+    kp.blist = pp.blist;
+    kp.bcount = pp.bcount;
+    kp.order = sb.order;
+    kp.counter = sb.counter;
+    kp.n_items = (int)s.n_kv_items;
+    kp.lse2 = bp.lse2;
+    kp.dsum = bp.dsum;
+    kp.dq = static_cast<__nv_bfloat16*>(dq);
+    kp.dk = static_cast<__nv_bfloat16*>(dk);
+    kp.dv = static_cast<__nv_bfloat16*>(dv);
+    kp.dqacc = reinterpret_cast<float*>(ws + L.dqacc);
+    kp.status = di.status;
+    kp.wait_limit_ns = (uint64_t)g_wait_limit_ns.load();
+    const int grid = persistent_grid(kp.n_items, di.sm_count);
+    if (ax) {
+      FM_CUDA(cudaStreamWaitEvent(st, ax->pre, 0));  // D, LSE2 and the zeroed accumulator
+      join_guard.armed = false;                      // nothing of this call is left on the second stream
+    }
+    const int prof = profile_begin(3, st);
+    if (grid > 0) FM_CUDA(launch_bwd_fused(kp, tq, tk, tv, tdo, grid, st));
+    if (has_q) FM_CUDA(launch_dq_finalize(kp, 64 * di.sm_count, st));
+    profile_end(prof, st);
+    return FLASHMASK_OK;
+  }
+
+  // split backward -- key side: per k-tile q-tile lists, longest-first units
   PlanParams pp{};
   pp.s = s;
   pp.ksum = mp.ksum;
@@ -621,6 +676,14 @@ int flashmask_tile_costs(const int32_t* lts, const int32_t* lte, const int32_t* 
   FM_CUDA(launch_tile_costs(mp, d.Hq, d.Nq, costs, static_cast<cudaStream_t>(stream)));
   return FLASHMASK_OK;
 }
+
+int flashmask_set_bwd_mode(int32_t mode) {
+  if (mode != FLASHMASK_BWD_FUSED && mode != FLASHMASK_BWD_SPLIT) return FLASHMASK_ERR_INVALID_ARG;
+  g_bwd_mode.store(mode);
+  return FLASHMASK_OK;
+}
+
+int flashmask_get_bwd_mode(void) { return g_bwd_mode.load(); }
 
 int flashmask_set_max_ctas(int32_t n) {
   if (n < 0) return FLASHMASK_ERR_INVALID_ARG;

@@ -34,6 +34,11 @@ cudaError_t launch_bwd_dkdv(const BwdParams& p, const CUtensorMap& tq, const CUt
                             const CUtensorMap& tdo, int grid, cudaStream_t st);
 cudaError_t launch_bwd_dq(const BwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                           const CUtensorMap& tdo, int grid, cudaStream_t st);
+// Fused backward (dQ, dK, dV in one key-stationary pass; dQ into p.dqacc) and
+// the conversion of the fp32 dQ accumulator into bf16 dQ.
+cudaError_t launch_bwd_fused(const BwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                             const CUtensorMap& tdo, int grid, cudaStream_t st);
+cudaError_t launch_dq_finalize(const BwdParams& p, int max_blocks, cudaStream_t st);
 
 // Launch bookkeeping: counts every launch.
 void note_launch();
@@ -61,8 +66,10 @@ cudaError_t launch_after(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t
 }
 // Kernel timing (while profiling is on): begin records a start event on st and
 // returns a handle (-1 when nothing was recorded); end records the matching
-// stop event.  Kinds: 0 forward, 1 backward key side, 2 backward query side,
-// 3 the backward attention pair (fork to join).
+// stop event.  Kinds: 0 forward, 1 backward key side, 2 backward query side
+// (split backward), 3 the backward's attention unit (split: the two kernels,
+// fork to join; fused: the fused kernel and the dQ finalize), 4 the fused
+// backward kernel, 5 the dQ finalize.
 int profile_begin(int kind, cudaStream_t st);
 void profile_end(int handle, cudaStream_t st);
 

@@ -117,25 +117,43 @@ int flashmask_fwd_noalloc(const void* q, const void* k, const void* v, const int
                           void* o, float* lse, void* stream);
 
 /* Bytes of workspace flashmask_bwd needs (forward's plus the backward lists,
- * and per-row D = rowsum(dO*O) and LSE in log2 units over whole 128-row
- * tiles). */
+ * per-row D = rowsum(dO*O) and LSE in log2 units over whole 128-row tiles, and
+ * the fused backward's fp32 dQ accumulator, 4 * B * Hq * ceil(Nq/128) * 128 * d
+ * bytes).  The same size serves both backward modes. */
 size_t flashmask_bwd_workspace_size(const flashmask_dims* dims);
+
+/* Backward modes (process-wide, flashmask_set_bwd_mode). */
+#define FLASHMASK_BWD_FUSED 0 /* default: one key-stationary pass, dQ by fp32 reductions   */
+#define FLASHMASK_BWD_SPLIT 1 /* key-side dK/dV kernel + query-side dQ kernel, deterministic */
 
 /*
  * Backward of the forward above for the loss sum(O * dO) (same page and
- * section: the mask-aware kernels cover both passes): dQ, dK, dV.  dK and dV sum the contributions of the
- * Hq/Hkv q-heads that share a KV head.  `o` and `lse` must be the forward's
- * outputs for the same inputs.  Key columns that no row sees get dK = dV = 0;
- * fully masked rows get dQ = 0.  Outputs are written in full, each element by
- * exactly one CTA (no atomics): results are deterministic.
- * The mask summary, lists, orders and the dK/dV kernel run on `stream`; the
- * preprocess (each row's D = rowsum(dO*O) and LSE in log2 units) and the dQ
- * kernel run on a stream the library owns (one per device, created on first
- * use), ordered after the call's earlier work on `stream` by an event and
- * joined back to `stream` by another: everything the call writes is complete
- * in `stream` order when the call's last operation there completes.
- * Concurrent calls from several host threads share that stream and are
- * serialised on it.
+ * section: the mask-aware kernels cover both passes): dQ, dK, dV.  dK and dV
+ * sum the contributions of the Hq/Hkv q-heads that share a KV head.  `o` and
+ * `lse` must be the forward's outputs for the same inputs.  Key columns that
+ * no row sees get dK = dV = 0; fully masked rows get dQ = 0.  Outputs are
+ * written in full.
+ *
+ * FLASHMASK_BWD_FUSED (default): each non-skipped (q-tile, k-tile) pair is
+ * visited once by a key-stationary kernel that forms S, dP and dS once and
+ * computes all five matmuls of the pair; dK and dV are accumulated on chip
+ * and written once (deterministic); each pair's dQ contribution is added into
+ * an fp32 accumulator in the workspace with fp32 reductions, and a finalize
+ * kernel writes dQ = bf16(scale * acc).  dQ is therefore exact up to the
+ * order of fp32 additions, which varies from run to run.
+ * FLASHMASK_BWD_SPLIT: a key-stationary dK/dV kernel and a query-stationary
+ * dQ kernel that recomputes S and dP (1.4x the matmul work); every output
+ * element is written by exactly one CTA, no atomics: bit-reproducible.
+ *
+ * Streams: the preprocess (each row's D = rowsum(dO*O) and LSE in log2 units;
+ * in fused mode also zeroing the dQ accumulator) runs on a stream the library
+ * owns (one per device, created on first use), ordered after the call's
+ * earlier work on `stream` by an event; the mask summary, lists and orders run
+ * on `stream` meanwhile.  In split mode the dQ kernel also runs on the
+ * library's stream, joined back to `stream` by another event.  Either way
+ * everything the call writes is complete in `stream` order when the call's
+ * last operation there completes.  Concurrent calls from several host threads
+ * share the library's stream and are serialised on it.
  */
 int flashmask_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
                   const int32_t* lts, const int32_t* lte, const int32_t* uts, const int32_t* ute, float scale,
@@ -217,6 +235,12 @@ int flashmask_tile_costs(const int32_t* lts, const int32_t* lte, const int32_t* 
  */
 int flashmask_balance_chunks(const int64_t* costs, int32_t n, int32_t parts, int32_t* bounds, int64_t* max_cost);
 
+/* Selects the backward mode (FLASHMASK_BWD_FUSED or FLASHMASK_BWD_SPLIT) for
+ * every later flashmask_bwd call of the process; FLASHMASK_ERR_INVALID_ARG
+ * for any other value.  flashmask_get_bwd_mode returns the current one. */
+int flashmask_set_bwd_mode(int32_t mode);
+int flashmask_get_bwd_mode(void);
+
 /* Synchronises the current device, returns its status word (0 or a negative
  * FLASHMASK_ERR_* code written by a kernel) and resets it to 0. */
 int flashmask_get_status(void);
@@ -225,7 +249,7 @@ int flashmask_get_status(void);
  * the bounded wait that caused the first FLASHMASK_ERR_TIMEOUT since the
  * status word was last cleared (left unchanged when none occurred since):
  * info[0] kernel (0 forward, 1 backward key side, 2 backward query side,
- * 3 the flashmask_test_wait_timeout self-test), info[1] byte offset of the
+ * 3 the flashmask_test_wait_timeout self-test, 4 fused backward), info[1] byte offset of the
  * mbarrier in that kernel's shared-memory block, info[2] the phase parity
  * waited for, info[3] block index, info[4] thread index.  Returns
  * FLASHMASK_ERR_INVALID_ARG for a NULL info. */
@@ -253,14 +277,15 @@ int flashmask_test_wait_timeout(int64_t limit_ns, void* stream);
 /*
  * Kernel timing for benchmarks.  While enabled (on != 0), every launch of an
  * attention kernel is bracketed by a CUDA event pair recorded on the stream it
- * runs on, and so is the backward's pair of attention kernels as a whole (on
- * the call's stream, from before the key-side launch to after both kernels
- * completed).  flashmask_profiler_read() waits for the recorded events and
- * fills ms[4] / launches[4] (either may be NULL) with the summed milliseconds
- * and counts of kind 0 = forward, 1 = backward key side (dK, dV), 2 = backward
- * query side (dQ), 3 = the backward pair (kinds 1 and 2 run concurrently, so
- * 3 is their joint duration), then clears them.  Event pairs are pooled (at
- * most 4096 outstanding).  Host-side, process-wide.
+ * runs on, and so is the backward's attention unit as a whole (on the call's
+ * stream).  flashmask_profiler_read() waits for the recorded events and fills
+ * ms[6] / launches[6] (either may be NULL) with the summed milliseconds and
+ * counts of kind 0 = forward, 1 = split backward key side (dK, dV), 2 = split
+ * backward query side (dQ), 3 = the backward's attention unit (split: kinds 1
+ * and 2, which run concurrently, from before the first launch to after both
+ * completed; fused: the fused kernel and the dQ finalize), 4 = fused backward
+ * kernel, 5 = dQ finalize, then clears them.  Event pairs are pooled (at most
+ * 4096 outstanding).  Host-side, process-wide.
  */
 int flashmask_profiler_enable(int on);
 int flashmask_profiler_read(double* ms, int64_t* launches);

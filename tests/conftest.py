@@ -27,3 +27,15 @@ def cuda_available() -> bool:
         return torch.cuda.is_available()
     except Exception:  # pragma: no cover
         return False
+
+
+@pytest.fixture(params=["fused", "split"])
+def bwd_mode(request):
+    """Runs a test once per backward mode; restores the default (fused) afterwards."""
+    import column_sparse_masked_b200 as fm
+
+    fm.set_bwd_mode(request.param)
+    try:
+        yield request.param
+    finally:
+        fm.set_bwd_mode("fused")

@@ -17,7 +17,8 @@ Checked on every schedule:
     MMA or a compute role reads or overwrites it.
 
 The sequences restate the kernels in csrc/ (fwd_sm100.cu, bwd_dq_sm100.cu,
-bwd_dkdv_sm100.cu); a change to a kernel's protocol needs the same change here.
+bwd_dkdv_sm100.cu, bwd_fused_sm100.cu); a change to a kernel's protocol needs
+the same change here.
 """
 from __future__ import annotations
 
@@ -632,7 +633,231 @@ def dkdv_model(items, seed, R=4, QST=3, DOST=2, LST=2):
              "compute1": compute(1)})
 
 
-MODELS = {"fwd": fwd_model, "dq": dq_model, "dkdv": dkdv_model}
+# ----------------------------------------------------------------------------
+# fused backward (fm_bwd_fused_kernel): dkdv's roles plus dQ(t) = dS K into the
+# dP^T region, read out by the compute warpgroups between the halves of P^T(t+1)
+# ----------------------------------------------------------------------------
+def fused_model(items, seed, R=4, QST=2, DOST=2, LST=2):
+    sim = Sim(seed)
+    for i in range(R):
+        sim.bar(f"ring_full{i}")
+        sim.bar(f"ring_empty{i}", 1 + 1 + 2)  # MMA + second producer + the two compute warpgroups
+    for nm in ("k_full", "k_empty", "v_full", "v_empty", "s_full", "dp_full", "dq_full", "dkdv_full"):
+        sim.bar(nm)
+    for nm in ("p_full", "ds_full", "dq_free", "dkdv_free"):
+        sim.bar(nm, 2)
+    for i in range(QST):
+        sim.bar(f"q_full{i}")
+        sim.bar(f"q_empty{i}")
+    for i in range(DOST):
+        sim.bar(f"do_full{i}")
+        sim.bar(f"do_empty{i}")
+    for i in range(LST):
+        sim.bar(f"l_full{i}")
+        sim.bar(f"l_empty{i}", 2)
+    ring = [None] * R
+    st = {"k": None, "v": None, "q": [None] * QST, "do": [None] * DOST, "l": [None] * LST,
+          "S": [None, None], "dP": [None, None], "dsm": [None, None], "dV": "free", "dK": "free"}
+    seq = list(items) + [None]
+
+    def producer():  # K and every q-tile's Q; K is freed after the item's last dQ
+        sq = act = k = 0
+        for it in seq:
+            yield wait(f"ring_empty{k % R}", k // R - 1)
+            ring[k % R] = it
+            sim.arrive(f"ring_full{k % R}")
+            k += 1
+            if it is None:
+                return
+            j, n = it
+            if n == 0:
+                continue
+            yield wait("k_empty", act - 1)
+            sim.tma.append(("k_full", lambda j=j: st.__setitem__("k", j)))
+            act += 1
+            for t in range(n):
+                s = sq % QST
+                yield wait(f"q_empty{s}", sq // QST - 1)
+                sim.tma.append((f"q_full{s}", lambda s=s, c=(j, t): st["q"].__setitem__(s, c)))
+                sq += 1
+
+    def producer2():  # V, every q-tile's dO and LSE2 / D rows
+        sq = act = k = 0
+        while True:
+            it = yield from ring_reader(sim, ring, k, R)
+            k += 1
+            if it is None:
+                return
+            j, n = it
+            if n == 0:
+                continue
+            yield wait("v_empty", act - 1)
+            sim.tma.append(("v_full", lambda j=j: st.__setitem__("v", j)))
+            act += 1
+            for t in range(n):
+                s, l = sq % DOST, sq % LST
+                yield wait(f"do_empty{s}", sq // DOST - 1)
+                sim.tma.append((f"do_full{s}", lambda s=s, c=(j, t): st["do"].__setitem__(s, c)))
+                yield wait(f"l_empty{l}", sq // LST - 1)
+                sim.tma.append((f"l_full{l}", lambda l=l, c=(j, t): st["l"].__setitem__(l, c)))
+                sq += 1
+
+    def op_s(j, t, tj, qs):
+        def f():
+            if st["k"] != j or st["q"][qs] != (j, t):
+                raise Hazard(f"S({j},{t}): K {st['k']} Q {st['q'][qs]}")
+            if any(h is not None and h[0] != "used" for h in st["S"]):
+                raise Hazard(f"S({j},{t}) overwrites {st['S']}")
+            st["S"] = [("S", tj), ("S", tj)]
+        return f
+
+    def op_dp(j, t, tj, ds):
+        def f():
+            if st["v"] != j or st["do"][ds] != (j, t):
+                raise Hazard(f"dP({j},{t}): V {st['v']} dO {st['do'][ds]}")
+            if any(h is not None and h[0] != "used" for h in st["dP"]):
+                raise Hazard(f"dP({j},{t}) overwrites {st['dP']}")
+            st["dP"] = [("dP", tj), ("dP", tj)]
+        return f
+
+    def op_dv(j, t, tj, ds):
+        def f():
+            if st["S"] != [("P", tj), ("P", tj)] or st["do"][ds] != (j, t):
+                raise Hazard(f"dV({j},{t}): P {st['S']} dO {st['do'][ds]}")
+            a = st["dV"]
+            if (t == 0 and a != "free") or (t > 0 and a != (j, t - 1)):
+                raise Hazard(f"dV({j},{t}): accumulator holds {a}")
+            st["S"] = [("used", tj), ("used", tj)]
+            st["dV"] = (j, t)
+        return f
+
+    def op_dk(j, t, tj, qs):
+        def f():
+            if st["dP"] != [("dS", tj), ("dS", tj)] or st["q"][qs] != (j, t):
+                raise Hazard(f"dK({j},{t}): dS {st['dP']} Q {st['q'][qs]}")
+            a = st["dK"]
+            if (t == 0 and a != "free") or (t > 0 and a != (j, t - 1)):
+                raise Hazard(f"dK({j},{t}): accumulator holds {a}")
+            st["dP"] = [("read", tj), ("read", tj)]
+            st["dK"] = (j, t)
+        return f
+
+    def op_dq(j, t, tj):
+        def f():
+            if st["k"] != j or st["dsm"] != [("dS", tj), ("dS", tj)]:
+                raise Hazard(f"dQ({j},{t}): K {st['k']} dS {st['dsm']}")
+            if st["dP"] != [("read", tj), ("read", tj)]:
+                raise Hazard(f"dQ({j},{t}) overwrites {st['dP']}")
+            st["dsm"] = [("used", tj), ("used", tj)]
+            st["dP"] = [("dQ", tj), ("dQ", tj)]
+        return f
+
+    def mma():
+        sq = tc = act = k = 0
+        while True:
+            it = yield from ring_reader(sim, ring, k, R)
+            k += 1
+            if it is None:
+                return
+            j, n = it
+            if n == 0:
+                continue
+            qs, ds = sq % QST, sq % DOST
+            yield wait("k_full", act)
+            yield wait(f"q_full{qs}", sq // QST)
+            sim.pipe += [("mma", op_s(j, 0, tc, qs)), ("commit", "s_full")]
+            yield wait("v_full", act)
+            yield wait(f"do_full{ds}", sq // DOST)
+            if tc > 0:
+                yield wait("dq_free", tc - 1)
+            sim.pipe += [("mma", op_dp(j, 0, tc, ds)), ("commit", "dp_full")]
+            if n == 1:
+                sim.pipe.append(("commit", "v_empty"))
+            for t in range(n):
+                sj, tj = sq + t, tc + t
+                qs, ds = sj % QST, sj % DOST
+                qs2, ds2 = (sj + 1) % QST, (sj + 1) % DOST
+                if t == 0:
+                    yield wait("dkdv_free", act - 1)
+                yield wait("p_full", tj)
+                sim.pipe += [("mma", op_dv(j, t, tj, ds)), ("commit", f"do_empty{ds}")]
+                if t + 1 < n:
+                    yield wait(f"q_full{qs2}", (sj + 1) // QST)
+                    sim.pipe += [("mma", op_s(j, t + 1, tj + 1, qs2)), ("commit", "s_full")]
+                yield wait("ds_full", tj)
+                sim.pipe += [("mma", op_dk(j, t, tj, qs)), ("commit", f"q_empty{qs}")]
+                sim.pipe += [("mma", op_dq(j, t, tj)), ("commit", "dq_full")]
+                if t + 1 == n:
+                    sim.pipe.append(("commit", "k_empty"))
+                if t + 1 < n:
+                    yield wait("dq_free", tj)
+                    yield wait(f"do_full{ds2}", (sj + 1) // DOST)
+                    sim.pipe += [("mma", op_dp(j, t + 1, tj + 1, ds2)), ("commit", "dp_full")]
+                    if t + 2 == n:
+                        sim.pipe.append(("commit", "v_empty"))
+            sq += n
+            tc += n
+            act += 1
+            sim.pipe.append(("commit", "dkdv_full"))  # after the item's last dK and dQ
+
+    def compute(h):
+        sq = tc = act = k = 0
+
+        def drain(tq):  # reads dQ(tq) out of the dP^T region, then frees it
+            yield wait("dq_full", tq)
+            if st["dP"][h] != ("dQ", tq):
+                raise Hazard(f"compute{h} drain({tq}): dP region holds {st['dP'][h]}")
+            yield STEP
+            st["dP"][h] = ("used", tq)
+            sim.arrive("dq_free")
+
+        while True:
+            it = yield from ring_reader(sim, ring, k, R)
+            k += 1
+            if it is None:
+                return
+            j, n = it
+            if n == 0:  # dK = dV = 0 written directly
+                continue
+            for t in range(n):
+                l = sq % LST
+                yield wait("s_full", tc)
+                yield wait(f"l_full{l}", sq // LST)
+                if st["S"][h] != ("S", tc) or st["l"][l] != (j, t):
+                    raise Hazard(f"compute{h}({j},{t}): S {st['S'][h]} rows {st['l'][l]}")
+                yield STEP  # first half of P^T
+                if t > 0:
+                    yield from drain(tc - 1)
+                yield STEP  # second half of P^T
+                st["S"][h] = ("P", tc)
+                sim.arrive("p_full")
+                yield wait("dp_full", tc)
+                if st["dP"][h] != ("dP", tc):
+                    raise Hazard(f"compute{h}({j},{t}): dP {st['dP'][h]}")
+                if st["dsm"][h] is not None and st["dsm"][h][0] != "used":
+                    raise Hazard(f"compute{h}({j},{t}): dS buffer still holds {st['dsm'][h]}")
+                yield STEP
+                st["dP"][h] = ("dS", tc)
+                st["dsm"][h] = ("dS", tc)
+                sim.arrive("ds_full")
+                sim.arrive(f"l_empty{l}")
+                sq += 1
+                tc += 1
+            yield from drain(tc - 1)
+            yield wait("dkdv_full", act)  # warpgroup 0 writes dV, warpgroup 1 dK
+            acc = "dV" if h == 0 else "dK"
+            if st[acc] != (j, n - 1):
+                raise Hazard(f"compute{h} epilogue({j}): {acc} holds {st[acc]}")
+            yield STEP
+            st[acc] = "free"
+            sim.arrive("dkdv_free")
+            act += 1
+
+    sim.run({"producer": producer(), "producer2": producer2(), "mma": mma(), "compute0": compute(0),
+             "compute1": compute(1)})
+
+
+MODELS = {"fwd": fwd_model, "dq": dq_model, "dkdv": dkdv_model, "fused": fused_model}
 
 
 def random_items(rng):

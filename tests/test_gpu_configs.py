@@ -128,6 +128,8 @@ def _identity_checks(w, inp, dk, dv):
 
 @pytest.mark.parametrize("name", ["doc8k", "sharequestion32k", "prefixwindow64k", "docblocksparse128k"])
 def test_config_sampled_parity(oracle_mod, name):
+    """Fused backward (the default mode); the split mode's agreement with it on the 8K and 32K
+    workloads is checked in test_gpu_kernels.py."""
     w = wl.CONFIGS[name]
     inp = wl.make_inputs(w)
     dev, m, o, lse, dq, dk, dv = run_full(w, inp)

@@ -75,13 +75,36 @@ MUTATIONS = [
        '                    if t + 2 == n:\n                        sim.pipe.append(("commit", "k_empty"))\n'
        '                yield wait("p_full", tj)\n                sim.pipe += [("mma", op_dv(j, t, tj, ds)), ("commit", f"do_empty{ds}")]\n')]),
     ("dkdv", "dV/dK handed to the epilogue before the item's last dK step",
-     [('                sim.pipe += [("mma", op_dk(j, t, tj, qs)), ("commit", f"q_empty{qs}")]',
+     [('                sim.pipe += [("mma", op_dk(j, t, tj, qs)), ("commit", f"q_empty{qs}")]\n'
+       '                if t + 1 < n:\n                    yield wait(f"do_full{ds2}"',
        '                if t == n - 1:\n                    sim.pipe.append(("commit", "dkdv_full"))\n'
-       '                sim.pipe += [("mma", op_dk(j, t, tj, qs)), ("commit", f"q_empty{qs}")]'),
+       '                sim.pipe += [("mma", op_dk(j, t, tj, qs)), ("commit", f"q_empty{qs}")]\n'
+       '                if t + 1 < n:\n                    yield wait(f"do_full{ds2}"'),
       ('            act += 1\n            sim.pipe.append(("commit", "dkdv_full"))\n', '            act += 1\n')]),
     ("dkdv", "Q stage released before its dK step",
-     [('                sim.pipe += [("mma", op_dk(j, t, tj, qs)), ("commit", f"q_empty{qs}")]',
-       '                sim.pipe += [("commit", f"q_empty{qs}"), ("mma", op_dk(j, t, tj, qs))]')]),
+     [('                sim.pipe += [("mma", op_dk(j, t, tj, qs)), ("commit", f"q_empty{qs}")]\n'
+       '                if t + 1 < n:\n                    yield wait(f"do_full{ds2}"',
+       '                sim.pipe += [("commit", f"q_empty{qs}"), ("mma", op_dk(j, t, tj, qs))]\n'
+       '                if t + 1 < n:\n                    yield wait(f"do_full{ds2}"')]),
+    ("fused", "dP^T(t+1) issued before dQ(t) was read out of its region",
+     [('                    yield wait("dq_free", tj)\n', '')]),
+    ("fused", "an item's first dP^T issued before the previous item's last dQ was read out",
+     [('            if tc > 0:\n                yield wait("dq_free", tc - 1)\n', '')]),
+    ("fused", "dQ(t) issued before dK(t) read dS^T(t) from the same TMEM columns",
+     [('                sim.pipe += [("mma", op_dk(j, t, tj, qs)), ("commit", f"q_empty{qs}")]\n'
+       '                sim.pipe += [("mma", op_dq(j, t, tj)), ("commit", "dq_full")]\n',
+       '                sim.pipe += [("mma", op_dq(j, t, tj)), ("commit", "dq_full")]\n'
+       '                sim.pipe += [("mma", op_dk(j, t, tj, qs)), ("commit", f"q_empty{qs}")]\n')]),
+    ("fused", "K released before the item's last dQ",
+     [('                sim.pipe += [("mma", op_dq(j, t, tj)), ("commit", "dq_full")]\n'
+       '                if t + 1 == n:\n                    sim.pipe.append(("commit", "k_empty"))\n',
+       '                if t + 1 == n:\n                    sim.pipe.append(("commit", "k_empty"))\n'
+       '                sim.pipe += [("mma", op_dq(j, t, tj)), ("commit", "dq_full")]\n')]),
+    ("fused", "dQ(t) not read out before P^T(t+1) is handed over",
+     [('                if t > 0:\n                    yield from drain(tc - 1)\n', '')]),
+    ("fused", "dQ region counted free after one warpgroup",
+     [('    for nm in ("p_full", "ds_full", "dq_free", "dkdv_free"):\n        sim.bar(nm, 2)\n',
+       '    for nm in ("p_full", "ds_full", "dkdv_free"):\n        sim.bar(nm, 2)\n    sim.bar("dq_free", 1)\n')]),
     ("dkdv", "P^T counted complete after one warpgroup",
      [('    for nm in ("p_full", "ds_full", "dkdv_free"):\n        sim.bar(nm, 2)\n',
        '    for nm in ("ds_full", "dkdv_free"):\n        sim.bar(nm, 2)\n    sim.bar("p_full", 1)\n')]),
