@@ -54,7 +54,10 @@ class FlashMaskError(RuntimeError):
 
 
 def lib_path() -> str:
-    return os.path.join(_HERE, _LIB_NAME)
+    """The library this process loads: libflashmask.so, or the checks build
+    (libflashmask_checks.so) when FLASHMASK_LIBRARY=checks."""
+    name = "libflashmask_checks.so" if os.environ.get("FLASHMASK_LIBRARY") == "checks" else _LIB_NAME
+    return os.path.join(_HERE, name)
 
 
 def load_library():
@@ -341,6 +344,8 @@ def get_status() -> int:
     """Synchronises the device; returns and clears the kernels' status word."""
     return int(load_library().flashmask_get_status())
 
+
+ERR_BOUNDS = -9
 
 _TIMEOUT_KERNELS = ("forward", "backward key side", "backward query side", "wait self-test", "fused backward")
 

@@ -77,7 +77,13 @@ __device__ __forceinline__ QItem decode_q_item(const BwdParams& p, int item) {
   QItem it{};
   it.item = item;
   if (item >= p.n_items2) return it;
-  const ItemCoord c = decode_q_item_coord(sh, p.forder[item]);
+  const int unit = p.forder[item];
+  if (kChecks && (unit < 0 || unit >= p.n_items2)) {
+    atomicCAS(p.status, 0, kDevErrBounds);
+    it.item = INT_MAX;  // ends the CTA's work
+    return it;
+  }
+  const ItemCoord c = decode_q_item_coord(sh, unit);
   it.b = c.b;
   it.h = c.hkv * sh.G + c.hg;
   it.hm = (sh.Hm == 1) ? 0 : it.h;
@@ -86,6 +92,18 @@ __device__ __forceinline__ QItem decode_q_item(const BwdParams& p, int item) {
   const size_t lrow = ((size_t)it.b * sh.Hm + it.hm) * sh.nQB + (c.t >> 1);
   it.cnt = (it.qt < sh.nQt) ? p.fcount[lrow] : 0;
   it.n = (it.qt < sh.nQt) ? p.qcount[lrow * 2 + it.g] : 0;  // per-q-tile count of the lists
+  if (kChecks) {  // the block's k-tile list and this q-tile's share of it
+    bool bad = it.cnt < 0 || it.cnt > sh.nKt || it.n < 0 || it.n > it.cnt;
+    for (int t = 0; !bad && t < it.cnt; ++t) {
+      const int e = it.list(p)[t];
+      bad = (e >> 8) < 0 || (e >> 8) >= sh.nKt;
+    }
+    if (bad) {
+      atomicCAS(p.status, 0, kDevErrBounds);
+      it.item = INT_MAX;
+      return it;
+    }
+  }
   return it;
 }
 

@@ -2,6 +2,8 @@
 // tile) and the walk over their non-skipped q-tiles, shared by the split
 // key-side kernel and the fused backward kernel.
 #pragma once
+#include <climits>
+
 #include "common.cuh"
 
 namespace fm {
@@ -18,7 +20,13 @@ __device__ __forceinline__ KvItem decode_kv_item(const BwdParams& p, int item) {
   KvItem it{};
   it.item = item;
   if (item >= p.n_items) return it;
-  const ItemCoord c = decode_kv_item_coord(sh, p.order[item]);
+  const int unit = p.order[item];
+  if (kChecks && (unit < 0 || unit >= p.n_items)) {
+    atomicCAS(p.status, 0, kDevErrBounds);
+    it.item = INT_MAX;  // ends the CTA's work
+    return it;
+  }
+  const ItemCoord c = decode_kv_item_coord(sh, unit);
   it.b = c.b;
   it.hkv = c.hkv;
   it.kt = c.t;
@@ -26,7 +34,21 @@ __device__ __forceinline__ KvItem decode_kv_item(const BwdParams& p, int item) {
   for (int gi = 0; gi < sh.G; ++gi) {
     const int h = it.hkv * sh.G + gi;
     const int hm = (sh.Hm == 1) ? 0 : h;
-    it.total += p.bcount[((size_t)it.b * sh.Hm + hm) * sh.nKt + it.kt];
+    const size_t lrow = ((size_t)it.b * sh.Hm + hm) * sh.nKt + it.kt;
+    const int cnt = p.bcount[lrow];
+    if (kChecks) {  // the q-tile list: a count within [0, nQt], entries in range and not skipped
+      bool bad = cnt < 0 || cnt > sh.nQt;
+      for (int t = 0; !bad && t < cnt; ++t) {
+        const int e = p.blist[lrow * sh.nQt + t];
+        bad = (e >> 2) < 0 || (e >> 2) >= sh.nQt || (e & 3) == kClsSkip || (e & 3) > kClsFull;
+      }
+      if (bad) {
+        atomicCAS(p.status, 0, kDevErrBounds);
+        it.item = INT_MAX;
+        return it;
+      }
+    }
+    it.total += cnt;
   }
   return it;
 }

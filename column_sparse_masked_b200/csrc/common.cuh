@@ -8,6 +8,18 @@
 namespace fm {
 
 constexpr int kTile = 128;  // rows of a q-tile and columns of a k-tile
+
+// Checks build (compiled with -DFLASHMASK_CHECKS=1 into a library of its own):
+// mask values outside [0, Nq] and out-of-range scheduler indices (work orders,
+// list counts and entries) are recorded as FLASHMASK_ERR_BOUNDS in the status
+// word; a work item that fails a check is not processed (it ends the CTA's
+// work), so no access is made with a bad index.
+#ifdef FLASHMASK_CHECKS
+constexpr bool kChecks = true;
+#else
+constexpr bool kChecks = false;
+#endif
+constexpr int kDevErrBounds = -9;
 constexpr int kClsSkip = 0, kClsPartial = 1, kClsFull = 2;
 
 // Index of the 8 entries of a per-(batch, mask head, k-tile) summary.
@@ -134,6 +146,8 @@ __host__ __device__ __forceinline__ ItemCoord decode_q_item_coord(const Shape& s
 struct MaskPrepParams {
   const int32_t *lts, *lte, *uts, *ute;  // [B, Hm, Nk]; a null pair = empty intervals
   int B, Hm, Nk, nKt;
+  int Nq;        // checks build: mask values must lie in [0, Nq]
+  int* status;   // checks build: where a bad value is recorded
   int4* rec;    // [B, Hm, nKt*128] {LTS, LTE, UTS, UTE}; padded columns hide every row
   int* ksum;    // [B, Hm, nKt, 8]
 };

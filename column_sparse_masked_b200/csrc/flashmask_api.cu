@@ -207,10 +207,12 @@ float resolve_scale(float scale, int d) { return scale > 0.f ? scale : 1.0f / st
 // Steps shared by forward, backward and classify: padded boundary records
 // and the per-k-tile block summary.
 MaskPrepParams prep_params(const Shape& s, const WsLayout& L, uint8_t* ws, const int32_t* lts, const int32_t* lte,
-                           const int32_t* uts, const int32_t* ute) {
+                           const int32_t* uts, const int32_t* ute, int* status) {
   MaskPrepParams mp{};
   mp.lts = lts; mp.lte = lte; mp.uts = uts; mp.ute = ute;
   mp.B = s.B; mp.Hm = s.Hm; mp.Nk = s.Nk; mp.nKt = s.nKt;
+  mp.Nq = s.Nq;
+  mp.status = status;
   mp.rec = reinterpret_cast<int4*>(ws + L.rec);
   mp.ksum = reinterpret_cast<int*>(ws + L.ksum);
   return mp;
@@ -336,7 +338,7 @@ int flashmask_fwd(const void* q, const void* k, const void* v, const int32_t* lt
     FM_TRY(make_map(&tk, workspace, 1, 1, 1, s.d));
     tv = tk;
   }
-  const MaskPrepParams mp = prep_params(s, L, ws, lts, lte, uts, ute);
+  const MaskPrepParams mp = prep_params(s, L, ws, lts, lte, uts, ute, di.status);
   FM_CUDA(launch_mask_prep(mp, st));
 
   PlanParams pp{};
@@ -447,7 +449,7 @@ int flashmask_bwd(const void* q, const void* k, const void* v, const void* o, co
     FM_CUDA(launch_bwd_pre(bp, pre_blocks, st));
   }
 
-  const MaskPrepParams mp = prep_params(s, L, ws, lts, lte, uts, ute);
+  const MaskPrepParams mp = prep_params(s, L, ws, lts, lte, uts, ute, di.status);
   FM_CUDA(launch_mask_prep(mp, st));
 
   if (fused) {
@@ -605,7 +607,7 @@ int flashmask_classify(const int32_t* lts, const int32_t* lte, const int32_t* ut
   FM_TRY(current_device(&di));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  const MaskPrepParams mp = prep_params(s, L, ws, lts, lte, uts, ute);
+  const MaskPrepParams mp = prep_params(s, L, ws, lts, lte, uts, ute, di.status);
   FM_CUDA(launch_mask_prep(mp, st));
   PlanParams pp{};
   pp.s = s;
@@ -766,6 +768,8 @@ const char* flashmask_strerror(int code) {
       return g_last_cuda_error[0] ? g_last_cuda_error : "CUDA runtime or launch failure";
     case FLASHMASK_ERR_TIMEOUT: return "a device-side bounded wait timed out";
     case FLASHMASK_ERR_NO_DEVICE: return "no sm_100 (B200-class) device is current";
+    case FLASHMASK_ERR_BOUNDS:
+      return "a mask value outside [0, Nq] or an internal index out of range (checks build)";
     case FLASHMASK_ERR_TOO_LARGE:
       return "problem too large for flashmask_fwd_noalloc: its forward workspace exceeds "
              "FLASHMASK_NOALLOC_SCRATCH_BYTES (16 MiB); use flashmask_fwd with a workspace";

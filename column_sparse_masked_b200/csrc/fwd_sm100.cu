@@ -68,7 +68,13 @@ __device__ __forceinline__ FwdItem decode_fwd(const FwdParams& p, int item) {
   FwdItem it{};
   it.item = item;
   if (item >= p.n_items) return it;
-  const ItemCoord c = decode_fwd_item(sh, p.order[item]);
+  const int unit = p.order[item];
+  if (kChecks && (unit < 0 || unit >= p.n_items)) {
+    atomicCAS(p.status, 0, kDevErrBounds);
+    it.item = INT_MAX;  // ends the CTA's work
+    return it;
+  }
+  const ItemCoord c = decode_fwd_item(sh, unit);
   it.b = c.b;
   it.qb = c.t;
   it.hkv = c.hkv;
@@ -76,6 +82,18 @@ __device__ __forceinline__ FwdItem decode_fwd(const FwdParams& p, int item) {
   it.hm = (sh.Hm == 1) ? 0 : it.h;
   const size_t lrow = ((size_t)it.b * sh.Hm + it.hm) * sh.nQB + it.qb;
   it.n = p.fcount[lrow];
+  if (kChecks) {  // the k-tile list: a count within [0, nKt], entries in range
+    bool bad = it.n < 0 || it.n > sh.nKt;
+    for (int t = 0; !bad && t < it.n; ++t) {
+      const int e = p.flist[lrow * sh.nKt + t];
+      bad = (e >> 8) < 0 || (e >> 8) >= sh.nKt || (e & 3) > kClsFull || ((e >> 2) & 3) > kClsFull;
+    }
+    if (bad) {
+      atomicCAS(p.status, 0, kDevErrBounds);
+      it.item = INT_MAX;
+      return it;
+    }
+  }
   it.e0 = it.n > 0 ? p.flist[lrow * sh.nKt] : 0;
   return it;
 }

@@ -37,6 +37,11 @@ __global__ void __launch_bounds__(128) mask_prep_kernel(MaskPrepParams p) {
     r.w = p.ute ? p.ute[idx] : 0;
   }
   p.rec[(row * p.nKt + kt) * kTile + t] = r;
+  if (kChecks && real && p.status) {
+    const bool bad = (p.lts && (r.x < 0 || r.x > p.Nq)) || (p.lte && (r.y < 0 || r.y > p.Nq)) ||
+                     (p.uts && (r.z < 0 || r.z > p.Nq)) || (p.ute && (r.w < 0 || r.w > p.Nq));
+    if (bad) atomicCAS(p.status, 0, kDevErrBounds);
+  }
   // min/max over the real columns of the tile
   int v[8];
   v[kMnLts] = real ? r.x : INT_MAX; v[kMxLts] = real ? r.x : INT_MIN;

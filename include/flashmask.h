@@ -36,6 +36,12 @@
  *  - Tiles are 128 query rows x 128 key columns.
  *  - Device-side failures (a bounded wait that timed out) are recorded in a
  *    per-device status word that flashmask_get_status() reads and clears.
+ *  - Mask values are applied literally, in or out of [0, Nq].  The checks
+ *    build of the library (libflashmask_checks.so, the same entry points
+ *    compiled with FLASHMASK_CHECKS) also records FLASHMASK_ERR_BOUNDS in the
+ *    status word for a mask value outside [0, Nq] and for any work-order or
+ *    work-list index out of range; a work item that fails a check is skipped,
+ *    so no access is made with a bad index.
  */
 #ifndef FLASHMASK_H_
 #define FLASHMASK_H_
@@ -56,6 +62,8 @@ extern "C" {
 #define FLASHMASK_ERR_TIMEOUT (-6)     /* a kernel's bounded wait expired (status word)   */
 #define FLASHMASK_ERR_NO_DEVICE (-7)   /* no sm_100 device current                        */
 #define FLASHMASK_ERR_TOO_LARGE (-8)   /* problem needs more than the static no-alloc scratch */
+#define FLASHMASK_ERR_BOUNDS (-9)      /* checks build: mask value outside [0, Nq], or an internal
+                                          index out of range (status word)                   */
 
 /* Problem shape.  B batch, Hq query heads, Hkv key/value heads, Hm mask heads
  * (1 or Hq), Nq query rows, Nk key columns, d head dimension. */

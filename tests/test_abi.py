@@ -101,3 +101,15 @@ def test_localize_argument_checks(lib):
     a = (ctypes.c_int32 * 2)(0, 5)
     b = (ctypes.c_int32 * 2)(10, 20)  # overlapping chunks
     assert lib.flashmask_localize_multi(None, None, ctypes.c_int64(4), a, b, 2, None) == -1
+
+
+def test_checks_build_exports_every_declared_symbol():
+    """The checks build (FLASHMASK_CHECKS) has the same C ABI."""
+    from column_sparse_masked_b200 import build
+
+    path = build.build(checks=True)
+    chk = ctypes.CDLL(path)
+    for n in declared_functions():
+        assert hasattr(chk, n), n
+    chk.flashmask_strerror.restype = ctypes.c_char_p
+    assert b"checks build" in chk.flashmask_strerror(-9)
