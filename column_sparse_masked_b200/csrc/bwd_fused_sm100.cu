@@ -562,35 +562,54 @@ __global__ void __launch_bounds__(fb::kThreads, 1)
 
 // ----------------------------------------------------------------------------
 // dQ finalize: dQ = bf16(scale * acc), from the tiled fp32 accumulator to the
-// [B, Nq, Hq, D] layout.  Thread = (tile, row, 8-column group): it reads two
-// 16-byte chunks (coalesced across the warp's 32 consecutive rows) and writes
-// 16 bytes of its row.  HBM-bound.
+// [B, Nq, Hq, D] layout.  One CTA per (batch, q-head, q-tile), 64 columns at a
+// time through shared memory: the accumulator is read in its own order (each
+// warp 512 contiguous bytes), rows are written as whole 128-byte segments.
+// HBM-bound: 4 bytes read and 2 written per element.
 // ----------------------------------------------------------------------------
 template <int D>
 __global__ void __launch_bounds__(256) fm_dq_finalize_kernel(BwdParams p) {
   const Shape& sh = p.s;
-  constexpr int kGroups = D / 8;
-  const int64_t total = (int64_t)sh.B * sh.Hq * sh.nQt * kTile * kGroups;
-  for (int64_t t = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; t < total; t += (int64_t)gridDim.x * blockDim.x) {
-    const int r = (int)(t % kTile);
-    const int64_t rest = t / kTile;
-    const int g = (int)(rest % kGroups);
-    const int64_t tile = rest / kGroups;  // (b * Hq + h) * nQt + qt
-    const int qt = (int)(tile % sh.nQt);
-    const int64_t bh = tile / sh.nQt;
+  constexpr int kPad = 68;  // row stride in floats (64 + 4): 16-byte aligned, spreads banks
+  __shared__ __align__(16) float tile[kTile * kPad];
+  const int64_t n_tiles = (int64_t)sh.B * sh.Hq * sh.nQt;
+  const int t = threadIdx.x;
+  const float sc = p.scale;
+  for (int64_t tix = blockIdx.x; tix < n_tiles; tix += gridDim.x) {
+    const int qt = (int)(tix % sh.nQt);
+    const int64_t bh = tix / sh.nQt;
     const int h = (int)(bh % sh.Hq), b = (int)(bh / sh.Hq);
-    const int i = qt * kTile + r;
-    if (i >= sh.Nq) continue;
-    const float* acc = p.dqacc + tile * ((int64_t)kTile * D);
-    const float4 a = *reinterpret_cast<const float4*>(acc + ((size_t)(2 * g) * kTile + r) * 4);
-    const float4 c = *reinterpret_cast<const float4*>(acc + ((size_t)(2 * g + 1) * kTile + r) * 4);
-    const float sc = p.scale;
-    uint4 o;
-    o.x = pack_bf16x2(a.x * sc, a.y * sc);
-    o.y = pack_bf16x2(a.z * sc, a.w * sc);
-    o.z = pack_bf16x2(c.x * sc, c.y * sc);
-    o.w = pack_bf16x2(c.z * sc, c.w * sc);
-    *reinterpret_cast<uint4*>(p.dq + (((size_t)b * sh.Nq + i) * sh.Hq + h) * D + g * 8) = o;
+    const float4* acc = reinterpret_cast<const float4*>(p.dqacc + tix * ((int64_t)kTile * D));
+#pragma unroll
+    for (int half = 0; half < D / 64; ++half) {
+      // 16 four-column chunks x 128 rows of this half: 2048 float4, 8 per thread
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int f = t + 256 * i;
+        const int c = f >> 7, r = f & 127;
+        const float4 x = acc[(half * 16 + c) * kTile + r];
+        *reinterpret_cast<float4*>(&tile[r * kPad + 4 * c]) = x;
+      }
+      __syncthreads();
+      // 128 rows x 64 columns as bf16: 8 threads per row, 16 bytes each
+#pragma unroll
+      for (int pass = 0; pass < 4; ++pass) {
+        const int r = pass * 32 + (t >> 3), seg = t & 7;
+        const int i = qt * kTile + r;
+        if (i < sh.Nq) {
+          const float* src = &tile[r * kPad + seg * 8];
+          const float4 a = *reinterpret_cast<const float4*>(src);
+          const float4 c = *reinterpret_cast<const float4*>(src + 4);
+          uint4 o;
+          o.x = pack_bf16x2(a.x * sc, a.y * sc);
+          o.y = pack_bf16x2(a.z * sc, a.w * sc);
+          o.z = pack_bf16x2(c.x * sc, c.y * sc);
+          o.w = pack_bf16x2(c.z * sc, c.w * sc);
+          *reinterpret_cast<uint4*>(p.dq + (((size_t)b * sh.Nq + i) * sh.Hq + h) * D + half * 64 + seg * 8) = o;
+        }
+      }
+      __syncthreads();
+    }
   }
 }
 
@@ -614,10 +633,10 @@ cudaError_t launch_bwd_fused(const BwdParams& p, const CUtensorMap& tq, const CU
 }
 
 cudaError_t launch_dq_finalize(const BwdParams& p, int max_blocks, cudaStream_t st) {
-  const int64_t total = (int64_t)p.s.B * p.s.Hq * p.s.nQt * kTile * (p.s.d / 8);
-  if (total == 0) return cudaSuccess;
-  int64_t blocks = (total + 255) / 256;
-  if (blocks > max_blocks) blocks = max_blocks;
+  const int64_t n_tiles = (int64_t)p.s.B * p.s.Hq * p.s.nQt;
+  if (n_tiles == 0) return cudaSuccess;
+  int64_t blocks = n_tiles;
+  if (blocks > max_blocks) blocks = max_blocks;  // grid-stride loop over the tiles
   const int prof = profile_begin(5, st);
   note_launch();
   if (p.s.d == 128)
