@@ -32,6 +32,7 @@ from ._binding import (  # noqa: F401
     load_library,
     localize,
     localize_multi,
+    merge_partials,
     profiler_enable,
     profiler_read,
     get_bwd_mode,
@@ -46,6 +47,6 @@ from ._binding import (  # noqa: F401
 
 __all__ = [
     "FlashMaskError", "balance_chunks", "classify", "count_unmasked", "flashmask_attention", "fwd", "bwd", "get_status", "get_timeout_info",
-    "launch_count", "lib_path", "load_library", "localize", "localize_multi", "profiler_enable", "profiler_read", "get_bwd_mode", "set_bwd_mode", "set_max_ctas", "set_wait_limit_ns", "test_wait_timeout", "tile_costs",
+    "launch_count", "lib_path", "load_library", "localize", "localize_multi", "merge_partials", "profiler_enable", "profiler_read", "get_bwd_mode", "set_bwd_mode", "set_max_ctas", "set_wait_limit_ns", "test_wait_timeout", "tile_costs",
     "version", "workspace_size",
 ]

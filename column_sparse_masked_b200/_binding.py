@@ -26,6 +26,7 @@ _SIGS = {
     "flashmask_localize_multi": (ctypes.c_int, [_P, _P, ctypes.c_int64, _P, _P, ctypes.c_int32, _P]),
     "flashmask_count_unmasked": (ctypes.c_int, [_P, _P, _P, _P, _DIMS, _P, _P]),
     "flashmask_tile_costs": (ctypes.c_int, [_P, _P, _P, _P, _DIMS, _P, _P]),
+    "flashmask_merge_partials": (ctypes.c_int, [_P, _P, ctypes.c_int32, _DIMS, _P, _P, _P]),
     "flashmask_balance_chunks": (ctypes.c_int, [_P, ctypes.c_int32, ctypes.c_int32, _P, _P]),
     "flashmask_set_max_ctas": (ctypes.c_int, [ctypes.c_int32]),
     "flashmask_set_bwd_mode": (ctypes.c_int, [ctypes.c_int32]),
@@ -301,6 +302,29 @@ def tile_costs(lts, lte, uts, ute, Nq: int, Hq: int) -> torch.Tensor:
     rc = lib.flashmask_tile_costs(*[_ptr(x) for x in vecs], ctypes.byref(dm), _ptr(out), _stream(ref.device))
     _check(rc, "flashmask_tile_costs")
     return out[: -(-int(Nq) // 128)]
+
+
+def merge_partials(o_parts: Sequence[torch.Tensor], lse_parts: Sequence[torch.Tensor]):
+    """Attention over the union of disjoint key sets from per-set results (o_c, lse_c):
+    lse = ln sum exp(lse_c), o = sum exp(lse_c - lse) o_c, per row.  Returns (o, lse)."""
+    lib = load_library()
+    n = len(o_parts)
+    if n < 1 or n != len(lse_parts):
+        raise ValueError("need as many lse parts as o parts (at least one)")
+    B, Nq, Hq, d = o_parts[0].shape
+    for i, (oc, lc) in enumerate(zip(o_parts, lse_parts)):
+        _shaped(f"o_parts[{i}]", oc, (B, Nq, Hq, d), torch.bfloat16)
+        _shaped(f"lse_parts[{i}]", lc, (B, Hq, Nq), torch.float32)
+    _on_device(o_parts[0].device, [(f"o{i}", t) for i, t in enumerate(o_parts)] +
+               [(f"l{i}", t) for i, t in enumerate(lse_parts)])
+    o = torch.empty_like(o_parts[0])
+    lse = torch.empty_like(lse_parts[0])
+    op = (ctypes.c_void_p * n)(*[t.data_ptr() for t in o_parts])
+    lp = (ctypes.c_void_p * n)(*[t.data_ptr() for t in lse_parts])
+    dm = _dims(B, Hq, 1, 1, Nq, 0, d)
+    rc = lib.flashmask_merge_partials(op, lp, n, ctypes.byref(dm), _ptr(o), _ptr(lse), _stream(o.device))
+    _check(rc, "flashmask_merge_partials")
+    return o, lse
 
 
 def set_max_ctas(n: int) -> None:

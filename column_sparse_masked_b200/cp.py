@@ -19,6 +19,13 @@ point-to-point schedule:
             the dK/dV contributions of every received chunk back to the
             chunk's owner, which sums them (fp32) with its own.
 
+With ``overlap=True`` the forward attends the rank's own key chunk while the
+exchange is in flight (its rows against its own keys need nothing from other
+ranks), then each received chunk, and merges the per-chunk results per row
+(``flashmask_merge_partials``: lse = ln sum exp(lse_c), o = sum exp(lse_c -
+lse) o_c, exact up to the rounding of the bf16 partials).  The backward then
+runs once on the gathered K/V with the merged O and LSE.
+
 The exchange uses torch.distributed point-to-point operations (NCCL between
 GPUs, one process per GPU; gloo on CPU for the host-logic tests) into this
 rank's own buffers; no kernel reads another GPU's memory.  A plain
@@ -80,6 +87,9 @@ class LibraryOps:
 
     def bwd(self, q, k, v, o, lse, do, masks, scale):
         return self.b.bwd(q, k, v, o, lse, do, *masks, scale=scale)
+
+    def merge(self, o_parts, lse_parts):
+        return self.b.merge_partials(o_parts, lse_parts)
 
 
 def equal_bounds(N: int, world: int) -> List[Tuple[int, int]]:
@@ -145,10 +155,12 @@ class ContextParallelAttention:
     receive with NaN (a check that pruned chunks are never read).
     """
 
-    def __init__(self, plan: CPPlan, rank: int, ops=None, group=None, poison_unreceived: bool = False):
+    def __init__(self, plan: CPPlan, rank: int, ops=None, group=None, poison_unreceived: bool = False,
+                 overlap: bool = False):
         self.plan, self.rank, self.group = plan, rank, group
         self.ops = ops or LibraryOps()
         self.poison = poison_unreceived
+        self.overlap = overlap
         self.peer = (lambda r: r) if group is None else (lambda r: _group_rank(group, r))
 
     def forward(self, q, k, v, masks, scale: Optional[float] = None):
@@ -177,12 +189,29 @@ class ContextParallelAttention:
             ops += [dist.P2POp(dist.irecv, kb, self.peer(src), self.group),
                     dist.P2POp(dist.irecv, vb, self.peer(src), self.group)]
             recv.append((ac, bc, kb, vb))
-        _p2p(ops)
-        for ac, bc, kb, vb in recv:
-            k_full[:, ac:bc] = kb
-            v_full[:, ac:bc] = vb
         loc = [None if m is None else self.ops.localize(m, a, b) for m in masks]
-        o, lse = self.ops.fwd(q, k_full, v_full, loc, scale)
+        if not self.overlap:
+            _p2p(ops)
+            for ac, bc, kb, vb in recv:
+                k_full[:, ac:bc] = kb
+                v_full[:, ac:bc] = vb
+            o, lse = self.ops.fwd(q, k_full, v_full, loc, scale)
+        else:
+            works = dist.batch_isend_irecv(ops) if ops else []
+            # own rows against own keys while the exchange is in flight
+            own = [None if m is None else self.ops.localize(m[:, :, a:b].contiguous(), a, b) for m in masks]
+            parts = [self.ops.fwd(q, k, v, own, scale)]
+            for wk in works:
+                wk.wait()
+            for ac, bc, kb, vb in recv:  # then each received chunk, merged per row
+                k_full[:, ac:bc] = kb
+                v_full[:, ac:bc] = vb
+                loc_c = [None if m is None else self.ops.localize(m[:, :, ac:bc].contiguous(), a, b) for m in masks]
+                parts.append(self.ops.fwd(q, kb, vb, loc_c, scale))
+            if len(parts) == 1:
+                o, lse = parts[0]
+            else:
+                o, lse = self.ops.merge([x[0] for x in parts], [x[1] for x in parts])
         ctx = {"q": q, "k_full": k_full, "v_full": v_full, "loc": loc, "o": o, "lse": lse, "scale": scale}
         return o, lse, ctx
 

@@ -176,6 +176,16 @@ struct SortParams {
   int n_buckets;  // > 0: counting sort over (wave, cost) buckets; 0: bitonic sort
 };
 
+// Partial attention results over disjoint key sets, merged per row.
+constexpr int kMaxMergeParts = 16;
+struct MergeParams {
+  const __nv_bfloat16* o[kMaxMergeParts];  // [B, Nq, Hq, d]
+  const float* lse[kMaxMergeParts];        // [B, Hq, Nq]
+  int n, B, Nq, Hq, d;
+  __nv_bfloat16* out_o;
+  float* out_lse;
+};
+
 struct FwdParams {
   Shape s;
   float scale_log2;          // scale * log2(e)

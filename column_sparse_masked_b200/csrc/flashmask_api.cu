@@ -679,6 +679,32 @@ int flashmask_tile_costs(const int32_t* lts, const int32_t* lte, const int32_t* 
   return FLASHMASK_OK;
 }
 
+int flashmask_merge_partials(const void* const* o_parts, const float* const* lse_parts, int32_t n,
+                             const flashmask_dims* dims, void* o, float* lse, void* stream) {
+  NvtxRange nvtx("flashmask_merge_partials");
+  FM_TRY(check_dims(dims));
+  if (n < 1 || n > kMaxMergeParts || !o_parts || !lse_parts) return FLASHMASK_ERR_INVALID_ARG;
+  const flashmask_dims& d = *dims;
+  if ((int64_t)d.B * d.Nq == 0) return FLASHMASK_OK;
+  if (!o || !lse) return FLASHMASK_ERR_INVALID_ARG;
+  MergeParams mp{};
+  for (int c = 0; c < n; ++c) {
+    if (!o_parts[c] || !lse_parts[c]) return FLASHMASK_ERR_INVALID_ARG;
+    if (!aligned16(o_parts[c]) || !aligned16(lse_parts[c])) return FLASHMASK_ERR_ALIGN;
+    mp.o[c] = static_cast<const __nv_bfloat16*>(o_parts[c]);
+    mp.lse[c] = lse_parts[c];
+  }
+  if (!aligned16(o) || !aligned16(lse)) return FLASHMASK_ERR_ALIGN;
+  DeviceInfo di;
+  FM_TRY(current_device(&di));
+  mp.n = n;
+  mp.B = d.B; mp.Nq = d.Nq; mp.Hq = d.Hq; mp.d = d.d;
+  mp.out_o = static_cast<__nv_bfloat16*>(o);
+  mp.out_lse = lse;
+  FM_CUDA(launch_merge_partials(mp, 64 * di.sm_count, static_cast<cudaStream_t>(stream)));
+  return FLASHMASK_OK;
+}
+
 int flashmask_set_bwd_mode(int32_t mode) {
   if (mode != FLASHMASK_BWD_FUSED && mode != FLASHMASK_BWD_SPLIT) return FLASHMASK_ERR_INVALID_ARG;
   g_bwd_mode.store(mode);

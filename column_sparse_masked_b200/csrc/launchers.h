@@ -24,6 +24,7 @@ cudaError_t launch_count_unmasked(const MaskPrepParams& p, int Hq, int Nq, int64
 // Unmasked pairs of each 128-row q-tile over batches and Hq q-heads: out[ceil(Nq/128)].
 cudaError_t launch_tile_costs(const MaskPrepParams& p, int Hq, int Nq, int64_t* out, cudaStream_t st);
 cudaError_t launch_wait_timeout(int* status, uint64_t limit_ns, cudaStream_t st);
+cudaError_t launch_merge_partials(const MergeParams& p, int max_blocks, cudaStream_t st);
 
 // Forward / backward attention kernels.  `grid` is the persistent CTA count.
 cudaError_t launch_fwd(const FwdParams& p, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,

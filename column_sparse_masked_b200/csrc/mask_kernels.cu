@@ -8,7 +8,9 @@
 // per key column), tiles decided from O(n) data, and the exchange-free
 // clip-shift-max localisation of a query chunk.
 #include <cuda_runtime.h>
+#include <cuda_bf16.h>
 #include <climits>
+#include <cmath>
 #include <cstdint>
 
 #include "common.cuh"
@@ -562,6 +564,70 @@ cudaError_t launch_tile_costs(const MaskPrepParams& p, int Hq, int Nq, int64_t* 
 cudaError_t launch_wait_timeout(int* status, uint64_t limit_ns, cudaStream_t st) {
   { note_launch(); wait_timeout_kernel<<<1, 32, 0, st>>>(status, limit_ns);
   }
+  return cudaGetLastError();
+}
+
+}  // namespace fm
+
+namespace fm {
+
+// ----------------------------------------------------------------------------
+// 7. merge of partial attention results over disjoint key sets (context
+//    parallelism with overlap: each received key chunk is attended as soon as
+//    it lands).  Per row: lse = log(sum_c exp(lse_c)), o = sum_c exp(lse_c - lse) o_c.
+//    16 threads per (batch, row, head), each 8 columns (16-byte loads/stores).
+// ----------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) merge_partials_kernel(MergeParams p) {
+  constexpr float kLog2e = 1.4426950408889634f, kLn2 = 0.69314718055994531f;
+  const int lanes = p.d / 8;  // threads per row
+  const int64_t rows = (int64_t)p.B * p.Nq * p.Hq;
+  const int64_t t0 = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
+  for (int64_t t = t0; t < rows * lanes; t += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = t / lanes;  // row index in [B, Nq, Hq] order
+    const int sl = (int)(t % lanes);
+    const int h = (int)(r % p.Hq);
+    const int64_t bi = r / p.Hq;
+    const int i = (int)(bi % p.Nq), b = (int)(bi / p.Nq);
+    const size_t lidx = ((size_t)b * p.Hq + h) * p.Nq + i;
+    float m = -INFINITY;
+    for (int c = 0; c < p.n; ++c) m = fmaxf(m, p.lse[c][lidx]);
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    float lse_out = -INFINITY;
+    if (m != -INFINITY) {
+      float wsum = 0.f;
+      for (int c = 0; c < p.n; ++c) wsum += exp2f((p.lse[c][lidx] - m) * kLog2e);
+      const float inv = 1.f / wsum;
+      for (int c = 0; c < p.n; ++c) {
+        const float wgt = exp2f((p.lse[c][lidx] - m) * kLog2e) * inv;
+        if (wgt == 0.f) continue;
+        const uint4 v = *reinterpret_cast<const uint4*>(p.o[c] + r * p.d + sl * 8);
+        const __nv_bfloat162* v2 = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const float2 f = __bfloat1622float2(v2[u]);
+          acc[2 * u] = fmaf(wgt, f.x, acc[2 * u]);
+          acc[2 * u + 1] = fmaf(wgt, f.y, acc[2 * u + 1]);
+        }
+      }
+      lse_out = m + log2f(wsum) * kLn2;
+    }
+    uint4 out;
+    out.x = pack_bf16x2(acc[0], acc[1]);
+    out.y = pack_bf16x2(acc[2], acc[3]);
+    out.z = pack_bf16x2(acc[4], acc[5]);
+    out.w = pack_bf16x2(acc[6], acc[7]);
+    *reinterpret_cast<uint4*>(p.out_o + r * p.d + sl * 8) = out;
+    if (sl == 0) p.out_lse[lidx] = lse_out;
+  }
+}
+
+cudaError_t launch_merge_partials(const MergeParams& p, int max_blocks, cudaStream_t st) {
+  const int64_t threads = (int64_t)p.B * p.Nq * p.Hq * (p.d / 8);
+  if (threads == 0) return cudaSuccess;
+  int64_t blocks = (threads + 255) / 256;
+  if (blocks > max_blocks) blocks = max_blocks;
+  note_launch();
+  merge_partials_kernel<<<(unsigned)blocks, 256, 0, st>>>(p);
   return cudaGetLastError();
 }
 

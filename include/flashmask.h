@@ -213,6 +213,21 @@ int flashmask_count_unmasked(const int32_t* lts, const int32_t* lte, const int32
                              const flashmask_dims* dims, int64_t* pairs, void* stream);
 
 /*
+ * Merge of partial attention results over DISJOINT key sets (the same rows
+ * attended to n separate key chunks, e.g. by a context-parallel rank as each
+ * chunk arrives; same page and section: compute/communication overlap).  Per
+ * row of every (batch, q-head): lse = ln(sum_c exp(lse_c)) and
+ * o = sum_c exp(lse_c - lse) * o_c -- exactly the attention over the union of
+ * the key sets, up to the rounding of the bf16 partials.  Rows with
+ * lse_c = -inf for every c get o = 0, lse = -inf.  o_parts / lse_parts: HOST
+ * arrays of n (1..16) device pointers to bf16 [B, Nq, Hq, d] and fp32
+ * [B, Hq, Nq]; o, lse: outputs of the same shapes (not aliasing any part).  Uses
+ * dims->B, Hq, Nq, d.
+ */
+int flashmask_merge_partials(const void* const* o_parts, const float* const* lse_parts, int32_t n,
+                             const flashmask_dims* dims, void* o, float* lse, void* stream);
+
+/*
  * Work of each 128-row query tile: costs[t] (device int64, ceil(Nq/128)
  * entries, 16-byte aligned) receives the number of unmasked (i, j) pairs with
  * row i in [128 t, min(128 t + 128, Nq)), over all batches, all Hq query heads

@@ -49,6 +49,18 @@ class OracleOps:
         dq, dk, dv = self.o.attention_backward(q, k, v, do, *masks, scale=scale)
         return torch.from_numpy(dq), torch.from_numpy(dk), torch.from_numpy(dv)
 
+    def merge(self, o_parts, lse_parts):
+        """The merge identity in fp64: lse = ln sum exp(lse_c), o = sum exp(lse_c - lse) o_c."""
+        L = np.stack([x.numpy() for x in lse_parts])            # [n, B, Hq, Nq]
+        m = L.max(0)
+        fin = np.isfinite(m)
+        w = np.where(fin[None], np.exp(L - np.where(fin, m, 0)[None]), 0.0)
+        s_ = w.sum(0)
+        lse = np.where(fin, np.where(fin, m, 0) + np.log(np.where(fin, s_, 1)), -np.inf)
+        wn = w / np.where(fin, s_, 1)[None]                       # [n, B, Hq, Nq]
+        o = sum(wn[c].transpose(0, 2, 1)[..., None] * o_parts[c].numpy() for c in range(len(o_parts)))
+        return torch.from_numpy(o), torch.from_numpy(lse)
+
 
 def _free_port():
     s = socket.socket()
@@ -77,7 +89,7 @@ def _case(seed, N=1024, B=1, Hq=2, Hkv=1, d=16, kind="doc"):
     return q, k, v, do, masks
 
 
-def _worker(rank, world, port, seed, kind, out):
+def _worker(rank, world, port, seed, kind, out, overlap=False):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     from datetime import timedelta
 
@@ -88,7 +100,7 @@ def _worker(rank, world, port, seed, kind, out):
         N = q.shape[1]
         plan = cp.make_plan(masks, N, cp.equal_bounds(N, world), ops=ops)
         a, b = plan.bounds[rank]
-        att = cp.ContextParallelAttention(plan, rank, ops=ops)
+        att = cp.ContextParallelAttention(plan, rank, ops=ops, overlap=overlap)
         o, lse, ctx = att.forward(q[:, a:b].contiguous(), k[:, a:b].contiguous(), v[:, a:b].contiguous(), masks)
         dq, dk, dv = att.backward(ctx, do[:, a:b].contiguous())
         out[rank] = {"o": o.numpy(), "lse": lse.numpy(), "dq": dq.numpy(), "dk": dk.numpy(), "dv": dv.numpy(),
@@ -105,9 +117,13 @@ def _dense_visible(masks, N):
 
 
 @pytest.mark.timeout(600)
-@pytest.mark.parametrize("world,kind,seed", [(2, "doc", 1), (4, "doc", 2), (4, "blocksparse", 3), (4, "causal", 4),
-                                             (4, "docs_aligned", 5)])
-def test_context_parallel_equals_full_run(world, kind, seed):
+@pytest.mark.parametrize("world,kind,seed,overlap", [(2, "doc", 1, False), (4, "doc", 2, False),
+                                                     (4, "blocksparse", 3, False), (4, "causal", 4, False),
+                                                     (4, "docs_aligned", 5, False), (2, "doc", 6, True),
+                                                     (4, "blocksparse", 7, True)])
+def test_context_parallel_equals_full_run(world, kind, seed, overlap):
+    """overlap=True: each rank attends its own chunk while the exchange runs, then each received
+    chunk, and merges the per-chunk results (the compute/communication overlap)."""
     import oracle
 
     oracle.build_oracle()
@@ -117,7 +133,8 @@ def test_context_parallel_equals_full_run(world, kind, seed):
     rdq, rdk, rdv = oracle.attention_backward(q, k, v, do, *masks)
     port = _free_port()
     out = mp.get_context("spawn").Manager().dict()
-    mp.start_processes(_worker, args=(world, port, seed, kind, out), nprocs=world, join=True, start_method="spawn")
+    mp.start_processes(_worker, args=(world, port, seed, kind, out, overlap), nprocs=world, join=True,
+                       start_method="spawn")
     bounds = cp.equal_bounds(N, world)
     for r, (a, b) in enumerate(bounds):
         res = out[r]
@@ -193,3 +210,30 @@ def test_context_parallel_emulated_ranks_on_gpu(name, balanced):
     for nm, s_, full in (("dK", dk_sum, dk), ("dV", dv_sum, dv)):
         err = (s_ - full.float()).abs()
         assert (err <= 2e-2 + 4 * 2.0 ** -8 * full.float().abs()).all(), f"{nm}: {err.max().item()}"
+
+
+@pytest.mark.gpu
+def test_merge_partials_equals_attention_over_the_union(oracle_mod):
+    """Per-chunk forwards over disjoint key chunks (mask sliced on the key axis), merged by the
+    library, equal the forward over all keys (and the oracle) within the parity tolerance; rows
+    that see no key at all get O = 0, LSE = -inf."""
+    import column_sparse_masked_b200 as fm
+
+    from _parity import check_lse, check_out, make_case
+
+    q, k, v, do, masks = make_case(2, 700, 900, 4, 2, 1, 128, "random", 901)
+    qg, kg, vg = q.cuda(), k.cuda(), v.cuda()
+    mg = [m.cuda() for m in masks]
+    o_full, l_full = fm.fwd(qg, kg, vg, *mg)
+    cuts = [(0, 256), (256, 300), (300, 900)]
+    parts = [fm.fwd(qg, kg[:, a:b].contiguous(), vg[:, a:b].contiguous(), *[m[:, :, a:b].contiguous() for m in mg])
+             for a, b in cuts]
+    o, lse = fm.merge_partials([x[0] for x in parts], [x[1] for x in parts])
+    torch.cuda.synchronize()
+    assert fm.get_status() == 0
+    ro, rl = oracle_mod.attention_forward(q, k, v, *masks)
+    check_out("O(merged)", o, ro, case="merge")
+    check_lse(lse, rl, case="merge")
+    err = (o.float() - o_full.float()).abs()
+    assert (err <= 1e-2 + 2.0 ** -7 * o_full.float().abs()).all(), err.max().item()
+    assert torch.equal(torch.isneginf(lse), torch.isneginf(l_full))
