@@ -57,7 +57,7 @@ constexpr int kThreads = 352;
 constexpr int kProducerWarp = 8, kMmaWarp = 9, kProducer2Warp = 10;
 constexpr int kRing = 4;
 constexpr int kQStages = 2;   // Q tiles: last read by dK(t)
-constexpr int kDoStages = 2;  // dO tiles: last read by dV(t)
+constexpr int kDoStages = 1;  // dO tiles: last read by dV(t); dO(t+1) is needed only after dQ(t) is read out
 constexpr int kLStages = 2;   // LSE2 / D rows: last read by the compute warps
 constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256;
 constexpr uint32_t kColDQ = kColDP;  // dQ(t) reuses the dP^T region
@@ -70,6 +70,9 @@ struct __align__(1024) FusedSmem {
   uint8_t q[fb::kQStages][kTile * D * 2];
   uint8_t dout[fb::kDoStages][kTile * D * 2];
   uint8_t ds[2][kTile * 64 * 2];  // dS^T bf16: rows = keys, box g = query columns [64g, 64g+64), SW128
+  // dQ staging of warpgroup g: 8 four-column chunks x 128 rows x 4 fp32, the
+  // layout of 16 KiB of the accumulator tile, reduced into it by the TMA unit
+  float4 stage[2][8 * kTile];
   float lse2[fb::kLStages][kTile];
   float dsum[fb::kLStages][kTile];
   KvItem ring[fb::kRing];
@@ -361,25 +364,39 @@ __global__ void __launch_bounds__(fb::kThreads, 1)
     // Reads dQ(t) (parity par) out of TMEM into fp32 reductions of its tile in
     // the accumulator ([B, Hq, nQt, D/4, 128, 4]); frees the TMEM region once
     // the loads have completed, then issues the reductions.
+    // Reads dQ(t) (parity par) out of TMEM and hands it to the TMA unit as
+    // asynchronous bulk fp32 reductions into its accumulator tile
+    // ([B, Hq, nQt, D/4, 128, 4]): 32 columns per pass through the warpgroup's
+    // 16 KiB staging buffer, whose previous reduction must have finished
+    // reading it.  The warps never wait for the reductions themselves.
+    const bool elected = (wq == 0 && lane == 0);  // issues this warpgroup's bulk reductions
     auto drain_dq = [&](uint32_t par, int b, int h, int qt) -> bool {
       if (!__all_sync(0xffffffffu, mbar_wait(&s.dq_full, par, w))) return false;
       tc_fence_after();
-      constexpr int kCols = D / 2;  // dQ columns of this warpgroup, read 32 at a time
+      constexpr int kCols = D / 2;  // dQ columns of this warpgroup
       float* acc = p.dqacc + (((size_t)b * sh.Hq + h) * sh.nQt + qt) * ((size_t)kTile * D);
+      float4* stg = s.stage[wg];
 #pragma unroll
       for (int c = 0; c < kCols / 32; ++c) {
         uint32_t r[32];
         tmem_ld32x(tb + kColDQ + wg * kCols + c * 32, r);
+        if (elected) bulk_wait_read_all();  // the staging buffer's previous reduction has read it
         tmem_ld_wait();
         if (c == kCols / 32 - 1) {  // every column read: the region may take dP^T(t+1)
           tc_fence_before();
           mbar_arrive(&s.dq_free);
         }
+        named_barrier_sync(1 + wg, 128);  // staging free for every warp of the warpgroup
 #pragma unroll
-        for (int c4 = 0; c4 < 8; ++c4) {
-          const int chunk = wg * (kCols / 4) + c * 8 + c4;  // 4-column chunk of the tile
-          red_add_v4(acc + ((size_t)chunk * kTile + jl) * 4, __uint_as_float(r[4 * c4]),
-                     __uint_as_float(r[4 * c4 + 1]), __uint_as_float(r[4 * c4 + 2]), __uint_as_float(r[4 * c4 + 3]));
+        for (int c4 = 0; c4 < 8; ++c4)
+          stg[c4 * kTile + jl] = make_float4(__uint_as_float(r[4 * c4]), __uint_as_float(r[4 * c4 + 1]),
+                                             __uint_as_float(r[4 * c4 + 2]), __uint_as_float(r[4 * c4 + 3]));
+        fence_async_smem();
+        named_barrier_sync(1 + wg, 128);  // the whole 16 KiB written
+        if (elected) {
+          const int chunk0 = wg * (kCols / 4) + c * 8;  // first 4-column chunk of this pass
+          bulk_reduce_add_f32(acc + (size_t)chunk0 * kTile * 4, stg, 8 * kTile * 16);
+          bulk_commit_group();
         }
       }
       return true;
@@ -532,6 +549,7 @@ __global__ void __launch_bounds__(fb::kThreads, 1)
   }
 
   // ---------------- teardown ----------------
+  if (warp < 8 && (warp & 3) == 0 && lane == 0) bulk_wait_all();  // every dQ reduction has landed
   __syncthreads();
   if (s.abort_flag) {
     const WaitCtx w2{&s.no_abort, p.status, p.wait_limit_ns, smem_addr(smem_raw), 4};

@@ -651,7 +651,7 @@ def dkdv_model(items, seed, R=4, QST=3, DOST=2, LST=2):
 # fused backward (fm_bwd_fused_kernel): dkdv's roles plus dQ(t) = dS K into the
 # dP^T region, read out by the compute warpgroups between the halves of P^T(t+1)
 # ----------------------------------------------------------------------------
-def fused_model(items, seed, R=4, QST=2, DOST=2, LST=2):
+def fused_model(items, seed, R=4, QST=2, DOST=1, LST=2):
     sim = Sim(seed)
     for i in range(R):
         sim.bar(f"ring_full{i}")
