@@ -82,6 +82,7 @@ struct __align__(1024) FusedSmem {
   uint64_t do_full[fb::kDoStages], do_empty[fb::kDoStages];
   uint64_t l_full[fb::kLStages], l_empty[fb::kLStages];
   uint64_t s_full, dp_full, p_full, ds_full, dq_full, dq_free;
+  uint64_t stage_free[2], stage_ready[2];  // per warpgroup: staging reusable / written
   uint64_t dkdv_full, dkdv_free;
   uint64_t teardown;
   uint32_t tmem_base;
@@ -179,6 +180,10 @@ __global__ void __launch_bounds__(fb::kThreads, 1)
     mbar_init(&s.ds_full, 256);
     mbar_init(&s.dq_full, 1);
     mbar_init(&s.dq_free, 256);
+    for (int g = 0; g < 2; ++g) {
+      mbar_init(&s.stage_free[g], 1);     // the warpgroup's elected thread: previous reduction has read it
+      mbar_init(&s.stage_ready[g], 128);  // every thread of the warpgroup wrote its rows
+    }
     mbar_init(&s.dkdv_full, 1);
     mbar_init(&s.dkdv_free, 256);
     mbar_init(&s.teardown, 1);
@@ -370,6 +375,7 @@ __global__ void __launch_bounds__(fb::kThreads, 1)
     // 16 KiB staging buffer, whose previous reduction must have finished
     // reading it.  The warps never wait for the reductions themselves.
     const bool elected = (wq == 0 && lane == 0);  // issues this warpgroup's bulk reductions
+    uint32_t n_pass = 0;  // staging passes of this warpgroup so far (barrier phases)
     auto drain_dq = [&](uint32_t par, int b, int h, int qt) -> bool {
       if (!__all_sync(0xffffffffu, mbar_wait(&s.dq_full, par, w))) return false;
       tc_fence_after();
@@ -377,27 +383,35 @@ __global__ void __launch_bounds__(fb::kThreads, 1)
       float* acc = p.dqacc + (((size_t)b * sh.Hq + h) * sh.nQt + qt) * ((size_t)kTile * D);
       float4* stg = s.stage[wg];
 #pragma unroll
-      for (int c = 0; c < kCols / 32; ++c) {
+      for (int c = 0; c < kCols / 32; ++c, ++n_pass) {
         uint32_t r[32];
         tmem_ld32x(tb + kColDQ + wg * kCols + c * 32, r);
-        if (elected) bulk_wait_read_all();  // the staging buffer's previous reduction has read it
+        if (elected) {
+          bulk_wait_read_all();  // the staging buffer's previous reduction has read it
+          mbar_arrive(&s.stage_free[wg]);
+        }
         tmem_ld_wait();
         if (c == kCols / 32 - 1) {  // every column read: the region may take dP^T(t+1)
           tc_fence_before();
           mbar_arrive(&s.dq_free);
         }
-        named_barrier_sync(1 + wg, 128);  // staging free for every warp of the warpgroup
+        if (!__all_sync(0xffffffffu, mbar_wait(&s.stage_free[wg], n_pass & 1, w))) return false;
 #pragma unroll
         for (int c4 = 0; c4 < 8; ++c4)
           stg[c4 * kTile + jl] = make_float4(__uint_as_float(r[4 * c4]), __uint_as_float(r[4 * c4 + 1]),
                                              __uint_as_float(r[4 * c4 + 2]), __uint_as_float(r[4 * c4 + 3]));
         fence_async_smem();
-        named_barrier_sync(1 + wg, 128);  // the whole 16 KiB written
+        mbar_arrive(&s.stage_ready[wg]);
+        bool staged = true;
         if (elected) {
-          const int chunk0 = wg * (kCols / 4) + c * 8;  // first 4-column chunk of this pass
-          bulk_reduce_add_f32(acc + (size_t)chunk0 * kTile * 4, stg, 8 * kTile * 16);
-          bulk_commit_group();
+          staged = mbar_wait(&s.stage_ready[wg], n_pass & 1, w);  // all 16 KiB written
+          if (staged) {
+            const int chunk0 = wg * (kCols / 4) + c * 8;  // first 4-column chunk of this pass
+            bulk_reduce_add_f32(acc + (size_t)chunk0 * kTile * 4, stg, 8 * kTile * 16);
+            bulk_commit_group();
+          }
         }
+        if (!__all_sync(0xffffffffu, staged)) return false;
       }
       return true;
     };
