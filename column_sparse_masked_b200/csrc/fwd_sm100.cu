@@ -12,28 +12,16 @@
 //     through a ring of mbarriers, so consecutive items overlap (the next
 //     item's Q load and first QK^T run while the softmax warps write O);
 //   * warp 8 issues TMA loads: Q once per item, and K(0), V(0), K(1), V(1), ...
-//     through one ring of tile-sized slots; a slot is released once both MMA
-//     issuers have read it;
-//   * warps 9 and 10 issue the tcgen05 MMAs of q-tile 0 and q-tile 1 of the
-//     block (one issuer per q-tile, so neither waits behind the other);
+//     through one ring of tile-sized slots; a K slot is released after the
+//     second q-tile's QK^T, a V slot after its P V, so V tiles are requested
+//     about two key steps before they are used;
+//   * warp 9 issues tcgen05 MMAs: S_g = Q_g K^T into TMEM, O_g += P_g V with
+//     P_g read from TMEM (bf16, written over S_g), ping-pong between the two
+//     q-tiles: S0 S1 | PV0 S0' PV1 S1' | ...;
 //   * warps 0-3 and 4-7 are the softmax groups of q-tiles 0 and 1: one thread
 //     per query row; online softmax in the exp2 domain with the scale folded
-//     into one FMA per element, O rescaled in TMEM only when a row maximum
-//     grows by more than 2^8.
-//
-// Each S = Q K^T tile is computed as two 64-key halves.  A q-tile's S region
-// (128 TMEM columns) holds two 64-column halves R0, R1; its tile number c
-// (counted over all its items) puts keys 0-63 in R[c%2] and keys 64-127 in
-// R[1-c%2], and the softmax writes P (bf16 pairs, all 128 keys) over R[c%2].
-// So the first half of the NEXT tile can be computed into R[1-c%2] as soon
-// as the softmax has loaded it -- while the softmax still works on this tile
-// -- and only the next tile's second half waits for P V to read P.  The
-// softmax of tile c+1 starts on its first half right after finishing tile c;
-// the per-q-tile chain softmax -> P V -> next Q K^T -> softmax is broken.
-// A maximum that grows in the second half after the first half's P was
-// written rescales that P in TMEM (rare: the rescale threshold is 2^8); the O
-// rescale waits for the second half, whose completion implies the previous
-// P V has completed.
+//     into one FMA per element, O rescaled in TMEM
+//     only when a row maximum grows by more than 2^8.
 //
 // The element mask of a partial tile is built per key column: each lane reads
 // the boundary records of 4 columns (L2-resident), turns them into 32-bit words
@@ -58,9 +46,9 @@ struct FwdCfg {
   static constexpr int kSlots = (D == 128) ? 5 : 10;  // K/V ring slots of one tile each
   static constexpr int kTileBytes = kTile * D * 2;  // one 128-row bf16 tile
   static constexpr int kBoxes = D / 64;             // 64-column (128-byte) TMA boxes per tile
-  static constexpr int kThreads = 352;
+  static constexpr int kThreads = 320;
   static constexpr int kProducerWarp = 8;
-  static constexpr int kMmaWarp0 = 9;  // issuer of q-tile g is warp kMmaWarp0 + g
+  static constexpr int kMmaWarp = 9;
   static constexpr int kRing = 4;
 };
 
@@ -119,12 +107,11 @@ struct __align__(1024) FwdSmem {
   uint64_t q_full, q_empty;
   uint64_t slot_full[FwdCfg<D>::kSlots];
   uint64_t slot_empty[FwdCfg<D>::kSlots];
-  uint64_t s1_full[2], s2_full[2];  // first / second 64-key half of S computed
-  uint64_t y_free[2];               // second half loaded by the softmax (its columns are free)
+  uint64_t s_full[2];
   uint64_t p_full[2];
   uint64_t o_full[2];
   uint64_t o_free[2];
-  uint64_t teardown[2];
+  uint64_t teardown;
   uint32_t tmem_base;
   int abort_flag;
   int no_abort;
@@ -145,20 +132,6 @@ __device__ __forceinline__ void issue_qk(uint32_t d_tmem, const uint8_t* qs, con
   }
 }
 
-// Half of S = Q K^T: M = 128 rows, N = 64 keys (keys 64*half .. 64*half+63 of
-// the K tile), K = D; both operands K-major SW128 (rows 64-127 start 8 KiB into
-// each 16 KiB box, a multiple of the 1 KiB swizzle period).
-template <int D>
-__device__ __forceinline__ void issue_qk_half(uint32_t d_tmem, const uint8_t* qs, const uint8_t* ks, int half) {
-  constexpr uint32_t idesc = idesc_bf16(128, 64, false, false);
-  const uint32_t qa = smem_addr(qs), ka = smem_addr(ks) + half * 8192;
-#pragma unroll
-  for (int kk = 0; kk < D / 16; ++kk) {
-    const uint32_t off = (kk / 4) * 16384 + (kk % 4) * 32;
-    mma_ss(d_tmem, sdesc_sw128(qa + off, 16, 1024), sdesc_sw128(ka + off, 16, 1024), idesc, kk > 0 ? 1u : 0u);
-  }
-}
-
 // O (+)= P V: M = 128 rows, N = D, K = 128 keys.  P from TMEM (bf16 pairs,
 // 8 columns per 16 keys); V is MN-major (d contiguous) SW128.
 template <int D>
@@ -169,20 +142,6 @@ __device__ __forceinline__ void issue_pv(uint32_t d_tmem, uint32_t p_tmem, const
   for (int kk = 0; kk < kTile / 16; ++kk)
     mma_ts(d_tmem, p_tmem + kk * 8, sdesc_sw128(va + kk * 2048, 16384, 1024), idesc,
            (accumulate || kk > 0) ? 1u : 0u);
-}
-
-// Row maximum of 64 raw logits (three-input max instructions).
-__device__ __forceinline__ float row_max64(const float (&x)[64]) {
-  float m4[4];
-#pragma unroll
-  for (int j = 0; j < 4; ++j) m4[j] = max3f(x[j], x[4 + j], x[8 + j]);
-#pragma unroll
-  for (int i = 12; i + 7 < 64; i += 8)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) m4[j] = max3f(m4[j], x[i + j], x[i + 4 + j]);
-  m4[0] = max3f(m4[0], x[60], x[61]);
-  m4[1] = max3f(m4[1], x[62], x[63]);
-  return fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
 }
 
 template <int D>
@@ -201,30 +160,28 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
     if (tid == 0) atomicCAS(p.status, 0, -5);
     return;
   }
-  if (warp == Cfg::kMmaWarp0) {
+  if (warp == Cfg::kMmaWarp) {
     tmem_alloc(&s.tmem_base, 512);
     tmem_relinquish();
   }
   if (tid == 0) {
     for (int i = 0; i < kRing; ++i) {
       mbar_init(&s.ring_full[i], 1);
-      mbar_init(&s.ring_empty[i], 10);  // lane 0 of the 2 MMA warps and of the 8 softmax warps
+      mbar_init(&s.ring_empty[i], 9);  // MMA lane 0 + lane 0 of the 8 softmax warps
     }
     mbar_init(&s.q_full, 1);
-    mbar_init(&s.q_empty, 2);  // both issuers' last Q K^T of the item
+    mbar_init(&s.q_empty, 1);
     for (int i = 0; i < kSlots; ++i) {
       mbar_init(&s.slot_full[i], 1);
-      mbar_init(&s.slot_empty[i], 2);  // read by both issuers
+      mbar_init(&s.slot_empty[i], 1);
     }
     for (int g = 0; g < 2; ++g) {
-      mbar_init(&s.s1_full[g], 1);
-      mbar_init(&s.s2_full[g], 1);
-      mbar_init(&s.y_free[g], 128);
+      mbar_init(&s.s_full[g], 1);
       mbar_init(&s.p_full[g], 128);
       mbar_init(&s.o_full[g], 1);
       mbar_init(&s.o_free[g], 128);
-      mbar_init(&s.teardown[g], 1);
     }
+    mbar_init(&s.teardown, 1);
     s.abort_flag = 0;
     s.no_abort = 0;
     fence_mbar_init();
@@ -300,11 +257,8 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
         }
       }
     }
-  } else if (warp == Cfg::kMmaWarp0 || warp == Cfg::kMmaWarp0 + 1) {
-    // ---------------- MMA issuer of q-tile g ----------------
+  } else if (warp == Cfg::kMmaWarp) {
     if (lane == 0) {
-      const int g = warp - Cfg::kMmaWarp0;
-      const uint32_t sbase = tmem + g * 128, obase = tmem + 256 + g * D;
       uint32_t pos = 0, tile_cnt = 0, act = 0;
       bool ok = true;
       for (uint32_t k = 0; ok; ++k) {
@@ -317,44 +271,47 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
         if (n == 0) continue;
         if (!(ok = mbar_wait(&s.q_full, act & 1, w))) break;
         tc_fence_after();
-        for (int t = 0; t < n; ++t, pos += 2, ++tile_cnt) {
-          // ring slots of V(t) and K(t+1)
+        for (int t = 0; t < n; ++t, pos += 2) {
+          // ring slots of K(t+1) and V(t)
           const int sv = (pos + 1) % kSlots;
           const uint32_t pv_ph = ((pos + 1) / kSlots) & 1;
           const int sk2 = (pos + 2) % kSlots;
           const uint32_t k2_ph = ((pos + 2) / kSlots) & 1;
-          const uint32_t xcol = (tile_cnt & 1) ? 64u : 0u, ycol = 64u - xcol;  // this tile's halves
           if (t == 0) {
             const int sk = pos % kSlots;
             if (!(ok = mbar_wait(&s.slot_full[sk], (pos / kSlots) & 1, w))) break;
             tc_fence_after();
-            issue_qk_half<D>(sbase + xcol, s.q[g], s.slot[sk], 0);
-            mma_commit(&s.s1_full[g]);
-            issue_qk_half<D>(sbase + ycol, s.q[g], s.slot[sk], 1);
-            mma_commit(&s.s2_full[g]);
+            issue_qk<D>(tmem + 0, s.q[0], s.slot[sk]);
+            mma_commit(&s.s_full[0]);
+            issue_qk<D>(tmem + 128, s.q[1], s.slot[sk]);
+            mma_commit(&s.s_full[1]);
             mma_commit(&s.slot_empty[sk]);
             if (n == 1) mma_commit(&s.q_empty);
           }
-          if (t + 1 < n) {
-            // next tile's first half into this tile's second half, once loaded
-            if (!(ok = mbar_wait(&s.y_free[g], tile_cnt & 1, w) && mbar_wait(&s.slot_full[sk2], k2_ph, w))) break;
-            tc_fence_after();
-            issue_qk_half<D>(sbase + ycol, s.q[g], s.slot[sk2], 0);
-            mma_commit(&s.s1_full[g]);
-          }
-          if (!(ok = mbar_wait(&s.slot_full[sv], pv_ph, w) && mbar_wait(&s.p_full[g], tile_cnt & 1, w))) break;
-          if (t == 0 && !(ok = mbar_wait(&s.o_free[g], (act & 1) ^ 1, w))) break;  // previous O read out
+          if (!(ok = mbar_wait(&s.slot_full[sv], pv_ph, w) && mbar_wait(&s.p_full[0], tile_cnt & 1, w))) break;
+          if (t == 0 && !(ok = mbar_wait(&s.o_free[0], (act & 1) ^ 1, w))) break;  // previous O0 read out
           tc_fence_after();
-          issue_pv<D>(obase, sbase + xcol, s.slot[sv], t > 0);
-          if (t == n - 1) mma_commit(&s.o_full[g]);
+          issue_pv<D>(tmem + 256, tmem + 0, s.slot[sv], t > 0);
+          if (t == n - 1) mma_commit(&s.o_full[0]);
+          if (t + 1 < n) {
+            if (!(ok = mbar_wait(&s.slot_full[sk2], k2_ph, w))) break;
+            tc_fence_after();
+            issue_qk<D>(tmem + 0, s.q[0], s.slot[sk2]);
+            mma_commit(&s.s_full[0]);
+          }
+          if (!(ok = mbar_wait(&s.p_full[1], tile_cnt & 1, w))) break;
+          if (t == 0 && !(ok = mbar_wait(&s.o_free[1], (act & 1) ^ 1, w))) break;
+          tc_fence_after();
+          issue_pv<D>(tmem + 256 + D, tmem + 128, s.slot[sv], t > 0);
+          if (t == n - 1) mma_commit(&s.o_full[1]);
           mma_commit(&s.slot_empty[sv]);
           if (t + 1 < n) {
-            // next tile's second half over this tile's P, after P V read it
-            issue_qk_half<D>(sbase + xcol, s.q[g], s.slot[sk2], 1);
-            mma_commit(&s.s2_full[g]);
+            issue_qk<D>(tmem + 128, s.q[1], s.slot[sk2]);
+            mma_commit(&s.s_full[1]);
             mma_commit(&s.slot_empty[sk2]);
-            if (t + 2 == n) mma_commit(&s.q_empty);  // last Q K^T of the item issued
+            if (t + 2 == n) mma_commit(&s.q_empty);  // last QK^T of the item issued
           }
+          ++tile_cnt;
         }
         if (!ok) break;
         ++act;
@@ -401,113 +358,58 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
 #pragma unroll
           for (int c = 0; c < 4; ++c) mw[c] = warp_transpose32(column_row_bits(r4[c], rbase), lane);
         }
-        // This tile's halves: keys 0-63 in X, keys 64-127 in Y; P goes over X.
-        const uint32_t xcol = s_col + ((tile_cnt & 1) ? 64u : 0u);
-        const uint32_t ycol = s_col + ((tile_cnt & 1) ? 0u : 64u);
-        float x[64];
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(&s.s_full[g], tile_cnt & 1, w)))) break;
+        tc_fence_after();
+        float x[128];
         uint32_t* raw = reinterpret_cast<uint32_t*>(x);
-        float alpha_o = 1.f;   // O rescale pending for this tile (applied after the second half)
-        bool rescale_o = false;
-        const bool o_live = (m_run != -INFINITY);  // O holds P V sums of this item's earlier tiles
-        // ---- first half: keys 0-63 ----
-        if (!(ok = __all_sync(0xffffffffu, mbar_wait(&s.s1_full[g], tile_cnt & 1, w)))) break;
-        tc_fence_after();
-        tmem_ld32x(tb + xcol, raw);
-        tmem_ld32x(tb + xcol + 32, raw + 32);
+        tmem_ld32x(tb + s_col + 0, raw + 0);
+        tmem_ld32x(tb + s_col + 32, raw + 32);
+        tmem_ld32x(tb + s_col + 64, raw + 64);
+        tmem_ld32x(tb + s_col + 96, raw + 96);
         tmem_ld_wait();
         if (need) {
 #pragma unroll
-          for (int i = 0; i < 64; ++i) x[i] = ((mw[i >> 5] >> (i & 31)) & 1u) ? -INFINITY : x[i];
+          for (int i = 0; i < 128; ++i) x[i] = ((mw[i >> 5] >> (i & 31)) & 1u) ? -INFINITY : x[i];
         }
-        {
-          const float mx = row_max64(x) * sl2;
-          // Lazy rescale: only when the maximum grows by more than 8 (log2 units).
-          if (mx > m_run + 8.f) {
-            const float a = fast_exp2(m_run - mx);  // 0 when m_run = -inf
-            rescale_o = o_live;
-            alpha_o = a;
-            m_run = mx;
-            l_run *= a;
+        // row maximum of the raw logits (the scale is positive)
+        float m4[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) m4[j] = max3f(x[j], x[4 + j], x[8 + j]);
+#pragma unroll
+        for (int i = 12; i + 7 < 128; i += 8)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) m4[j] = max3f(m4[j], x[i + j], x[i + 4 + j]);
+        m4[0] = max3f(m4[0], x[124], x[125]);
+        m4[1] = max3f(m4[1], x[126], x[127]);
+        const float mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl2;
+        // Lazy rescale: only when the maximum grows by more than 8 (log2 units).
+        float alpha = 1.f;
+        bool rescale = false;
+        if (mx > m_run + 8.f) {
+          alpha = fast_exp2(m_run - mx);  // 0 when m_run = -inf
+          rescale = (m_run != -INFINITY);
+          m_run = mx;
+          l_run *= alpha;
+        }
+        const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
+        float sa = 0.f, sb = 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {  // 32 columns -> 16 packed bf16 pairs per store
+          uint32_t pk[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float a0 = fast_exp2(fmaf(x[c * 32 + 2 * i], sl2, neg_m));
+            const float a1 = fast_exp2(fmaf(x[c * 32 + 2 * i + 1], sl2, neg_m));
+            sa += a0;
+            sb += a1;
+            pk[i] = pack_bf16x2(a0, a1);
           }
+          tmem_st16(tb + s_col + c * 16, pk);
         }
-        {
-          const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
-          float sa = 0.f, sb = 0.f;
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {  // 32 keys -> 16 packed bf16 pairs per store
-            uint32_t pk[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float a0 = fast_exp2(fmaf(x[c * 32 + 2 * i], sl2, neg_m));
-              const float a1 = fast_exp2(fmaf(x[c * 32 + 2 * i + 1], sl2, neg_m));
-              sa += a0;
-              sb += a1;
-              pk[i] = pack_bf16x2(a0, a1);
-            }
-            tmem_st16(tb + xcol + c * 16, pk);
-          }
-          l_run += sa + sb;
-        }
-        // ---- second half: keys 64-127 ----
-        if (!(ok = __all_sync(0xffffffffu, mbar_wait(&s.s2_full[g], tile_cnt & 1, w)))) break;
-        tc_fence_after();
-        tmem_ld32x(tb + ycol, raw);
-        tmem_ld32x(tb + ycol + 32, raw + 32);
-        tmem_ld_wait();
-        tc_fence_before();
-        mbar_arrive(&s.y_free[g]);  // Y loaded: the next tile's first half may go there
-        if (need) {
-#pragma unroll
-          for (int i = 0; i < 64; ++i) x[i] = ((mw[2 + (i >> 5)] >> (i & 31)) & 1u) ? -INFINITY : x[i];
-        }
-        float alpha_p = 1.f;  // rescale of the first half's P, already in TMEM
-        {
-          const float mx = row_max64(x) * sl2;
-          if (mx > m_run + 8.f) {
-            const float a = fast_exp2(m_run - mx);
-            if (m_run != -INFINITY) alpha_p = a;  // the first half's P used the old maximum
-            rescale_o = o_live;
-            alpha_o *= a;
-            m_run = mx;
-            l_run *= a;
-          }
-        }
-        if (__any_sync(0xffffffffu, alpha_p != 1.f)) {
-          // the first half's P was computed against the smaller maximum
-          uint32_t pp[32];
-          tmem_st_wait();  // the first half's stores have landed
-          tmem_ld32x(tb + xcol, pp);
-          tmem_ld_wait();
-#pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(&pp[i]);
-            const float2 f = __bfloat1622float2(v);
-            pp[i] = pack_bf16x2(f.x * alpha_p, f.y * alpha_p);
-          }
-          tmem_st32x(tb + xcol, pp);
-        }
-        {
-          const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
-          float sa = 0.f, sb = 0.f;
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            uint32_t pk[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float a0 = fast_exp2(fmaf(x[c * 32 + 2 * i], sl2, neg_m));
-              const float a1 = fast_exp2(fmaf(x[c * 32 + 2 * i + 1], sl2, neg_m));
-              sa += a0;
-              sb += a1;
-              pk[i] = pack_bf16x2(a0, a1);
-            }
-            tmem_st16(tb + xcol + 32 + c * 16, pk);
-          }
-          l_run += sa + sb;
-        }
+        l_run += sa + sb;
         // O correction (the previous P V of this q-tile has completed: the
-        // commit that signalled the second half was issued after it).
-        if (__any_sync(0xffffffffu, rescale_o)) {
-          const float alpha = rescale_o ? alpha_o : 1.f;
+        // commit that signalled this S was issued after it).
+        if (__any_sync(0xffffffffu, rescale)) {
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             uint32_t o[32];
@@ -585,10 +487,9 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
     // Let copies and MMAs that are still in flight land before the CTA's
     // shared memory and tensor memory are released.
     const WaitCtx w2{&s.no_abort, p.status, p.wait_limit_ns, smem_addr(smem_raw), 0};
-    if ((warp == Cfg::kMmaWarp0 || warp == Cfg::kMmaWarp0 + 1) && lane == 0) {
-      const int g = warp - Cfg::kMmaWarp0;
-      mma_commit(&s.teardown[g]);
-      (void)mbar_wait(&s.teardown[g], 0, w2);
+    if (warp == Cfg::kMmaWarp && lane == 0) {
+      mma_commit(&s.teardown);
+      (void)mbar_wait(&s.teardown, 0, w2);
     }
     if (warp == Cfg::kProducerWarp && lane == 0) {
       if (q_armed) (void)mbar_wait(&s.q_full, q_par, w2);
@@ -598,7 +499,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == Cfg::kMmaWarp0) {
+  if (warp == Cfg::kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }

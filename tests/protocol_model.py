@@ -119,25 +119,20 @@ def ring_reader(sim, ring, k, R):
 # forward (fm_fwd_kernel): producer, MMA, two softmax groups that also write O
 # ----------------------------------------------------------------------------
 def fwd_model(items, seed, R=4, SLOTS=5):
-    """Forward: one producer, one MMA issuer per q-tile of the block, two softmax groups.
-    Each q-tile's S region is two 64-key halves R0, R1; tile number c (counted per q-tile
-    over all items) puts keys 0-63 of its S in R[c % 2] and keys 64-127 in R[1 - c % 2],
-    and its P (all 128 keys, packed) over R[c % 2].  The next tile's first half goes into
-    the half the softmax has just read (y_free), its second half over P once PV has read it."""
     sim = Sim(seed)
     for i in range(R):
         sim.bar(f"ring_full{i}")
-        sim.bar(f"ring_empty{i}", 2 + 2)  # the two MMA issuers + the two softmax groups
-    sim.bar("q_full")
-    sim.bar("q_empty", 2)
+        sim.bar(f"ring_empty{i}", 1 + 2)  # MMA + the two softmax groups
+    for nm in ("q_full", "q_empty"):
+        sim.bar(nm)
     for i in range(SLOTS):
         sim.bar(f"slot_full{i}")
-        sim.bar(f"slot_empty{i}", 2)
+        sim.bar(f"slot_empty{i}")
     for g in range(2):
-        for nm in ("s1_full", "s2_full", "y_free", "o_full", "p_full", "o_free"):
+        for nm in ("s_full", "o_full", "p_full", "o_free"):
             sim.bar(f"{nm}{g}")
     ring = [None] * R
-    st = {"slot": [None] * SLOTS, "q": None, "R": [[None, None], [None, None]], "O": ["free", "free"]}
+    st = {"slot": [None] * SLOTS, "q": None, "S": [None, None], "O": ["free", "free"]}
     seq = list(items) + [None]
 
     def producer():
@@ -170,30 +165,27 @@ def fwd_model(items, seed, R=4, SLOTS=5):
                     sim.tma.append((f"slot_full{sl}", lambda sl=sl, c=(j, t, kv): st["slot"].__setitem__(sl, c)))
                     pos += 1
 
-    def op_s(g, j, t, sl, half, c):
+    def op_s(g, j, t, sl):
         def f():
-            r = c % 2 if half == 1 else 1 - c % 2
             if st["q"] != j or st["slot"][sl] != (j, t, 0):
-                raise Hazard(f"S{g}h{half}({j},{t}): Q {st['q']} slot {st['slot'][sl]}")
-            cur = st["R"][g][r]
-            if cur is not None and cur[0] not in ("used", "read"):
-                raise Hazard(f"S{g}h{half}({j},{t}) overwrites {cur}")
-            st["R"][g][r] = (f"S{half}", c)
+                raise Hazard(f"S{g}({j},{t}): Q {st['q']} slot {st['slot'][sl]}")
+            if st["S"][g] is not None and st["S"][g][0] != "used":
+                raise Hazard(f"S{g}({j},{t}) overwrites {st['S'][g]}")
+            st["S"][g] = ("S", j, t)
         return f
 
-    def op_pv(g, j, t, sl, c):
+    def op_pv(g, j, t, sl):
         def f():
-            r = c % 2
-            if st["slot"][sl] != (j, t, 1) or st["R"][g][r] != ("P", c):
-                raise Hazard(f"PV{g}({j},{t}): slot {st['slot'][sl]} P {st['R'][g][r]}")
+            if st["slot"][sl] != (j, t, 1) or st["S"][g] != ("P", j, t):
+                raise Hazard(f"PV{g}({j},{t}): slot {st['slot'][sl]} S/P {st['S'][g]}")
             o = st["O"][g]
             if (t == 0 and o != "free") or (t > 0 and o != (j, t - 1)):
                 raise Hazard(f"PV{g}({j},{t}): O holds {o}")
-            st["R"][g][r] = ("used", c)
+            st["S"][g] = ("used", j, t)
             st["O"][g] = (j, t)
         return f
 
-    def mma(g):
+    def mma():
         pos = tile = act = k = 0
         while True:
             it = yield from ring_reader(sim, ring, k, R)
@@ -209,25 +201,30 @@ def fwd_model(items, seed, R=4, SLOTS=5):
                 if t == 0:
                     sk = pos % SLOTS
                     yield wait(f"slot_full{sk}", pos // SLOTS)
-                    sim.pipe += [("mma", op_s(g, j, 0, sk, 1, tile)), ("commit", f"s1_full{g}"),
-                                 ("mma", op_s(g, j, 0, sk, 2, tile)), ("commit", f"s2_full{g}"),
-                                 ("commit", f"slot_empty{sk}")]
+                    for g in range(2):
+                        sim.pipe += [("mma", op_s(g, j, 0, sk)), ("commit", f"s_full{g}")]
+                    sim.pipe.append(("commit", f"slot_empty{sk}"))
                     if n == 1:
                         sim.pipe.append(("commit", "q_empty"))
-                if t + 1 < n:
-                    yield wait(f"y_free{g}", tile)
-                    yield wait(f"slot_full{sk2}", (pos + 2) // SLOTS)
-                    sim.pipe += [("mma", op_s(g, j, t + 1, sk2, 1, tile + 1)), ("commit", f"s1_full{g}")]
                 yield wait(f"slot_full{sv}", (pos + 1) // SLOTS)
-                yield wait(f"p_full{g}", tile)
+                yield wait("p_full0", tile)
                 if t == 0:
-                    yield wait(f"o_free{g}", act - 1)
-                sim.pipe.append(("mma", op_pv(g, j, t, sv, tile)))
+                    yield wait("o_free0", act - 1)
+                sim.pipe.append(("mma", op_pv(0, j, t, sv)))
                 if t == n - 1:
-                    sim.pipe.append(("commit", f"o_full{g}"))
+                    sim.pipe.append(("commit", "o_full0"))
+                if t + 1 < n:
+                    yield wait(f"slot_full{sk2}", (pos + 2) // SLOTS)
+                    sim.pipe += [("mma", op_s(0, j, t + 1, sk2)), ("commit", "s_full0")]
+                yield wait("p_full1", tile)
+                if t == 0:
+                    yield wait("o_free1", act - 1)
+                sim.pipe.append(("mma", op_pv(1, j, t, sv)))
+                if t == n - 1:
+                    sim.pipe.append(("commit", "o_full1"))
                 sim.pipe.append(("commit", f"slot_empty{sv}"))
                 if t + 1 < n:
-                    sim.pipe += [("mma", op_s(g, j, t + 1, sk2, 2, tile + 1)), ("commit", f"s2_full{g}"),
+                    sim.pipe += [("mma", op_s(1, j, t + 1, sk2)), ("commit", "s_full1"),
                                  ("commit", f"slot_empty{sk2}")]
                     if t + 2 == n:
                         sim.pipe.append(("commit", "q_empty"))
@@ -242,23 +239,13 @@ def fwd_model(items, seed, R=4, SLOTS=5):
         while it is not None:
             j, n = it
             for t in range(n):
-                x, y = tile % 2, 1 - tile % 2
-                yield wait(f"s1_full{g}", tile)
-                if st["R"][g][x] != ("S1", tile):
-                    raise Hazard(f"softmax{g}({j},{t}) h1: R{x} holds {st['R'][g][x]}")
-                yield STEP  # first half: P of keys 0-63 written over the half it read
-                st["R"][g][x] = ("P1", tile)
-                yield wait(f"s2_full{g}", tile)
-                if st["R"][g][y] != ("S2", tile):
-                    raise Hazard(f"softmax{g}({j},{t}) h2: R{y} holds {st['R'][g][y]}")
-                st["R"][g][y] = ("read", tile)
-                sim.arrive(f"y_free{g}")
+                yield wait(f"s_full{g}", tile)
+                if st["S"][g] != ("S", j, t):
+                    raise Hazard(f"softmax{g}({j},{t}): S holds {st['S'][g]}")
                 if t > 0 and sim.rng.random() < 0.3 and st["O"][g] != (j, t - 1):  # lazy O rescale
                     raise Hazard(f"softmax{g}({j},{t}) rescale: O holds {st['O'][g]}")
-                yield STEP  # second half: P of keys 64-127 into the rest of R[x]
-                if st["R"][g][x] != ("P1", tile):
-                    raise Hazard(f"softmax{g}({j},{t}) h2 writes over {st['R'][g][x]}")
-                st["R"][g][x] = ("P", tile)
+                yield STEP
+                st["S"][g] = ("P", j, t)
                 sim.arrive(f"p_full{g}")
                 tile += 1
             it_next = yield from ring_reader(sim, ring, k, R)  # next item taken before the epilogue
@@ -273,8 +260,7 @@ def fwd_model(items, seed, R=4, SLOTS=5):
                 act += 1
             it = it_next
 
-    sim.run({"producer": producer(), "mma0": mma(0), "mma1": mma(1), "softmax0": softmax(0),
-             "softmax1": softmax(1)})
+    sim.run({"producer": producer(), "mma": mma(), "softmax0": softmax(0), "softmax1": softmax(1)})
 
 
 # ----------------------------------------------------------------------------

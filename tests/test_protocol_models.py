@@ -35,33 +35,23 @@ def test_protocol_is_safe(name):
 
 
 MUTATIONS = [
-    ("fwd", "second half of S(t+1) issued before P V(t) read P(t)",
-     [('                sim.pipe.append(("mma", op_pv(g, j, t, sv, tile)))\n'
-       '                if t == n - 1:\n                    sim.pipe.append(("commit", f"o_full{g}"))\n'
-       '                sim.pipe.append(("commit", f"slot_empty{sv}"))\n'
-       '                if t + 1 < n:\n'
-       '                    sim.pipe += [("mma", op_s(g, j, t + 1, sk2, 2, tile + 1)), ("commit", f"s2_full{g}"),\n'
-       '                                 ("commit", f"slot_empty{sk2}")]\n'
-       '                    if t + 2 == n:\n                        sim.pipe.append(("commit", "q_empty"))\n',
-       '                if t + 1 < n:\n'
-       '                    sim.pipe += [("mma", op_s(g, j, t + 1, sk2, 2, tile + 1)), ("commit", f"s2_full{g}"),\n'
-       '                                 ("commit", f"slot_empty{sk2}")]\n'
-       '                    if t + 2 == n:\n                        sim.pipe.append(("commit", "q_empty"))\n'
-       '                sim.pipe.append(("mma", op_pv(g, j, t, sv, tile)))\n'
-       '                if t == n - 1:\n                    sim.pipe.append(("commit", f"o_full{g}"))\n'
-       '                sim.pipe.append(("commit", f"slot_empty{sv}"))\n')]),
-    ("fwd", "first half of S(t+1) issued before the softmax read the half it overwrites",
-     [('                    yield wait(f"y_free{g}", tile)\n', '')]),
+    ("fwd", "S(t+1) issued before P(t) was consumed",
+     [('                yield wait(f"slot_full{sv}", (pos + 1) // SLOTS)\n                yield wait("p_full0", tile)\n',
+       '                yield wait(f"slot_full{sv}", (pos + 1) // SLOTS)\n                if t + 1 < n:\n'
+       '                    yield wait(f"slot_full{sk2}", (pos + 2) // SLOTS)\n'
+       '                    sim.pipe.append(("mma", op_s(0, j, t + 1, sk2)))\n                yield wait("p_full0", tile)\n')]),
     ("fwd", "O committed before the item's last P V",
-     [('                sim.pipe.append(("mma", op_pv(g, j, t, sv, tile)))\n                if t == n - 1:\n'
-       '                    sim.pipe.append(("commit", f"o_full{g}"))\n',
-       '                if t == n - 1:\n                    sim.pipe.append(("commit", f"o_full{g}"))\n'
-       '                sim.pipe.append(("mma", op_pv(g, j, t, sv, tile)))\n')]),
-    ("fwd", "V slot released by one issuer's P V",
-     [('        sim.bar(f"slot_empty{i}", 2)', '        sim.bar(f"slot_empty{i}", 1)')]),
+     [('                sim.pipe.append(("mma", op_pv(0, j, t, sv)))\n                if t == n - 1:\n'
+       '                    sim.pipe.append(("commit", "o_full0"))\n',
+       '                if t == n - 1:\n                    sim.pipe.append(("commit", "o_full0"))\n'
+       '                sim.pipe.append(("mma", op_pv(0, j, t, sv)))\n')]),
+    ("fwd", "V slot released before its last P V",
+     [('                sim.pipe.append(("mma", op_pv(1, j, t, sv)))\n                if t == n - 1:\n'
+       '                    sim.pipe.append(("commit", "o_full1"))\n                sim.pipe.append(("commit", f"slot_empty{sv}"))\n',
+       '                sim.pipe.append(("commit", f"slot_empty{sv}"))\n                sim.pipe.append(("mma", op_pv(1, j, t, sv)))\n'
+       '                if t == n - 1:\n                    sim.pipe.append(("commit", "o_full1"))\n')]),
     ("fwd", "item ring released by too few readers",
-     [('        sim.bar(f"ring_empty{i}", 2 + 2)  # the two MMA issuers + the two softmax groups',
-       '        sim.bar(f"ring_empty{i}", 2 + 1)')]),
+     [('        sim.bar(f"ring_empty{i}", 1 + 2)  # MMA + the two softmax groups', '        sim.bar(f"ring_empty{i}", 1 + 1)')]),
     ("dq", "single dS barrier waited by tile index (the earlier bug)",
      [('                yield wait(f"ds_full{tj & 1}", tj >> 1)\n', '                yield wait("ds_full0", tj)\n'),
       ('                sim.arrive(f"ds_full{b}")\n', '                sim.arrive("ds_full0")\n')]),
