@@ -11,6 +11,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <unordered_map>
@@ -231,14 +232,31 @@ size_t g_prof_used = 0;
 constexpr size_t kProfMax = 4096;
 
 // Groups per longest-first wave: as many (batch, KV head) groups as keep the
-// data a group's items share (Q/dO for the key side, K/V otherwise) within
-// about half of the 126 MB L2; 0 (natural, position order) when a single group
-// is larger than that.
+// data a group's items share (Q/dO -- and, in the fused backward, the fp32 dQ
+// accumulator -- for the key side, K/V otherwise) within an L2 budget (half of
+// the 126 MB L2 by default; FLASHMASK_WAVE_BUDGET_MB overrides it, a tuning
+// knob read at each call); 0 (natural, position order) when a single group is
+// larger than that.  Small problems (fewer than 16 items per SM) order all
+// groups together for load balance unless the budget is set explicitly.
+size_t wave_budget_bytes(bool* explicit_budget) {
+  const char* e = getenv("FLASHMASK_WAVE_BUDGET_MB");
+  if (e && *e) {
+    const long mb = strtol(e, nullptr, 10);
+    if (mb > 0) {
+      *explicit_budget = true;
+      return (size_t)mb << 20;
+    }
+  }
+  *explicit_budget = false;
+  return (size_t)64 << 20;
+}
+
 int wave_groups(size_t group_bytes, int n_groups, int64_t n_items, int sm_count) {
-  const size_t budget = (size_t)64 << 20;
+  bool explicit_budget = false;
+  const size_t budget = wave_budget_bytes(&explicit_budget);
   // With few items per CTA the tail of the longest-first order decides the
   // makespan: order all groups together.
-  if (group_bytes == 0 || n_items < (int64_t)16 * sm_count) return n_groups;
+  if (group_bytes == 0 || (!explicit_budget && n_items < (int64_t)16 * sm_count)) return n_groups;
   const size_t w = budget / group_bytes;
   if (w == 0) return 0;
   return (int)(w < (size_t)n_groups ? w : (size_t)n_groups);
@@ -468,7 +486,8 @@ int flashmask_bwd(const void* q, const void* k, const void* v, const void* o, co
     sb.counter = reinterpret_cast<int*>(ws + L.counters) + 1;
     sb.n_items = (int)s.n_kv_items;
     sb.items_per_group = s.nKt;
-    sb.wave = wave_groups((size_t)s.G * s.Nq * s.d * 2 * 2, s.B * s.Hkv, s.n_kv_items, di.sm_count);
+    // a group's items share its q-heads' Q and dO (bf16) and dQ accumulator rows (fp32)
+    sb.wave = wave_groups((size_t)s.G * s.Nq * s.d * (2 + 2 + 4), s.B * s.Hkv, s.n_kv_items, di.sm_count);
     finish_sort_params(sb);
     if (sb.n_items > 0) FM_CUDA(launch_sort_units(&sb, 1, st));
     BwdParams kp{};

@@ -36,6 +36,11 @@
  *  - Tiles are 128 query rows x 128 key columns.
  *  - Device-side failures (a bounded wait that timed out) are recorded in a
  *    per-device status word that flashmask_get_status() reads and clears.
+ *  - Work items of the persistent kernels are taken longest-first in waves of
+ *    (batch, KV head) groups whose shared data fit an L2 budget (64 MiB by
+ *    default; the environment variable FLASHMASK_WAVE_BUDGET_MB overrides it,
+ *    read at each call: a tuning knob that changes the order of the work,
+ *    never its results beyond fp32 summation order in the fused backward's dQ).
  *  - Mask values are applied literally, in or out of [0, Nq].  The checks
  *    build of the library (libflashmask_checks.so, the same entry points
  *    compiled with FLASHMASK_CHECKS) also records FLASHMASK_ERR_BOUNDS in the
