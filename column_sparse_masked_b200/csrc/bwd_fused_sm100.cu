@@ -31,15 +31,16 @@
 // Tensor-core instructions of one thread execute in issue order, so S^T(t+1)
 // may overwrite the S^T region right after dV(t), and dQ(t) the dP^T region
 // right after dK(t) has read dS^T(t) from it.
-// The compute warps read dQ(t) out in the middle of P^T(t+1) (after the first
-// 32 of each warpgroup's 64 query columns): the first half hides dQ(t)'s MMA
-// latency, the second half the latency of dP^T(t+1), which may start once the
-// read-out is done.
+// A fourth warpgroup reads dQ(t) out of TMEM (freeing the region for
+// dP^T(t+1) as soon as the loads complete) and sends it as fp32 reductions:
+// only it waits on the L2's reduction rate (about 20 bytes per clock per SM
+// when every SM reduces), never the compute warps' chain.
 //
-// Roles (352 threads): warps 0-7 compute (two warpgroups; thread = key lane
-// for S^T/dP^T, query row for dQ; warpgroup 0 takes query columns 0-63 and dQ
-// columns [0, d/2), warpgroup 1 the rest), warp 8 TMA producer of K and Q,
-// warp 10 TMA producer of V, dO and the LSE2 / D rows, warp 9 MMA issuer.
+// Roles (512 threads, registers split per warpgroup with setmaxnreg): warps
+// 0-7 compute (two warpgroups; thread = key lane; warpgroup 0 takes query
+// columns 0-63, warpgroup 1 64-127), warps 8-11 the dQ read-out (thread =
+// query row), warp 12 TMA producer of K and Q, warp 14 TMA producer of V, dO
+// and the LSE2 / D rows, warp 13 MMA issuer, warp 15 idle.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <climits>
@@ -53,11 +54,18 @@
 namespace fm {
 
 namespace fb {
-constexpr int kThreads = 352;
-constexpr int kProducerWarp = 8, kMmaWarp = 9, kProducer2Warp = 10;
+constexpr int kThreads = 512;
+constexpr int kDrainWarp0 = 8;  // warps 8-11: the dQ read-out warpgroup
+constexpr int kProducerWarp = 12, kMmaWarp = 13, kProducer2Warp = 14;  // warp 15 idles
 constexpr int kRing = 4;
 constexpr int kQStages = 2;   // Q tiles: last read by dK(t)
 constexpr int kDoStages = 1;  // dO tiles: last read by dV(t); dO(t+1) is needed only after dQ(t) is read out
+// Registers per thread after the per-warpgroup split (setmaxnreg): compute,
+// dQ read-out, and the producer/MMA warpgroup.  The block is launched with
+// 128 per thread; the shares must not add up to more than that total.
+constexpr int kRegCompute = 168, kRegDrain = 56, kRegControl = 120;
+static_assert(2 * 128 * kRegCompute + 128 * kRegDrain + 128 * kRegControl <= kThreads * 128,
+              "the register split must fit the launch's registers");
 constexpr int kLStages = 2;   // LSE2 / D rows: last read by the compute warps
 constexpr uint32_t kColS = 0, kColDP = 128, kColDV = 256;
 constexpr uint32_t kColDQ = kColDP;  // dQ(t) reuses the dP^T region
@@ -69,10 +77,10 @@ struct __align__(1024) FusedSmem {
   uint8_t v[kTile * D * 2];
   uint8_t q[fb::kQStages][kTile * D * 2];
   uint8_t dout[fb::kDoStages][kTile * D * 2];
-  uint8_t ds[2][kTile * 64 * 2];  // dS^T bf16: rows = keys, box g = query columns [64g, 64g+64), SW128
-  // dQ staging of warpgroup g: 8 four-column chunks x 128 rows x 4 fp32, the
-  // layout of 16 KiB of the accumulator tile, reduced into it by the TMA unit
-  float4 stage[2][8 * kTile];
+  // dS^T bf16 (rows = keys, box g = query columns [64g, 64g+64), SW128); once
+  // dQ(t) has read it, the fp32 dQ(t) columns 0-63 staged for reduction
+  uint8_t ds[2][kTile * 64 * 2];
+  float4 stage[16 * kTile];  // fp32 dQ(t) columns 64-127 staged for reduction
   float lse2[fb::kLStages][kTile];
   float dsum[fb::kLStages][kTile];
   KvItem ring[fb::kRing];
@@ -82,7 +90,9 @@ struct __align__(1024) FusedSmem {
   uint64_t do_full[fb::kDoStages], do_empty[fb::kDoStages];
   uint64_t l_full[fb::kLStages], l_empty[fb::kLStages];
   uint64_t s_full, dp_full, p_full, ds_full, dq_full, dq_free;
-  uint64_t stage_free[2], stage_ready[2];  // per warpgroup: staging reusable / written
+  uint64_t staged;      // the read-out warpgroup wrote dQ(t) into the two buffers
+  uint64_t dsbuf_free;  // the reduction has read the dS buffer: dS(t+1) may be written
+  uint64_t buf_free;    // the reductions have read both buffers: dQ(t+1) may be staged
   uint64_t dkdv_full, dkdv_free;
   uint64_t teardown;
   uint32_t tmem_base;
@@ -156,7 +166,7 @@ __global__ void __launch_bounds__(fb::kThreads, 1)
   if (tid == 0) {
     for (int i = 0; i < kRing; ++i) {
       mbar_init(&s.ring_full[i], 1);
-      mbar_init(&s.ring_empty[i], 10);  // MMA + second producer + lane 0 of the 8 compute warps
+      mbar_init(&s.ring_empty[i], 14);  // MMA + second producer + lane 0 of the 8 compute and 4 read-out warps
     }
     mbar_init(&s.k_full, 1);
     mbar_init(&s.k_empty, 1);
@@ -179,11 +189,10 @@ __global__ void __launch_bounds__(fb::kThreads, 1)
     mbar_init(&s.p_full, 256);
     mbar_init(&s.ds_full, 256);
     mbar_init(&s.dq_full, 1);
-    mbar_init(&s.dq_free, 256);
-    for (int g = 0; g < 2; ++g) {
-      mbar_init(&s.stage_free[g], 1);     // the warpgroup's elected thread: previous reduction has read it
-      mbar_init(&s.stage_ready[g], 128);  // every thread of the warpgroup wrote its rows
-    }
+    mbar_init(&s.dq_free, 128);  // the read-out warpgroup
+    mbar_init(&s.staged, 128);
+    mbar_init(&s.dsbuf_free, 1);
+    mbar_init(&s.buf_free, 1);
     mbar_init(&s.dkdv_full, 1);
     mbar_init(&s.dkdv_free, 256);
     mbar_init(&s.teardown, 1);
@@ -207,7 +216,10 @@ __global__ void __launch_bounds__(fb::kThreads, 1)
   uint32_t q_par[kQStages] = {}, do_par[kDoStages] = {}, l_par[kLStages] = {};
   uint32_t q_armed = 0, do_armed = 0, l_armed = 0;
 
+  // Every role starts with its warpgroup's register share (setmaxnreg; all
+  // warps of a warpgroup execute the same one).
   if (warp == kProducerWarp) {
+    setmaxnreg_dec<kRegControl>();
     // first producer: the item's K tile and every q-tile's Q
     if (lane == 0) {
       uint32_t sq = 0, act = 0;
@@ -245,6 +257,7 @@ __global__ void __launch_bounds__(fb::kThreads, 1)
       }
     }
   } else if (warp == kProducer2Warp) {
+    setmaxnreg_dec<kRegControl>();
     // second producer: the item's V tile, every q-tile's dO and LSE2 / D rows
     if (lane == 0) {
       uint32_t sq = 0, act = 0;
@@ -287,6 +300,7 @@ __global__ void __launch_bounds__(fb::kThreads, 1)
       }
     }
   } else if (warp == kMmaWarp) {
+    setmaxnreg_dec<kRegControl>();
     if (lane == 0) {
       uint32_t sq = 0, tc = 0, act = 0;
       bool ok = true;
@@ -353,7 +367,80 @@ __global__ void __launch_bounds__(fb::kThreads, 1)
         mma_commit(&s.dkdv_full);
       }
     }
-  } else {
+  } else if (warp >= kDrainWarp0 && warp < kDrainWarp0 + 4) {
+    // ---------------- dQ read-out warpgroup: thread = query row (TMEM lane) ----------------
+    // Copies dQ(t) from TMEM into shared memory in the accumulator tile's
+    // layout (columns 0-63 into the dS buffer, which dQ(t) has finished
+    // reading, 64-127 into the staging buffer), frees the TMEM region after
+    // the last 32 columns (dP^T(t+1) may then be issued), and has one thread
+    // hand both halves to the TMA unit as asynchronous bulk fp32 reductions
+    // into [B, Hq, nQt, D/4, 128, 4].  Only that thread waits on the L2's
+    // reduction rate (about 20 bytes per clock per SM when every SM reduces):
+    // it releases the dS buffer, then the staging buffer, as the reductions
+    // read them.
+    setmaxnreg_dec<kRegDrain>();
+    const int wq = warp & 3;
+    const int jl = wq * 32 + lane;
+    const uint32_t tb = tmem + ((uint32_t)(wq * 32) << 16);
+    const bool elected = (wq == 0 && lane == 0);
+    float4* lo = reinterpret_cast<float4*>(s.ds[0]);  // 32 KiB: chunks 0 .. D/8 - 1
+    float4* hi = s.stage;                              // chunks D/8 .. D/4 - 1
+    uint32_t tc = 0;
+    bool ok = true;
+    for (uint32_t k = 0; ok; ++k) {
+      const int slot = k % kRing;
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(&s.ring_full[slot], (k / kRing) & 1, w)))) break;
+      const KvItem it = s.ring[slot];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.ring_empty[slot]);
+      if (it.item >= p.n_items) break;
+      if (it.total == 0) continue;
+      ok = for_each_qtile(p, it, [&](int, int h, int, int qt, int) {
+        // the previous reductions have read both buffers; dQ(t) has completed
+        if (tc > 0 && !__all_sync(0xffffffffu, mbar_wait(&s.buf_free, (tc - 1) & 1, w))) return false;
+        if (!__all_sync(0xffffffffu, mbar_wait(&s.dq_full, tc & 1, w))) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32x(tb + kColDQ + c * 32, r);
+          tmem_ld_wait();
+          if (c == D / 32 - 1) {  // every column read: the region may take dP^T(t+1)
+            tc_fence_before();
+            mbar_arrive(&s.dq_free);
+          }
+          float4* dst = (c < D / 64) ? lo + c * 8 * kTile : hi + (c - D / 64) * 8 * kTile;
+#pragma unroll
+          for (int c4 = 0; c4 < 8; ++c4)
+            dst[c4 * kTile + jl] = make_float4(__uint_as_float(r[4 * c4]), __uint_as_float(r[4 * c4 + 1]),
+                                               __uint_as_float(r[4 * c4 + 2]), __uint_as_float(r[4 * c4 + 3]));
+        }
+        fence_async_smem();
+        mbar_arrive(&s.staged);
+        bool issued = true;
+        if (elected) {
+          issued = mbar_wait(&s.staged, tc & 1, w);
+          if (issued) {
+            float* acc = p.dqacc + (((size_t)it.b * sh.Hq + h) * sh.nQt + qt) * ((size_t)kTile * D);
+            constexpr uint32_t kHalfBytes = (D / 8) * kTile * 16;
+            bulk_reduce_add_f32(acc, lo, kHalfBytes);
+            bulk_commit_group();
+            bulk_reduce_add_f32(acc + (D / 8) * kTile * 4, hi, kHalfBytes);
+            bulk_commit_group();
+            asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");  // the dS buffer has been read
+            mbar_arrive(&s.dsbuf_free);
+            bulk_wait_read_all();
+            mbar_arrive(&s.buf_free);
+          }
+        }
+        if (!__all_sync(0xffffffffu, issued)) return false;
+        ++tc;
+        return true;
+      });
+    }
+    if (elected) bulk_wait_all();  // every reduction has landed before the CTA ends
+  } else if (warp < 8) {
+    setmaxnreg_inc<kRegCompute>();
     // ---------------- compute warpgroups ----------------
     // S^T / dP^T: thread = key lane, warpgroup wg takes query columns
     // [64 wg, 64 wg + 64).  dQ: thread = query row (the same TMEM lane),
@@ -369,52 +456,6 @@ __global__ void __launch_bounds__(fb::kThreads, 1)
     // Reads dQ(t) (parity par) out of TMEM into fp32 reductions of its tile in
     // the accumulator ([B, Hq, nQt, D/4, 128, 4]); frees the TMEM region once
     // the loads have completed, then issues the reductions.
-    // Reads dQ(t) (parity par) out of TMEM and hands it to the TMA unit as
-    // asynchronous bulk fp32 reductions into its accumulator tile
-    // ([B, Hq, nQt, D/4, 128, 4]): 32 columns per pass through the warpgroup's
-    // 16 KiB staging buffer, whose previous reduction must have finished
-    // reading it.  The warps never wait for the reductions themselves.
-    const bool elected = (wq == 0 && lane == 0);  // issues this warpgroup's bulk reductions
-    uint32_t n_pass = 0;  // staging passes of this warpgroup so far (barrier phases)
-    auto drain_dq = [&](uint32_t par, int b, int h, int qt) -> bool {
-      if (!__all_sync(0xffffffffu, mbar_wait(&s.dq_full, par, w))) return false;
-      tc_fence_after();
-      constexpr int kCols = D / 2;  // dQ columns of this warpgroup
-      float* acc = p.dqacc + (((size_t)b * sh.Hq + h) * sh.nQt + qt) * ((size_t)kTile * D);
-      float4* stg = s.stage[wg];
-#pragma unroll
-      for (int c = 0; c < kCols / 32; ++c, ++n_pass) {
-        uint32_t r[32];
-        tmem_ld32x(tb + kColDQ + wg * kCols + c * 32, r);
-        if (elected) {
-          bulk_wait_read_all();  // the staging buffer's previous reduction has read it
-          mbar_arrive(&s.stage_free[wg]);
-        }
-        tmem_ld_wait();
-        if (c == kCols / 32 - 1) {  // every column read: the region may take dP^T(t+1)
-          tc_fence_before();
-          mbar_arrive(&s.dq_free);
-        }
-        if (!__all_sync(0xffffffffu, mbar_wait(&s.stage_free[wg], n_pass & 1, w))) return false;
-#pragma unroll
-        for (int c4 = 0; c4 < 8; ++c4)
-          stg[c4 * kTile + jl] = make_float4(__uint_as_float(r[4 * c4]), __uint_as_float(r[4 * c4 + 1]),
-                                             __uint_as_float(r[4 * c4 + 2]), __uint_as_float(r[4 * c4 + 3]));
-        fence_async_smem();
-        mbar_arrive(&s.stage_ready[wg]);
-        bool staged = true;
-        if (elected) {
-          staged = mbar_wait(&s.stage_ready[wg], n_pass & 1, w);  // all 16 KiB written
-          if (staged) {
-            const int chunk0 = wg * (kCols / 4) + c * 8;  // first 4-column chunk of this pass
-            bulk_reduce_add_f32(acc + (size_t)chunk0 * kTile * 4, stg, 8 * kTile * 16);
-            bulk_commit_group();
-          }
-        }
-        if (!__all_sync(0xffffffffu, staged)) return false;
-      }
-      return true;
-    };
     for (uint32_t k = 0; ok; ++k) {
       const int slot = k % kRing;
       if (!(ok = __all_sync(0xffffffffu, mbar_wait(&s.ring_full[slot], (k / kRing) & 1, w)))) break;
@@ -426,7 +467,6 @@ __global__ void __launch_bounds__(fb::kThreads, 1)
       if (it.total > 0) {
         int cur_hm = -1;
         int4 rec = make_int4(0, 0, 0, 0);
-        int prev_h = 0, prev_qt = 0;
         ok = for_each_qtile(p, it, [&](int j, int h, int hm, int qt, int cls) {
           if (hm != cur_hm) {
             rec = p.rec[(((size_t)it.b * sh.Hm + hm) * sh.nKt + it.kt) * kTile + jl];
@@ -471,10 +511,6 @@ __global__ void __launch_bounds__(fb::kThreads, 1)
             for (int i = 0; i < 16; ++i)
               pk[i] = pack_bf16x2(__uint_as_float(pr[half * 32 + 2 * i]), __uint_as_float(pr[half * 32 + 2 * i + 1]));
             tmem_st16(tb + kColS + c0 + half * 16, pk);
-            if (half == 0 && j > 0) {
-              // dQ of the previous q-tile, between the halves
-              if (!drain_dq((tc - 1) & 1, it.b, prev_h, prev_qt)) return false;
-            }
           }
           tmem_st_wait();
           tc_fence_before();
@@ -504,9 +540,9 @@ __global__ void __launch_bounds__(fb::kThreads, 1)
             for (int i = 0; i < 32; ++i)
               pk[i] = pack_bf16x2(__uint_as_float(pr[2 * i]), __uint_as_float(pr[2 * i + 1]));
             tmem_st32x(tb + kColDP + c0, pk);  // bf16 pairs over this warpgroup's own dP^T columns
-            // and the same 64 values into this key's row of the shared dS^T box
-            // (the previous q-tile's dQ, which read the box, has completed:
-            // its read-out waited for it)
+            // and the same 64 values into this key's row of the shared dS^T box,
+            // once the previous q-tile's dQ staged there has been read by its reduction
+            if (tc > 0 && !__all_sync(0xffffffffu, mbar_wait(&s.dsbuf_free, (tc - 1) & 1, w))) return false;
 #pragma unroll
             for (int c = 0; c < 8; ++c)
               *reinterpret_cast<uint4*>(ds_row + ((c ^ sw) << 4)) =
@@ -517,15 +553,11 @@ __global__ void __launch_bounds__(fb::kThreads, 1)
           tc_fence_before();
           mbar_arrive(&s.ds_full);
           mbar_arrive(&s.l_empty[sl]);  // LSE2 / D of this q-tile no longer read
-          prev_h = h;
-          prev_qt = qt;
           ++sq;
           ++tc;
           return true;
         });
         if (!ok) break;
-        // dQ of the item's last q-tile
-        if (!(ok = drain_dq((tc - 1) & 1, it.b, prev_h, prev_qt))) break;
         // epilogue: warpgroup 0 writes dV, warpgroup 1 writes dK
         if (!(ok = __all_sync(0xffffffffu, mbar_wait(&s.dkdv_full, act & 1, w)))) break;
         tc_fence_after();
@@ -560,10 +592,11 @@ __global__ void __launch_bounds__(fb::kThreads, 1)
         for (int i = 0; i < D / 8; ++i) d4[i] = make_uint4(0, 0, 0, 0);
       }
     }
+  } else {
+    setmaxnreg_dec<kRegControl>();  // warp 15: idle, in the producer/MMA warpgroup
   }
 
   // ---------------- teardown ----------------
-  if (warp < 8 && (warp & 3) == 0 && lane == 0) bulk_wait_all();  // every dQ reduction has landed
   __syncthreads();
   if (s.abort_flag) {
     const WaitCtx w2{&s.no_abort, p.status, p.wait_limit_ns, smem_addr(smem_raw), 4};

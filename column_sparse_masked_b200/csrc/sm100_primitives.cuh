@@ -308,6 +308,15 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
+// Per-warpgroup register re-allocation (every warp of the warpgroup executes
+// the same instruction).  inc waits until the registers are free in the
+// block's pool, which only decs of other warpgroups return: the shares of all
+// warpgroups must add up to the block's registers at launch.
+template <int N>
+__device__ __forceinline__ void setmaxnreg_inc() { asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N)); }
+template <int N>
+__device__ __forceinline__ void setmaxnreg_dec() { asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N)); }
+
 // Programmatic dependent launch.  griddep_wait: returns once the grid this one
 // was launched after (with programmatic stream serialisation) has completed
 // and its memory operations are visible; a no-op for a normal launch.  Every

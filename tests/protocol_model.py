@@ -641,11 +641,14 @@ def fused_model(items, seed, R=4, QST=2, DOST=1, LST=2):
     sim = Sim(seed)
     for i in range(R):
         sim.bar(f"ring_full{i}")
-        sim.bar(f"ring_empty{i}", 1 + 1 + 2)  # MMA + second producer + the two compute warpgroups
+        sim.bar(f"ring_empty{i}", 1 + 1 + 2 + 1)  # MMA + second producer + two compute warpgroups + drain
     for nm in ("k_full", "k_empty", "v_full", "v_empty", "s_full", "dp_full", "dq_full", "dkdv_full"):
         sim.bar(nm)
-    for nm in ("p_full", "ds_full", "dq_free", "dkdv_free"):
+    for nm in ("p_full", "ds_full", "dkdv_free"):  # the two compute warpgroups
         sim.bar(nm, 2)
+    sim.bar("dq_free", 1)  # the drain warpgroup
+    for nm in ("staged", "dsbuf_free", "buf_free"):
+        sim.bar(nm)
     for i in range(QST):
         sim.bar(f"q_full{i}")
         sim.bar(f"q_empty{i}")
@@ -657,7 +660,7 @@ def fused_model(items, seed, R=4, QST=2, DOST=1, LST=2):
         sim.bar(f"l_empty{i}", 2)
     ring = [None] * R
     st = {"k": None, "v": None, "q": [None] * QST, "do": [None] * DOST, "l": [None] * LST,
-          "S": [None, None], "dP": [None, None], "dsm": [None, None], "dV": "free", "dK": "free"}
+          "S": [None, None], "dP": [None, None], "dsm": [None, None], "stage": None, "dV": "free", "dK": "free"}
     seq = list(items) + [None]
 
     def producer():  # K and every q-tile's Q; K is freed after the item's last dQ
@@ -802,15 +805,6 @@ def fused_model(items, seed, R=4, QST=2, DOST=1, LST=2):
 
     def compute(h):
         sq = tc = act = k = 0
-
-        def drain(tq):  # reads dQ(tq) out of the dP^T region, then frees it
-            yield wait("dq_full", tq)
-            if st["dP"][h] != ("dQ", tq):
-                raise Hazard(f"compute{h} drain({tq}): dP region holds {st['dP'][h]}")
-            yield STEP
-            st["dP"][h] = ("used", tq)
-            sim.arrive("dq_free")
-
         while True:
             it = yield from ring_reader(sim, ring, k, R)
             k += 1
@@ -825,16 +819,15 @@ def fused_model(items, seed, R=4, QST=2, DOST=1, LST=2):
                 yield wait(f"l_full{l}", sq // LST)
                 if st["S"][h] != ("S", tc) or st["l"][l] != (j, t):
                     raise Hazard(f"compute{h}({j},{t}): S {st['S'][h]} rows {st['l'][l]}")
-                yield STEP  # first half of P^T
-                if t > 0:
-                    yield from drain(tc - 1)
-                yield STEP  # second half of P^T
+                yield STEP  # P^T
                 st["S"][h] = ("P", tc)
                 sim.arrive("p_full")
                 yield wait("dp_full", tc)
                 if st["dP"][h] != ("dP", tc):
                     raise Hazard(f"compute{h}({j},{t}): dP {st['dP'][h]}")
-                if st["dsm"][h] is not None and st["dsm"][h][0] != "used":
+                if tc > 0:
+                    yield wait("dsbuf_free", tc - 1)  # the reduction has read dQ(tc-1) staged there
+                if st["dsm"][h] is not None and st["dsm"][h][0] != "free":
                     raise Hazard(f"compute{h}({j},{t}): dS buffer still holds {st['dsm'][h]}")
                 yield STEP
                 st["dP"][h] = ("dS", tc)
@@ -843,7 +836,6 @@ def fused_model(items, seed, R=4, QST=2, DOST=1, LST=2):
                 sim.arrive(f"l_empty{l}")
                 sq += 1
                 tc += 1
-            yield from drain(tc - 1)
             yield wait("dkdv_full", act)  # warpgroup 0 writes dV, warpgroup 1 dK
             acc = "dV" if h == 0 else "dK"
             if st[acc] != (j, n - 1):
@@ -853,8 +845,49 @@ def fused_model(items, seed, R=4, QST=2, DOST=1, LST=2):
             sim.arrive("dkdv_free")
             act += 1
 
+    def drain():  # dQ(t): TMEM -> the dS buffer (cols 0-63) and the staging buffer
+        tc = k = 0
+        while True:
+            it = yield from ring_reader(sim, ring, k, R)
+            k += 1
+            if it is None:
+                return
+            j, n = it
+            for t in range(n):
+                if tc > 0:
+                    yield wait("buf_free", tc - 1)
+                yield wait("dq_full", tc)
+                if st["dP"] != [("dQ", tc), ("dQ", tc)]:
+                    raise Hazard(f"drain({j},{t}): dP region holds {st['dP']}")
+                if st["dsm"] != [("used", tc), ("used", tc)]:
+                    raise Hazard(f"drain({j},{t}): dS buffer holds {st['dsm']}")
+                if st["stage"] is not None and st["stage"][0] != "free":
+                    raise Hazard(f"drain({j},{t}): staging buffer holds {st['stage']}")
+                yield STEP
+                st["dP"] = [("used", tc), ("used", tc)]
+                sim.arrive("dq_free")
+                st["dsm"] = [("dQ", tc), ("dQ", tc)]
+                st["stage"] = ("dQ", tc)
+                sim.arrive("staged")
+                tc += 1
+
+    def reducer():  # the drain warpgroup's elected thread: the bulk reductions read both buffers
+        tc = 0
+        total = sum(n for _, n in items)
+        while tc < total:
+            yield wait("staged", tc)
+            if st["dsm"] != [("dQ", tc), ("dQ", tc)] or st["stage"] != ("dQ", tc):
+                raise Hazard(f"reducer({tc}): buffers hold {st['dsm']} / {st['stage']}")
+            yield STEP
+            st["dsm"] = [("free", tc), ("free", tc)]
+            sim.arrive("dsbuf_free")
+            yield STEP
+            st["stage"] = ("free", tc)
+            sim.arrive("buf_free")
+            tc += 1
+
     sim.run({"producer": producer(), "producer2": producer2(), "mma": mma(), "compute0": compute(0),
-             "compute1": compute(1)})
+             "compute1": compute(1), "drain": drain(), "reducer": reducer()})
 
 
 MODELS = {"fwd": fwd_model, "dq": dq_model, "dkdv": dkdv_model, "fused": fused_model}

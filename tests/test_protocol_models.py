@@ -100,11 +100,13 @@ MUTATIONS = [
        '                if t + 1 == n:\n                    sim.pipe.append(("commit", "k_empty"))\n',
        '                if t + 1 == n:\n                    sim.pipe.append(("commit", "k_empty"))\n'
        '                sim.pipe += [("mma", op_dq(j, t, tj)), ("commit", "dq_full")]\n')]),
-    ("fused", "dQ(t) not read out before P^T(t+1) is handed over",
-     [('                if t > 0:\n                    yield from drain(tc - 1)\n', '')]),
-    ("fused", "dQ region counted free after one warpgroup",
-     [('    for nm in ("p_full", "ds_full", "dq_free", "dkdv_free"):\n        sim.bar(nm, 2)\n',
-       '    for nm in ("p_full", "ds_full", "dkdv_free"):\n        sim.bar(nm, 2)\n    sim.bar("dq_free", 1)\n')]),
+    ("fused", "dS(t+1) written over dQ(t) staged in the dS buffer before its reduction read it",
+     [('                if tc > 0:\n                    yield wait("dsbuf_free", tc - 1)  # the reduction has read dQ(tc-1) staged there\n', '')]),
+    ("fused", "dQ(t+1) staged before the previous reductions read the buffers",
+     [('                if tc > 0:\n                    yield wait("buf_free", tc - 1)\n', '')]),
+    ("fused", "dQ region freed before the drain read it",
+     [('                yield STEP\n                st["dP"] = [("used", tc), ("used", tc)]\n                sim.arrive("dq_free")\n',
+       '                sim.arrive("dq_free")\n                yield STEP\n                st["dP"] = [("used", tc), ("used", tc)]\n')]),
     ("dkdv", "P^T counted complete after one warpgroup",
      [('    for nm in ("p_full", "ds_full", "dkdv_free"):\n        sim.bar(nm, 2)\n',
        '    for nm in ("ds_full", "dkdv_free"):\n        sim.bar(nm, 2)\n    sim.bar("p_full", 1)\n')]),
