@@ -9,10 +9,10 @@
 // Each (query tile, key tile) pair is visited once: S, dP and dS are formed
 // once and feed all three gradients (the method's 5 matmuls per pair).  dK and
 // dV accumulate in TMEM over the whole GQA group; each pair's dQ contribution
-// dS K leaves the SM as fp32 reductions into a tiled accumulator in global
-// memory (one 16-byte reduction per thread covers 4 columns of one row, a
-// warp's 32 rows 512 contiguous bytes), which a finalize kernel scales and
-// converts to bf16.  dK and dV are deterministic; dQ's fp32 sums depend on
+// dS K leaves the SM as fp32 bulk reductions (the TMA unit's
+// cp.reduce.async.bulk, two of 32 KiB per pair at d = 128) into a tiled
+// accumulator in global memory laid out so that each half of a tile's dQ is
+// one contiguous range, which a finalize kernel scales and converts to bf16.  dK and dV are deterministic; dQ's fp32 sums depend on
 // the order in which the CTAs' reductions land.
 //
 // KV-stationary persistent CTAs, one per SM.  A work item is (batch, KV head,

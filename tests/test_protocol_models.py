@@ -13,8 +13,9 @@ Not among them: dropping the MMA warp's wait for the accumulator's release
 read the accumulator out also produce the next item's first P or dS, so the
 MMA warp's wait for that operand already orders the accumulator's reuse; the
 model finds those waits redundant here.  They are kept so that the release
-stays explicit, and they become necessary as soon as a separate warpgroup reads
-the accumulators out.
+stays explicit.  The fused backward's dQ is the exception: a separate warpgroup
+reads it out, so there the wait for its release is necessary, and dropping it is
+one of the planted mistakes below.
 """
 import os
 import random
