@@ -63,7 +63,7 @@ constexpr int kDoStages = 1;  // dO tiles: last read by dV(t); dO(t+1) is needed
 // Registers per thread after the per-warpgroup split (setmaxnreg): compute,
 // dQ read-out, and the producer/MMA warpgroup.  The block is launched with
 // 128 per thread; the shares must not add up to more than that total.
-constexpr int kRegCompute = 168, kRegDrain = 56, kRegControl = 120;
+constexpr int kRegCompute = 160, kRegDrain = 72, kRegControl = 120;
 static_assert(2 * 128 * kRegCompute + 128 * kRegDrain + 128 * kRegControl <= kThreads * 128,
               "the register split must fit the launch's registers");
 constexpr int kLStages = 2;   // LSE2 / D rows: last read by the compute warps
@@ -401,19 +401,25 @@ __global__ void __launch_bounds__(fb::kThreads, 1)
         if (!__all_sync(0xffffffffu, mbar_wait(&s.dq_full, tc & 1, w))) return false;
         tc_fence_after();
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t r[32];
-          tmem_ld32x(tb + kColDQ + c * 32, r);
+        for (int cp = 0; cp < D / 64; ++cp) {  // 64 columns (two loads in flight) at a time
+          uint32_t r[64];
+          tmem_ld32x(tb + kColDQ + cp * 64, r);
+          tmem_ld32x(tb + kColDQ + cp * 64 + 32, r + 32);
           tmem_ld_wait();
-          if (c == D / 32 - 1) {  // every column read: the region may take dP^T(t+1)
+          if (cp == D / 64 - 1) {  // every column read: the region may take dP^T(t+1)
             tc_fence_before();
             mbar_arrive(&s.dq_free);
           }
-          float4* dst = (c < D / 64) ? lo + c * 8 * kTile : hi + (c - D / 64) * 8 * kTile;
 #pragma unroll
-          for (int c4 = 0; c4 < 8; ++c4)
-            dst[c4 * kTile + jl] = make_float4(__uint_as_float(r[4 * c4]), __uint_as_float(r[4 * c4 + 1]),
-                                               __uint_as_float(r[4 * c4 + 2]), __uint_as_float(r[4 * c4 + 3]));
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int c = 2 * cp + h2;
+            float4* dst = (c < D / 64) ? lo + c * 8 * kTile : hi + (c - D / 64) * 8 * kTile;
+#pragma unroll
+            for (int c4 = 0; c4 < 8; ++c4)
+              dst[c4 * kTile + jl] =
+                  make_float4(__uint_as_float(r[32 * h2 + 4 * c4]), __uint_as_float(r[32 * h2 + 4 * c4 + 1]),
+                              __uint_as_float(r[32 * h2 + 4 * c4 + 2]), __uint_as_float(r[32 * h2 + 4 * c4 + 3]));
+          }
         }
         fence_async_smem();
         mbar_arrive(&s.staged);
