@@ -22,6 +22,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import platform
 import socket
 import json
@@ -180,8 +181,12 @@ def effective_flops(pairs: int, d: int):
 
 
 def kernel_source_hash(name: str) -> str:
-    with open(os.path.join(ROOT, "column_sparse_masked_b200", "csrc", name), "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    """sha256[:16] of a kernel source's code: the file with `//` comments, trailing blanks and
+    empty lines removed, so that a comment edit keeps the recorded counters valid."""
+    with open(os.path.join(ROOT, "column_sparse_masked_b200", "csrc", name), encoding="utf-8") as f:
+        lines = [re.sub(r"//.*$", "", ln).rstrip() for ln in f]
+    code = "\n".join(ln for ln in lines if ln)
+    return hashlib.sha256(code.encode()).hexdigest()[:16]
 
 
 def recorded_traffic(kernel_file: str, workload: str):

@@ -371,8 +371,9 @@ __global__ void __launch_bounds__(fb::kThreads, 1)
     // ---------------- dQ read-out warpgroup: thread = query row (TMEM lane) ----------------
     // Copies dQ(t) from TMEM into shared memory in the accumulator tile's
     // layout (columns 0-63 into the dS buffer, which dQ(t) has finished
-    // reading, 64-127 into the staging buffer), frees the TMEM region after
-    // the last 32 columns (dP^T(t+1) may then be issued), and has one thread
+    // reading, 64-127 into the staging buffer), 64 columns (two loads) at a
+    // time, frees the TMEM region once the last load has completed
+    // (dP^T(t+1) may then be issued), and has one thread
     // hand both halves to the TMA unit as asynchronous bulk fp32 reductions
     // into [B, Hq, nQt, D/4, 128, 4].  Only that thread waits on the L2's
     // reduction rate (about 20 bytes per clock per SM when every SM reduces):
