@@ -44,7 +44,7 @@ METRIC = "FlashMask fwd+bwd effective TFLOP/s (unmasked FLOPs only), % of B200 b
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 CPU_SAMPLE_ROWS = 8192  # bounded oracle sample: first rows/keys of (batch 0, q-head 0)
 DEFAULT_CONFIG = "docblocksparse128k"
-SECONDARY = ("doc8k", "sharequestion32k")
+SECONDARY = ("doc8k", "sharequestion32k", "prefixwindow64k")
 SECONDARY_STEPS = 30
 
 
@@ -524,7 +524,7 @@ def run_ours(args, rank, world, local_rank):
     cpu_inp = pb["inp"]
     del pb
 
-    # ---- the other document / share-question workloads, same run (not the headline) ----
+    # ---- the other workloads (document, share-question, prefix + window), same run (not the headline) ----
     if not args.no_secondary:
         sec = {}
         for name in SECONDARY:
