@@ -460,9 +460,8 @@ __global__ void __launch_bounds__(qb::kThreads, 1)
         for (int i = 0; i < 16; ++i)
           pk2[i] = pack_bf16x2(__uint_as_float(rr[2 * i]) * p.scale, __uint_as_float(rr[2 * i + 1]) * p.scale);
         if (valid) {
-          uint4* d4 = reinterpret_cast<uint4*>(dqrow + c * 32);
 #pragma unroll
-          for (int i = 0; i < 4; ++i) d4[i] = make_uint4(pk2[4 * i], pk2[4 * i + 1], pk2[4 * i + 2], pk2[4 * i + 3]);
+          for (int i = 0; i < 4; ++i) st_global_v4_na(dqrow + c * 32 + i * 8, pk2[4 * i], pk2[4 * i + 1], pk2[4 * i + 2], pk2[4 * i + 3]);
         }
       }
       tc_fence_before();

@@ -462,11 +462,10 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
         if (valid) {
           if (o_v8) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) st_global_v8(orow + c * 64 + i * 16, pkd + 8 * i);
+            for (int i = 0; i < 4; ++i) st_global_v8_na(orow + c * 64 + i * 16, pkd + 8 * i);
           } else {
-            uint4* dst = reinterpret_cast<uint4*>(orow + c * 64);
 #pragma unroll
-            for (int i = 0; i < 8; ++i) dst[i] = make_uint4(pkd[4 * i], pkd[4 * i + 1], pkd[4 * i + 2], pkd[4 * i + 3]);
+            for (int i = 0; i < 8; ++i) st_global_v4_na(orow + c * 64 + i * 8, pkd[4 * i], pkd[4 * i + 1], pkd[4 * i + 2], pkd[4 * i + 3]);
           }
         }
       }

@@ -333,6 +333,20 @@ __device__ __forceinline__ void st_global_v8(void* p, const uint32_t* v) {
                : "memory");
 }
 
+// Output stores that do not allocate in L1: rows the SM writes once and never
+// reads back would otherwise take L1 lines (the L1 shares its storage with
+// shared memory) from data that is re-read.
+__device__ __forceinline__ void st_global_v8_na(void* p, const uint32_t* v) {
+  asm volatile("st.global.L1::no_allocate.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(v[0]),
+               "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+               : "memory");
+}
+
+__device__ __forceinline__ void st_global_v4_na(void* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.global.L1::no_allocate.v4.b32 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(a), "r"(b), "r"(c), "r"(d)
+               : "memory");
+}
+
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
