@@ -36,7 +36,9 @@ from ._binding import (  # noqa: F401
     profiler_enable,
     profiler_read,
     get_bwd_mode,
+    get_fwd_pairing,
     set_bwd_mode,
+    set_fwd_pairing,
     set_max_ctas,
     set_wait_limit_ns,
     test_wait_timeout,
@@ -47,6 +49,6 @@ from ._binding import (  # noqa: F401
 
 __all__ = [
     "FlashMaskError", "balance_chunks", "classify", "count_unmasked", "flashmask_attention", "fwd", "bwd", "get_status", "get_timeout_info",
-    "launch_count", "lib_path", "load_library", "localize", "localize_multi", "merge_partials", "profiler_enable", "profiler_read", "get_bwd_mode", "set_bwd_mode", "set_max_ctas", "set_wait_limit_ns", "test_wait_timeout", "tile_costs",
+    "launch_count", "lib_path", "load_library", "localize", "localize_multi", "merge_partials", "profiler_enable", "profiler_read", "get_bwd_mode", "set_bwd_mode", "get_fwd_pairing", "set_fwd_pairing", "set_max_ctas", "set_wait_limit_ns", "test_wait_timeout", "tile_costs",
     "version", "workspace_size",
 ]

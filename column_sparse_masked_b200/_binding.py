@@ -31,6 +31,8 @@ _SIGS = {
     "flashmask_set_max_ctas": (ctypes.c_int, [ctypes.c_int32]),
     "flashmask_set_bwd_mode": (ctypes.c_int, [ctypes.c_int32]),
     "flashmask_get_bwd_mode": (ctypes.c_int, []),
+    "flashmask_set_fwd_pairing": (ctypes.c_int, [ctypes.c_int32]),
+    "flashmask_get_fwd_pairing": (ctypes.c_int, []),
     "flashmask_get_timeout_info": (ctypes.c_int, [_P]),
     "flashmask_get_status": (ctypes.c_int, []),
     "flashmask_set_wait_limit_ns": (None, [ctypes.c_int64]),
@@ -346,6 +348,17 @@ def set_bwd_mode(mode) -> None:
 def get_bwd_mode() -> str:
     m = int(load_library().flashmask_get_bwd_mode())
     return {v: k for k, v in _BWD_MODES.items()}[m]
+
+
+def set_fwd_pairing(on: bool) -> None:
+    """Forward items of later ``fwd`` calls: one q-tile of two q-heads that share a KV head (True,
+    the default; used when the shape has one mask head and an even GQA group) or two q-tiles of one
+    q-head (False).  Outputs are bit-identical either way."""
+    _check(load_library().flashmask_set_fwd_pairing(1 if on else 0), "flashmask_set_fwd_pairing")
+
+
+def get_fwd_pairing() -> bool:
+    return bool(load_library().flashmask_get_fwd_pairing())
 
 
 def balance_chunks(costs: Sequence[int], parts: int) -> Tuple[List[int], int]:

@@ -52,23 +52,37 @@ struct Shape {
   int G;      // q-heads per KV head
   int nQt;    // q-tiles
   int nKt;    // k-tiles
-  int nQB;    // forward blocks of two q-tiles
+  int nQB;    // blocks of two q-tiles (the query-side lists of the backward)
+  // Forward items take two 128-row q-tiles of one q-head (a block of two
+  // q-tiles) or, with `fpair`, one q-tile of two q-heads that share a KV head
+  // and a mask (GQA with one mask head): both halves then see exactly the
+  // same key tiles, so no tile is computed for a q-tile that skips it.
+  int fpair;  // forward items pair two q-heads
+  int nFB;    // forward blocks: nQB, or nQt with fpair
+  int fG;     // forward items per (b, KV head, block): G, or G/2 with fpair
   // Work items of the three attention kernels, indexed group-major: a group
   // is one (batch, KV head), i.e. the data one L2-resident working set shares.
-  //   forward   (b, hkv, q-block, q-head in group): B*Hq*nQB items
-  //   key side  (b, hkv, k-tile):                   B*Hkv*nKt items
-  //   query side(b, hkv, q-tile, q-head in group):  B*Hq*nQt items
+  //   forward   (b, hkv, block, q-head (pair) in group): B*Hkv*fG*nFB items
+  //   key side  (b, hkv, k-tile):                         B*Hkv*nKt items
+  //   query side(b, hkv, q-tile, q-head in group):        B*Hq*nQt items
   int64_t n_fwd_items, n_kv_items, n_q_items;
 };
 
-inline Shape make_shape(int B, int Hq, int Hkv, int Hm, int Nq, int Nk, int d) {
+// Forward items pair q-heads when the shape allows it: one mask head and an
+// even number of q-heads per KV head.
+inline bool fwd_pairing_possible(int Hq, int Hkv, int Hm) { return Hm == 1 && (Hq / Hkv) % 2 == 0; }
+
+inline Shape make_shape(int B, int Hq, int Hkv, int Hm, int Nq, int Nk, int d, bool fpair = false) {
   Shape s{};
   s.B = B; s.Hq = Hq; s.Hkv = Hkv; s.Hm = Hm; s.Nq = Nq; s.Nk = Nk; s.d = d;
   s.G = Hq / Hkv;
   s.nQt = (Nq + kTile - 1) / kTile;
   s.nKt = (Nk + kTile - 1) / kTile;
   s.nQB = (s.nQt + 1) / 2;
-  s.n_fwd_items = (int64_t)B * Hq * s.nQB;
+  s.fpair = (fpair && fwd_pairing_possible(Hq, Hkv, Hm)) ? 1 : 0;
+  s.nFB = s.fpair ? s.nQt : s.nQB;
+  s.fG = s.fpair ? s.G / 2 : s.G;
+  s.n_fwd_items = (int64_t)B * Hkv * s.fG * s.nFB;
   s.n_kv_items = (int64_t)B * Hkv * s.nKt;
   s.n_q_items = (int64_t)B * Hq * s.nQt;
   return s;
@@ -98,9 +112,9 @@ inline WsLayout make_layout(const Shape& s) {
   const size_t bhm = (size_t)s.B * s.Hm;
   L.rec = take(bhm * s.nKt * kTile * 16);
   L.ksum = take(bhm * s.nKt * 8 * 4);
-  L.fcount = take(bhm * s.nQB * 4);
-  L.flist = take(bhm * s.nQB * s.nKt * 4);
-  L.qcount = take(bhm * s.nQB * 2 * 4);
+  L.fcount = take(bhm * s.nFB * 4);
+  L.flist = take(bhm * s.nFB * s.nKt * 4);
+  L.qcount = take(bhm * s.nFB * 2 * 4);
   L.forder = take((size_t)s.n_fwd_items * 4);
   L.counters = take(64);
   L.fwd_bytes = off;
@@ -116,12 +130,12 @@ inline WsLayout make_layout(const Shape& s) {
 }
 
 struct ItemCoord {
-  int b, hkv, t, hg;  // t = q-block, k-tile or q-tile; hg = q-head within the GQA group
+  int b, hkv, t, hg;  // t = forward block, k-tile or q-tile; hg = q-head (pair) within the GQA group
 };
 __host__ __device__ __forceinline__ ItemCoord decode_fwd_item(const Shape& s, int i) {
   ItemCoord c;
-  c.hg = i % s.G; i /= s.G;
-  c.t = i % s.nQB; i /= s.nQB;
+  c.hg = i % s.fG; i /= s.fG;
+  c.t = i % s.nFB; i /= s.nFB;
   c.hkv = i % s.Hkv; c.b = i / s.Hkv;
   return c;
 }
@@ -155,8 +169,8 @@ struct MaskPrepParams {
 struct PlanParams {
   Shape s;
   const int* ksum;
-  int* fcount; int* flist;   // forward lists  [B, Hm, nQB] / [B, Hm, nQB, nKt]
-  int* qcount;               // per q-tile non-skipped k-tiles [B, Hm, nQB*2]
+  int* fcount; int* flist;   // forward lists  [B, Hm, nFB] / [B, Hm, nFB, nKt]
+  int* qcount;               // per block slot non-skipped k-tiles [B, Hm, nFB*2]
   int* bcount; int* blist;   // backward lists [B, Hm, nKt] / [B, Hm, nKt, nQt]
   uint8_t* cls;              // optional export [B, Hm, nQt, nKt]
 };

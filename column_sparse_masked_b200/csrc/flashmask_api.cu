@@ -34,6 +34,7 @@ namespace {
 std::atomic<int64_t> g_wait_limit_ns{2000000000LL};
 std::atomic<int> g_max_ctas{0};  // 0: one persistent CTA per SM
 std::atomic<int> g_bwd_mode{FLASHMASK_BWD_FUSED};
+std::atomic<int> g_fwd_pairing{1};
 
 // Persistent grid of an attention kernel: one CTA per SM, at most one per
 // work item, at most the process-wide cap when one is set.
@@ -320,7 +321,9 @@ extern "C" {
 
 size_t flashmask_fwd_workspace_size(const flashmask_dims* d) {
   if (check_dims(d) != FLASHMASK_OK) return 0;
-  return make_layout(make_shape(d->B, d->Hq, d->Hkv, d->Hm, d->Nq, d->Nk, d->d)).fwd_bytes;
+  // sized for paired q-heads whenever the shape allows them (the larger
+  // layout), so the size holds whichever item kind a call uses
+  return make_layout(make_shape(d->B, d->Hq, d->Hkv, d->Hm, d->Nq, d->Nk, d->d, true)).fwd_bytes;
 }
 
 size_t flashmask_bwd_workspace_size(const flashmask_dims* d) {
@@ -335,7 +338,7 @@ int flashmask_fwd(const void* q, const void* k, const void* v, const int32_t* lt
   FM_TRY(check_dims(dims));
   FM_TRY(check_masks(lts, lte, uts, ute));
   const flashmask_dims& d = *dims;
-  const Shape s = make_shape(d.B, d.Hq, d.Hkv, d.Hm, d.Nq, d.Nk, d.d);
+  const Shape s = make_shape(d.B, d.Hq, d.Hkv, d.Hm, d.Nq, d.Nk, d.d, g_fwd_pairing.load() != 0);
   if ((int64_t)s.B * s.Nq == 0) return FLASHMASK_OK;
   if (!q || !o || !lse || (s.Nk > 0 && (!k || !v))) return FLASHMASK_ERR_INVALID_ARG;
   for (const void* p : {q, k, v, (const void*)o, (const void*)lse})
@@ -374,7 +377,7 @@ int flashmask_fwd(const void* q, const void* k, const void* v, const int32_t* lt
   sp.order = reinterpret_cast<int*>(ws + L.forder);
   sp.counter = reinterpret_cast<int*>(ws + L.counters);
   sp.n_items = (int)s.n_fwd_items;
-  sp.items_per_group = s.nQB * s.G;
+  sp.items_per_group = s.nFB * s.fG;
   sp.wave = wave_groups((size_t)s.Nk * s.d * 2 * 2, s.B * s.Hkv, s.n_fwd_items, di.sm_count);
   finish_sort_params(sp);
   FM_CUDA(launch_sort_units(&sp, 1, st));
@@ -731,6 +734,14 @@ int flashmask_set_bwd_mode(int32_t mode) {
 }
 
 int flashmask_get_bwd_mode(void) { return g_bwd_mode.load(); }
+
+int flashmask_set_fwd_pairing(int32_t on) {
+  if (on != 0 && on != 1) return FLASHMASK_ERR_INVALID_ARG;
+  g_fwd_pairing.store(on);
+  return FLASHMASK_OK;
+}
+
+int flashmask_get_fwd_pairing(void) { return g_fwd_pairing.load(); }
 
 int flashmask_set_max_ctas(int32_t n) {
   if (n < 0) return FLASHMASK_ERR_INVALID_ARG;

@@ -7,7 +7,9 @@
 // (TMA/WGMMA with three warp roles); this one is written for Blackwell:
 //
 //   * persistent CTAs (one per SM) take work items -- (batch, q-head, block of
-//     two 128-row q-tiles) -- from a locality-aware longest-first order through
+//     two 128-row q-tiles), or, when two q-heads share a KV head and the mask,
+//     (batch, pair of q-heads, one q-tile), so that both halves see exactly
+//     the same key tiles -- from a locality-aware longest-first order through
 //     an atomic counter; the producer warp hands each item to the other roles
 //     through a ring of mbarriers, so consecutive items overlap (the next
 //     item's Q load and first QK^T run while the softmax warps write O);
@@ -59,8 +61,14 @@ struct __align__(16) FwdItem {
   int item, b, h, hm, hkv, qb, n, e0;  // e0: first entry of the item's tile list
   __device__ __forceinline__ const int* list(const FwdParams& p) const {
     const Shape& sh = p.s;
-    return p.flist + (((size_t)b * sh.Hm + hm) * sh.nQB + qb) * sh.nKt;
+    return p.flist + (((size_t)b * sh.Hm + hm) * sh.nFB + qb) * sh.nKt;
   }
+  // first query row and q-head of half g: two q-tiles of head h, or (paired
+  // q-heads) one q-tile of heads h and h + 1
+  __device__ __forceinline__ int row0(const Shape& sh, int g) const {
+    return sh.fpair ? qb * kTile : qb * 2 * kTile + g * kTile;
+  }
+  __device__ __forceinline__ int head(const Shape& sh, int g) const { return sh.fpair ? h + g : h; }
 };
 
 __device__ __forceinline__ FwdItem decode_fwd(const FwdParams& p, int item) {
@@ -78,9 +86,9 @@ __device__ __forceinline__ FwdItem decode_fwd(const FwdParams& p, int item) {
   it.b = c.b;
   it.qb = c.t;
   it.hkv = c.hkv;
-  it.h = c.hkv * sh.G + c.hg;
-  it.hm = (sh.Hm == 1) ? 0 : it.h;
-  const size_t lrow = ((size_t)it.b * sh.Hm + it.hm) * sh.nQB + it.qb;
+  it.h = c.hkv * sh.G + (sh.fpair ? 2 * c.hg : c.hg);
+  it.hm = (sh.Hm == 1) ? 0 : it.h;  // paired q-heads share mask head 0
+  const size_t lrow = ((size_t)it.b * sh.Hm + it.hm) * sh.nFB + it.qb;
   it.n = p.fcount[lrow];
   if (kChecks) {  // the k-tile list: a count within [0, nKt], entries in range
     bool bad = it.n < 0 || it.n > sh.nKt;
@@ -219,7 +227,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
           for (int g = 0; g < 2; ++g)
 #pragma unroll
             for (int bx = 0; bx < Cfg::kBoxes; ++bx)
-              tma_prefetch_l2_4d(&tq, bx * 64, out.h, out.qb * 256 + g * kTile, out.b);
+              tma_prefetch_l2_4d(&tq, bx * 64, out.head(sh, g), out.row0(sh, g), out.b);
         }
         return true;
       };
@@ -238,7 +246,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
         for (int g = 0; g < 2; ++g)
 #pragma unroll
           for (int bx = 0; bx < Cfg::kBoxes; ++bx)
-            tma_load_4d(s.q[g] + bx * 16384, &tq, &s.q_full, bx * 64, it.h, it.qb * 256 + g * kTile, it.b);
+            tma_load_4d(s.q[g] + bx * 16384, &tq, &s.q_full, bx * 64, it.head(sh, g), it.row0(sh, g), it.b);
         ++act;
         for (int t = 0; t < it.n && ok; ++t) {
           const int kt = (t == 0 ? it.e0 : list[t]) >> 8;
@@ -340,7 +348,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
     while (ok && it.item < p.n_items) {
       const int n = it.n;
       const int* list = it.list(p);
-      const int rbase = it.qb * 256 + g * kTile + wq * 32;  // first row of this warp
+      const int rbase = it.row0(sh, g) + wq * 32;  // first row of this warp
       const int row = rbase + lane;
       const int4* recs = p.rec + ((size_t)it.b * sh.Hm + it.hm) * sh.nKt * kTile;
       float m_run = -INFINITY, l_run = 0.f;  // m_run in scaled log2 units
@@ -443,7 +451,8 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
       tc_fence_after();
       const bool valid = row < sh.Nq;
       const float inv_l = (l_run > 0.f) ? 1.f / l_run : 0.f;
-      __nv_bfloat16* orow = p.o + (((size_t)cur.b * sh.Nq + (valid ? row : 0)) * sh.Hq + cur.h) * D;
+      const int hg_out = cur.head(sh, g);
+      __nv_bfloat16* orow = p.o + (((size_t)cur.b * sh.Nq + (valid ? row : 0)) * sh.Hq + hg_out) * D;
 #pragma unroll
       for (int c = 0; c < D / 64; ++c) {
         uint32_t o[64];
@@ -475,7 +484,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::kThreads, 1)
         ++act;
       }
       if (valid)
-        p.lse[((size_t)cur.b * sh.Hq + cur.h) * sh.Nq + row] =
+        p.lse[((size_t)cur.b * sh.Hq + hg_out) * sh.Nq + row] =
             (l_run > 0.f) ? (m_run + log2f(l_run)) * 0.69314718055994531f : -INFINITY;
     }
   }

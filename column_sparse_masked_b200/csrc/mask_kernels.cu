@@ -87,17 +87,18 @@ __device__ __forceinline__ int block_compact128(bool flag, int* warp_tot, int* t
 
 // ----------------------------------------------------------------------------
 // 2a. forward work lists: per (b, hm, block of two q-tiles) the k-tiles that
-//     are not skipped for at least one of the two q-tiles, in increasing order
+//     are not skipped for at least one of the two q-tiles, in increasing order;
+//     with paired q-heads a block is one q-tile, whose class both halves share
 // ----------------------------------------------------------------------------
 __device__ void plan_fwd_body(const PlanParams& p, int qb) {
   const Shape& s = p.s;
   const int hm = blockIdx.y, b = blockIdx.z;
   const size_t row = (size_t)b * s.Hm + hm;
-  const int qt0 = 2 * qb, qt1 = 2 * qb + 1;
+  const int qt0 = s.fpair ? qb : 2 * qb, qt1 = s.fpair ? qb : 2 * qb + 1;
   const int r00 = qt0 * kTile, r01 = min(r00 + kTile, s.Nq);
   const int r10 = qt1 * kTile, r11 = min(r10 + kTile, s.Nq);
   const bool ragged_k = (s.Nk % kTile) != 0;
-  int* list = p.flist + (row * s.nQB + qb) * s.nKt;
+  int* list = p.flist + (row * s.nFB + qb) * s.nKt;
   __shared__ int warp_tot[4];
   __shared__ int total;
   __shared__ int qc[2];
@@ -113,7 +114,8 @@ __device__ void plan_fwd_body(const PlanParams& p, int qb) {
 #pragma unroll
       for (int e = 0; e < 8; ++e) sm[e] = src[e];
       c0 = classify_tile(sm, r00, r01);
-      if (qt1 < s.nQt) c1 = classify_tile(sm, r10, r11);
+      if (s.fpair) c1 = c0;
+      else if (qt1 < s.nQt) c1 = classify_tile(sm, r10, r11);
     }
     const bool keep = (c0 != kClsSkip) || (c1 != kClsSkip);
     const unsigned b0 = __ballot_sync(0xffffffffu, c0 != kClsSkip);
@@ -127,8 +129,8 @@ __device__ void plan_fwd_body(const PlanParams& p, int qb) {
     count += total;
     __syncthreads();
   }
-  if (threadIdx.x == 0) p.fcount[row * s.nQB + qb] = count;
-  if (threadIdx.x < 2) p.qcount[(row * s.nQB + qb) * 2 + threadIdx.x] = qc[threadIdx.x];
+  if (threadIdx.x == 0) p.fcount[row * s.nFB + qb] = count;
+  if (threadIdx.x < 2) p.qcount[(row * s.nFB + qb) * 2 + threadIdx.x] = qc[threadIdx.x];
 }
 
 // ----------------------------------------------------------------------------
@@ -219,8 +221,8 @@ __device__ __forceinline__ unsigned item_cost(const SortParams& p, int i) {
   const Shape& s = p.s;
   if (p.mode == 0) {
     const ItemCoord c = decode_fwd_item(s, i);
-    const int h = c.hkv * s.G + c.hg, hm = (s.Hm == 1) ? 0 : h;
-    return (unsigned)p.count[((size_t)c.b * s.Hm + hm) * s.nQB + c.t];
+    const int h = c.hkv * s.G + (s.fpair ? 2 * c.hg : c.hg), hm = (s.Hm == 1) ? 0 : h;
+    return (unsigned)p.count[((size_t)c.b * s.Hm + hm) * s.nFB + c.t];
   }
   if (p.mode == 1) {
     const ItemCoord c = decode_kv_item_coord(s, i);
@@ -463,8 +465,8 @@ cudaError_t launch_mask_prep(const MaskPrepParams& p, cudaStream_t st) {
 }
 
 cudaError_t launch_plan_fwd(const PlanParams& p, cudaStream_t st) {
-  if (p.s.B == 0 || p.s.nQB == 0) return cudaSuccess;
-  return launch_after(plan_fwd_kernel, dim3(p.s.nQB, p.s.Hm, p.s.B), dim3(128), 0, st, p);
+  if (p.s.B == 0 || p.s.nFB == 0) return cudaSuccess;
+  return launch_after(plan_fwd_kernel, dim3(p.s.nFB, p.s.Hm, p.s.B), dim3(128), 0, st, p);
 }
 
 cudaError_t launch_plan_both(const PlanParams& p, cudaStream_t st) {

@@ -77,7 +77,8 @@ typedef struct flashmask_dims {
 } flashmask_dims;
 
 /* Bytes of workspace flashmask_fwd needs for `dims` (mask summary, padded
- * boundary records, per-tile work lists, scheduler order). */
+ * boundary records, per-tile work lists, scheduler order), whichever forward
+ * item kind (flashmask_set_fwd_pairing) the call uses. */
 size_t flashmask_fwd_workspace_size(const flashmask_dims* dims);
 
 /*
@@ -268,6 +269,18 @@ int flashmask_balance_chunks(const int64_t* costs, int32_t n, int32_t parts, int
  * for any other value.  flashmask_get_bwd_mode returns the current one. */
 int flashmask_set_bwd_mode(int32_t mode);
 int flashmask_get_bwd_mode(void);
+
+/* Forward work items (process-wide, for every later forward call).  With
+ * on = 1 (the default) and a shape with one mask head and an even number of
+ * q-heads per KV head, an item is one 128-row q-tile of two q-heads that share
+ * a KV head: both halves see the same key tiles, so no tile is computed for a
+ * half that skips it.  Otherwise (on = 0, or any other shape) an item is two
+ * consecutive q-tiles of one q-head, which compute the union of their key
+ * tiles (the tiles one of them skips contribute exact zeros).  Outputs are
+ * bit-identical either way.  FLASHMASK_ERR_INVALID_ARG for values other than
+ * 0 and 1.  flashmask_get_fwd_pairing returns the current setting. */
+int flashmask_set_fwd_pairing(int32_t on);
+int flashmask_get_fwd_pairing(void);
 
 /* Synchronises the current device, returns its status word (0 or a negative
  * FLASHMASK_ERR_* code written by a kernel) and resets it to 0. */

@@ -71,6 +71,18 @@ def test_workspace_sizes(lib):
     assert lib.flashmask_fwd_workspace_size(ctypes.byref(_dims(d=96))) == 0
 
 
+def test_fwd_pairing_toggle_and_workspace(lib):
+    """Host-only: the pairing switch accepts 0 and 1, and the forward workspace size covers the
+    paired layout (one list per q-tile) whichever setting a later call uses."""
+    assert lib.flashmask_get_fwd_pairing() == 1
+    assert lib.flashmask_set_fwd_pairing(2) == -1
+    assert lib.flashmask_set_fwd_pairing(0) == 0 and lib.flashmask_get_fwd_pairing() == 0
+    f_off = lib.flashmask_fwd_workspace_size(ctypes.byref(_dims(Nq=4096, Nk=4096)))
+    assert lib.flashmask_set_fwd_pairing(1) == 0 and lib.flashmask_get_fwd_pairing() == 1
+    f_on = lib.flashmask_fwd_workspace_size(ctypes.byref(_dims(Nq=4096, Nk=4096)))
+    assert f_on == f_off > 0  # the size does not depend on the switch
+
+
 @pytest.mark.parametrize("kw,code", [
     (dict(d=96), -2), (dict(Hq=3, Hkv=2), -1), (dict(Hm=2), -1), (dict(Nq=-1), -1), (dict(Hkv=0), -1),
 ])

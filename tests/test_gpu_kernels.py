@@ -306,6 +306,60 @@ def test_fused_and_split_backward_agree(name):
     assert (err <= 1e-2 + 2.0 ** -7 * sq.float().abs()).all(), err.max().item()
 
 
+PAIR_CASES = [c for c in CASES if c[5] == 1 and (c[3] // c[4]) % 2 == 0] + [
+    (1, 1000, 1000, 8, 2, 1, 128, "doc", 21),   # two pairs per KV head
+    (1, 129, 129, 4, 1, 4, 128, "random", 22),  # one mask per head: pairing not possible
+]
+
+
+@pytest.mark.parametrize("case", PAIR_CASES, ids=_ids)
+def test_paired_forward_items_bit_identical(case):
+    """Forward items of one q-tile of two q-heads (the default where the shape allows) compute
+    exactly what items of two q-tiles of one q-head do: the tiles the latter add for a q-tile that
+    skips them contribute exact zeros, so O and LSE agree bit for bit, with 1 CTA and all SMs."""
+    q, k, v, do, masks = make_case(*case)
+    qg, kg, vg = cuda(q, k, v)
+    mg = cuda(*masks)
+    try:
+        for cap in (0, 1):
+            fm.set_max_ctas(cap)
+            fm.set_fwd_pairing(True)
+            o1, l1 = fm.fwd(qg, kg, vg, *mg)
+            fm.set_fwd_pairing(False)
+            o2, l2 = fm.fwd(qg, kg, vg, *mg)
+            torch.cuda.synchronize()
+            assert fm.get_status() == 0
+            assert torch.equal(o1, o2) and torch.equal(l1, l2), (case, cap)
+    finally:
+        fm.set_fwd_pairing(True)
+        fm.set_max_ctas(0)
+
+
+@pytest.mark.parametrize("name", ["doc8k", "docblocksparse128k"])
+def test_paired_forward_items_workloads(name):
+    """The same on the GQA workloads with one mask head."""
+    w = wl.CONFIGS[name]
+    d = {k: v.cuda() for k, v in wl.make_inputs(w, with_grad=False).items()}
+    m = [d[n] for n in ("lts", "lte", "uts", "ute")]
+    try:
+        fm.set_fwd_pairing(True)
+        o1, l1 = fm.fwd(d["q"], d["k"], d["v"], *m)
+        fm.set_fwd_pairing(False)
+        o2, l2 = fm.fwd(d["q"], d["k"], d["v"], *m)
+        torch.cuda.synchronize()
+    finally:
+        fm.set_fwd_pairing(True)
+    assert fm.get_status() == 0
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_fwd_pairing_setting():
+    assert fm.get_fwd_pairing() is True
+    fm.set_fwd_pairing(False)
+    assert fm.get_fwd_pairing() is False
+    fm.set_fwd_pairing(True)
+
+
 def test_bwd_mode_setting():
     assert fm.get_bwd_mode() == "fused"
     fm.set_bwd_mode("split")
